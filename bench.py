@@ -1,0 +1,377 @@
+#!/usr/bin/env python
+"""Benchmark: forward + backward frames/s of the tile rasterizer.
+
+Workload (default): 1M Gaussians, SH degree 3, 1920x1080, four camera poses
+per step; each pose runs the whole path through the C ABI -- cull (gates off),
+preprocess, bin/sort, rasterize forward, rasterize backward (2-D part and
+parameter part). Inputs are synthetic and resident in HBM before timing; the
+236 MB parameter set is larger than the 126 MB L2, so no flush is needed.
+
+Prints one JSON line on rank 0. Under torchrun (N > 1) each rank renders its
+own batch of poses with no collective on the data path (weak scaling); the
+time is the maximum over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fwd+bwd frames/s @1080p, 1M Gaussians SH3; blends/s; % of HBM/FP32 roofline"
+WORKLOAD_CONFIG = 2
+
+# Algorithmic fp32 operations per unit of work ("Roofline").
+OPS_EVAL = 21          # evaluate one (pixel, Gaussian) pair: quadratic form, exp2, alpha, test
+OPS_BLEND_FWD = 8      # blend it: weight, 3 colour FMAs, 1 - alpha, T update, T test
+OPS_BLEND_BWD = 45     # backward per blend: T recovery, 9 gradient terms, 3 colour updates, 9 sums
+FP32_LANES_PER_SM = 128
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle samples during the timed region."""
+
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU side
+def cpu_sample(scene, tile_stride=32, pose=0):
+    """Time the oracle on a bounded sample of one frame and scale to frames/s.
+
+    Sample: the full preprocess and bin/sort of one pose, forward and 2-D
+    backward over every `tile_stride`-th tile, and the full parameter-gradient
+    chain; the per-tile parts are scaled by (tiles / sampled tiles)."""
+    import oracle
+    cam = scene.cameras[pose]
+    t0 = time.perf_counter()
+    rec = oracle.preprocess(scene, cam)
+    t1 = time.perf_counter()
+    bins = oracle.bin_sort(rec, cam)
+    t2 = time.perf_counter()
+    TT = cam.tiles_x * cam.tiles_y
+    sub = np.arange(0, TT, tile_stride, dtype=np.int32)
+    oracle.raster_fwd(rec, bins, cam, scene.bg, tile_subset=sub)
+    t3 = time.perf_counter()
+    g = scene.grad_image(pose)
+    oracle.backward(scene, cam, rec, bins, g, params3d=True, tile_subset=sub)
+    t4 = time.perf_counter()
+    scale = TT / len(sub)
+    frame = (t1 - t0) + (t2 - t1) + (t3 - t2) * scale + (t4 - t3) * scale
+    return {"frame_s": frame, "sample_s": t4 - t0, "tiles_sampled": int(len(sub)), "tiles": int(TT),
+            "parts_s": {"preprocess": t1 - t0, "bin_sort": t2 - t1, "raster_fwd_sample": t3 - t2,
+                        "backward_sample": t4 - t3}}
+
+
+def run_reference(args):
+    """The oracle timed as it stands on this host's cores (reference arm)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from differentiable_tile_rasterizer_b200 import synthetic
+    scene = synthetic.make_config(WORKLOAD_CONFIG)
+    for _ in range(args.warmup):
+        cpu_sample(scene, tile_stride=args.ref_tile_stride)
+    frames = []
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        frames.append(cpu_sample(scene, tile_stride=args.ref_tile_stride, pose=s % len(scene.cameras))["frame_s"])
+    wall = time.perf_counter() - t0
+    ms = 1000.0 * float(np.mean(frames)) * len(scene.cameras)
+    value = 1000.0 * len(scene.cameras) / ms
+    sample = (f"per step: preprocess + bin/sort of 1 pose in full, forward and backward on every "
+              f"{args.ref_tile_stride}th tile, parameter gradients in full; scaled to a frame")
+    line = {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
+            "config": {"workload": scene.name, "gaussians": scene.N, "sh_degree": 3, "width": 1920,
+                       "height": 1080, "poses_per_step": len(scene.cameras)},
+            "cpu_baseline": {"value": value, "unit": "frames/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "wall_s": wall}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU side
+def run_ours(args):
+    import torch
+    from differentiable_tile_rasterizer_b200 import gs, synthetic
+    from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, Rasterizer
+
+    world, rank, local = _dist_setup()
+    gs.load(build_if_missing=False)
+    scene = synthetic.make_config(WORKLOAD_CONFIG)
+    poses = scene.cameras
+    cams = [gs.camera(c) for c in poses]
+    params = GaussianParams.from_scene(scene)
+    gimg = [torch.from_numpy(scene.grad_image(p)).cuda() for p in range(len(poses))]
+    W, H = poses[0].width, poses[0].height
+    R = Rasterizer(scene.N, scene.sh_degree, W, H, capacity=6 * scene.N)
+    bg = tuple(float(b) for b in scene.bg)
+
+    def step():
+        for p, c in enumerate(cams):
+            R.forward(params, c, bg)
+            R.backward(gimg[p])
+
+    # warm-up (also settles the instance capacity)
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    # work counts per pose (deterministic; measured outside the timed region)
+    counts = []
+    for p, c in enumerate(cams):
+        R.forward(params, c, bg)
+        counts.append(R.work_counts())
+    torch.cuda.synchronize()
+
+    # ---- timed region: whole steps, device-resident inputs
+    R.stage_events = {}
+    launches0 = gs.gs_debug_kernel_launches()
+    _barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record()
+        for _ in range(args.steps):
+            step()
+        ev1.record()
+        torch.cuda.synchronize()
+    _barrier(world)
+    launches = gs.gs_debug_kernel_launches() - launches0
+    elapsed_ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in R.stage_events.items()}
+    stage_n = {k: len(v) for k, v in R.stage_events.items()}
+    R.stage_events = None
+    frames = args.steps * len(poses) * world
+    value = 1000.0 * frames / elapsed_ms
+    ms_per_step = elapsed_ms / args.steps
+
+    # ---- roofline of the dominant kernel
+    peaks = _peaks()
+    clocks = clk.summary()
+    B = sum(c["B"] for c in counts)
+    E = sum(c["E"] for c in counts)
+    Eb = sum(c["E_bwd"] for c in counts)
+    per_kernel = {"raster_fwd": OPS_EVAL * E + OPS_BLEND_FWD * B,
+                  "raster_bwd": OPS_EVAL * Eb + OPS_BLEND_BWD * B}
+    dom = max(("raster_fwd", "raster_bwd", "preprocess", "preprocess_bwd"), key=lambda k: stage_ms.get(k, 0.0))
+    avg_ms = stage_ms[dom] / max(stage_n[dom], 1)
+    peak_alu = 148 * FP32_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12  # T fp32 op/s
+    if dom in per_kernel:
+        ops_per_launch = per_kernel[dom] / len(poses)
+        achieved = ops_per_launch / (avg_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
+                "frac": achieved / peak_alu, "traffic": None,
+                "peak_source": f"148 SMs x 128 fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz (fp32 ops, FMA = 1)",
+                "ops_per_launch": ops_per_launch, "avg_launch_ms": avg_ms}
+    else:
+        K = scene.K
+        nbytes = (11 + 3 * K) * 4 * scene.N + 64 * scene.N if dom == "preprocess" else \
+            ((11 + 3 * K) * 4 * 2 + 48 + 64) * scene.N
+        achieved = nbytes / (avg_ms * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "avg_launch_ms": avg_ms}
+    roof["peak_kind"] = peaks["source"]
+
+    line = {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": scene.name, "gaussians": scene.N, "sh_degree": scene.sh_degree,
+                       "width": W, "height": H, "poses_per_step": len(poses),
+                       "l2": "inputs larger than L2 (236 MB of parameters), no flush",
+                       "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+            "blends_per_s": 1000.0 * B * args.steps * world / elapsed_ms,
+            "evaluated_pairs_per_s": 1000.0 * E * args.steps * world / elapsed_ms,
+            "work_per_step": {"V": sum(c["V"] for c in counts), "I": sum(c["I"] for c in counts),
+                              "E": E, "E_bwd": Eb, "B": B},
+            "stages_ms_per_step": {k: v / args.steps for k, v in stage_ms.items()},
+            "roofline": roof, "gpu_launches": int(launches), "clocks": clocks}
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        line["e2e"] = e2e(args, scene, R, gimg, cams, bg, world)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        import oracle
+        cs = cpu_sample(scene, tile_stride=args.ref_tile_stride)
+        line["cpu_baseline"] = {"value": 1.0 / cs["frame_s"], "unit": "frames/s", "cores": oracle.num_threads(),
+                                "kind": "oracle",
+                                "sample": f"1 pose: preprocess and bin/sort in full, forward + backward on "
+                                          f"{cs['tiles_sampled']} of {cs['tiles']} tiles (scaled), parameter "
+                                          f"gradients in full; {cs['sample_s']:.1f} s of CPU time"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def e2e(args, scene, R, gimg, cams, bg, world):
+    """Same metric with pinned host buffers: each step copies the parameters
+    and the upstream image gradients in, and the images and parameter
+    gradients of every pose out."""
+    import torch
+    from differentiable_tile_rasterizer_b200.pipeline import GaussianParams
+    host = GaussianParams.empty_like_host(scene)
+    host_g = [g.cpu().pin_memory() for g in gimg]
+    dev = GaussianParams.from_scene(scene)
+    out_img = [torch.empty_like(R.image, device="cpu").pin_memory() for _ in cams]
+    out_grads = [{k: torch.empty_like(v, device="cpu").pin_memory() for k, v in R.grads.items()} for _ in cams]
+    dg = [torch.empty_like(g) for g in gimg]
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + sum(
+        t.numel() * t.element_size() for t in host_g)
+    d2h = sum(t.numel() * t.element_size() for t in out_img) + sum(
+        v.numel() * v.element_size() for o in out_grads for v in o.values())
+
+    def step():
+        for k in ("means", "log_scales", "quats", "opacity_logits", "sh"):
+            getattr(dev, k).copy_(host[k], non_blocking=True)
+        for p, c in enumerate(cams):
+            dg[p].copy_(host_g[p], non_blocking=True)
+            R.forward(dev, c, bg)
+            R.backward(dg[p])
+            out_img[p].copy_(R.image, non_blocking=True)
+            for k, v in R.grads.items():
+                out_grads[p][k].copy_(v, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    _barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(args.steps):
+        step()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
+    return {"value": 1000.0 * args.steps * len(cams) * world / ms, "unit": "frames/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms / args.steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--ref-tile-stride", type=int, default=32)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+// C ABI entry points of libgs.so: argument validation, workspace carving and
+// kernel launches. No entry point allocates device memory.
+
+#include <atomic>
+#include <cmath>
+
+#include "gs.h"
+#include "gs_internal.cuh"
+
+using namespace gs;
+
+namespace {
+
+int64_t g_stall_tile = -1;
+
+bool finite_f(float v) { return std::isfinite(v); }
+
+bool camera_ok(const gs_camera* c) {
+  if (!c) return false;
+  if (c->width < 1 || c->height < 1 || c->width > 65535 * 16 || c->height > 65535 * 16) return false;
+  for (int k = 0; k < 9; ++k)
+    if (!finite_f(c->R[k])) return false;
+  for (int k = 0; k < 3; ++k)
+    if (!finite_f(c->t[k]) || !finite_f(c->campos[k])) return false;
+  if (!finite_f(c->fx) || !finite_f(c->fy) || !finite_f(c->cx) || !finite_f(c->cy)) return false;
+  if (!finite_f(c->near_z) || c->near_z < 0.0f) return false;
+  return true;
+}
+
+bool records_ok(const gs_projected* r) {
+  return r && r->xyzo && r->conic && r->rgb && r->radius && r->rect && r->tiles_touched;
+}
+
+Records to_records(const gs_projected* r) {
+  Records o;
+  o.xyzo = reinterpret_cast<float4*>(r->xyzo);
+  o.conic = reinterpret_cast<float4*>(r->conic);
+  o.rgb = reinterpret_cast<float4*>(r->rgb);
+  o.radius = r->radius;
+  o.rect = reinterpret_cast<ushort4*>(r->rect);
+  o.tiles = r->tiles_touched;
+  return o;
+}
+
+bool params_ok(const float* means, const float* log_scales, const float* quats, const float* logits,
+               const float* sh, int64_t N) {
+  if (N < 0 || N >= (int64_t(1) << 31)) return false;
+  if (N == 0) return true;
+  return means && log_scales && quats && logits && sh;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? GS_OK : GS_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+GS_API int gs_version(void) { return 1; }
+
+GS_API const char* gs_status_string(int status) {
+  switch (status) {
+    case GS_OK: return "ok";
+    case GS_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case GS_ERR_CAPACITY: return "instance capacity exceeded";
+    case GS_ERR_CUDA: return "CUDA runtime error";
+    case GS_ERR_DEVICE_TIMEOUT: return "bounded device-side wait timed out";
+    case GS_ERR_UNSUPPORTED: return "unsupported argument value";
+    default: return "unknown status";
+  }
+}
+
+GS_API void gs_debug_set_stalled_sort_tile(int64_t tile) { g_stall_tile = tile < 0 ? -1 : tile; }
+
+GS_API int64_t gs_debug_kernel_launches(void) { return kernel_launches(); }
+
+GS_API int gs_cull(const float* means, const float* importance, int64_t N, const gs_camera* cam,
+                   float lod_dist, float importance_q, uint8_t* mask, int32_t* active_idx,
+                   int32_t* n_active, void* workspace, size_t* workspace_bytes, void* stream) {
+  if (!workspace_bytes || N < 0 || N >= (int64_t(1) << 31) || !camera_ok(cam)) return GS_ERR_INVALID_ARGUMENT;
+  if (!(importance_q >= 0.0f) || !(importance_q < 1.0f) || !std::isfinite(lod_dist))
+    return GS_ERR_INVALID_ARGUMENT;
+  const size_t need = cull_workspace_bytes(N);
+  if (!workspace) {
+    *workspace_bytes = need;
+    return GS_OK;
+  }
+  if (*workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GS_ERR_INVALID_ARGUMENT;
+  if (!n_active || (N > 0 && (!means || !mask || !active_idx))) return GS_ERR_INVALID_ARGUMENT;
+  if (importance_q > 0.0f && N > 0 && !importance) return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_cull(means, importance, N, make_devcam(*cam), lod_dist, importance_q, mask,
+                                 active_idx, n_active, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_preprocess(const float* means, const float* log_scales, const float* quats,
+                         const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                         const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
+                         const gs_projected* out, void* stream) {
+  if (sh_degree < 0) return GS_ERR_INVALID_ARGUMENT;
+  if (sh_degree > 3) return GS_ERR_UNSUPPORTED;
+  if (!params_ok(means, log_scales, quats, opacity_logits, sh, N) || !camera_ok(cam) || !records_ok(out))
+    return GS_ERR_INVALID_ARGUMENT;
+  Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};
+  return cuda_status(launch_preprocess(p, make_devcam(*cam), to_records(out), static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
+                       uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
+                       int64_t* n_instances, void* workspace, size_t* workspace_bytes, void* stream) {
+  if (!workspace_bytes || !camera_ok(cam) || n < 0 || n >= (int64_t(1) << 31) || capacity < 0 ||
+      capacity >= (int64_t(1) << 30))
+    return GS_ERR_INVALID_ARGUMENT;
+  const DevCam dc = make_devcam(*cam);
+  const BinSortPlan plan = binsort_plan(n, capacity, (int64_t)dc.TW * dc.TH);
+  if (!workspace) {
+    *workspace_bytes = plan.bytes;
+    return GS_OK;
+  }
+  if (*workspace_bytes < plan.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return GS_ERR_INVALID_ARGUMENT;
+  if (!records_ok(in) || !n_instances || !tile_ranges || (n > 0 && !offsets) ||
+      (capacity > 0 && (!keys || !vals)))
+    return GS_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Records rec = to_records(in);
+  cudaError_t e = launch_scan_tiles(rec.tiles, n, offsets, workspace, plan, s);
+  if (e != cudaSuccess) return GS_ERR_CUDA;
+  int64_t total = 0;
+  e = cudaMemcpyAsync(&total, binsort_total_ptr(workspace, plan), sizeof(int64_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return GS_ERR_CUDA;
+  *n_instances = total;
+  if (total > capacity) return GS_ERR_CAPACITY;
+  e = launch_emit_sort_ranges(rec, n, offsets, dc, total, keys, vals, tile_ranges, workspace, plan,
+                              g_stall_tile, s);
+  if (e != cudaSuccess) return GS_ERR_CUDA;
+  int32_t status = 0;
+  e = cudaMemcpyAsync(&status, binsort_status_ptr(workspace, plan), sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return GS_ERR_CUDA;
+  if (status != 0) {
+    // Leave every tile empty so that a raster call on these buffers reads nothing.
+    cudaMemsetAsync(tile_ranges, 0, (size_t)dc.TW * dc.TH * 2 * sizeof(uint32_t), s);
+    cudaStreamSynchronize(s);
+    return GS_ERR_DEVICE_TIMEOUT;
+  }
+  return GS_OK;
+}
+
+GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,
+                            const gs_camera* cam, const float* bg, float* image, float* final_T,
+                            int32_t* n_contrib, int32_t* last, void* stream) {
+  if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last)
+    return GS_ERR_INVALID_ARGUMENT;
+  const float b[3] = {bg[0], bg[1], bg[2]};
+  return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
+                                       n_contrib, last, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,
+                               const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                               const float* final_T, const int32_t* last, const float* dL_dimage,
+                               float* grad2d, void* stream) {
+  if (!records_ok(in) || !camera_ok(cam) || n_records < 0 || n_records >= (int64_t(1) << 31) || !tile_ranges ||
+      !bg || !final_T || !last || !dL_dimage || (n_records > 0 && !grad2d))
+    return GS_ERR_INVALID_ARGUMENT;
+  if (n_records == 0) return GS_OK;
+  const float b[3] = {bg[0], bg[1], bg[2]};
+  return cuda_status(launch_raster_bwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, final_T, last,
+                                       dL_dimage, reinterpret_cast<float4*>(grad2d), n_records,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const float* quats,
+                             const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                             const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
+                             const gs_camera* cam, const gs_projected* in, const float* grad2d,
+                             float* d_means, float* d_log_scales, float* d_quats, float* d_opacity_logits,
+                             float* d_sh, void* stream) {
+  if (sh_degree < 0) return GS_ERR_INVALID_ARGUMENT;
+  if (sh_degree > 3) return GS_ERR_UNSUPPORTED;
+  if (!params_ok(means, log_scales, quats, opacity_logits, sh, N) || !camera_ok(cam) || !records_ok(in))
+    return GS_ERR_INVALID_ARGUMENT;
+  if (active_idx && !mask) return GS_ERR_INVALID_ARGUMENT;
+  if (N > 0 && (!grad2d || !d_means || !d_log_scales || !d_quats || !d_opacity_logits || !d_sh))
+    return GS_ERR_INVALID_ARGUMENT;
+  Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};
+  Grads g{d_means, d_log_scales, d_quats, d_opacity_logits, d_sh};
+  return cuda_status(launch_preprocess_bwd(p, mask, make_devcam(*cam), to_records(in),
+                                           reinterpret_cast<const float4*>(grad2d), g,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const float* quats,
+                            const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                            const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
+                            const gs_camera* cam, const gs_projected* in, const uint32_t* vals,
+                            const uint32_t* tile_ranges, const float* bg, const float* final_T,
+                            const int32_t* last, const float* dL_dimage, float* grad2d, float* d_means,
+                            float* d_log_scales, float* d_quats, float* d_opacity_logits, float* d_sh,
+                            void* stream) {
+  if (sh_degree < 0) return GS_ERR_INVALID_ARGUMENT;
+  if (sh_degree > 3) return GS_ERR_UNSUPPORTED;
+  if (!params_ok(means, log_scales, quats, opacity_logits, sh, N) || !camera_ok(cam) || !records_ok(in))
+    return GS_ERR_INVALID_ARGUMENT;
+  if (!tile_ranges || !bg || !final_T || !last || !dL_dimage || (N > 0 && !grad2d)) return GS_ERR_INVALID_ARGUMENT;
+  if (active_idx && !mask) return GS_ERR_INVALID_ARGUMENT;
+  if (N > 0 && (!d_means || !d_log_scales || !d_quats || !d_opacity_logits || !d_sh)) return GS_ERR_INVALID_ARGUMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const DevCam dc = make_devcam(*cam);
+  const Records rec = to_records(in);
+  const float b[3] = {bg[0], bg[1], bg[2]};
+  if (N > 0) {
+    cudaError_t e = launch_raster_bwd(rec, vals, tile_ranges, dc, b, final_T, last, dL_dimage,
+                                      reinterpret_cast<float4*>(grad2d), N, s);
+    if (e != cudaSuccess) return GS_ERR_CUDA;
+  }
+  Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};
+  Grads g{d_means, d_log_scales, d_quats, d_opacity_logits, d_sh};
+  return cuda_status(launch_preprocess_bwd(p, mask, dc, rec, reinterpret_cast<const float4*>(grad2d), g, s));
+}
+
+}  // extern "C"
+
+namespace gs {
+namespace {
+std::atomic<int64_t> g_launches{0};
+}
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+int64_t kernel_launches() { return g_launches.load(std::memory_order_relaxed); }
+}  // namespace gs

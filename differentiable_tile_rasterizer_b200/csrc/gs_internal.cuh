@@ -1,0 +1,105 @@
+// Internal launch interface shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "gs.h"
+
+namespace gs {
+
+// Camera as passed by value to kernels.
+struct DevCam {
+  float W[9], t[3], campos[3];
+  float fx, fy, cx, cy, near_z;
+  int width, height, TW, TH;
+};
+
+inline DevCam make_devcam(const gs_camera& c) {
+  DevCam d;
+  for (int k = 0; k < 9; ++k) d.W[k] = c.R[k];
+  for (int k = 0; k < 3; ++k) d.t[k] = c.t[k];
+  for (int k = 0; k < 3; ++k) d.campos[k] = c.campos[k];
+  d.fx = c.fx; d.fy = c.fy; d.cx = c.cx; d.cy = c.cy; d.near_z = c.near_z;
+  d.width = c.width; d.height = c.height;
+  d.TW = (c.width + 15) / 16;
+  d.TH = (c.height + 15) / 16;
+  return d;
+}
+
+struct Params {
+  const float* means;
+  const float* log_scales;
+  const float* quats;
+  const float* logits;
+  const float* sh;
+  int64_t N;
+  int sh_degree;
+  const int32_t* active_idx;  // may be null
+  const int32_t* n_active;    // may be null
+};
+
+struct Records {
+  float4* xyzo;
+  float4* conic;
+  float4* rgb;
+  int32_t* radius;
+  ushort4* rect;
+  int32_t* tiles;
+};
+
+struct Grads {
+  float* d_means;
+  float* d_log_scales;
+  float* d_quats;
+  float* d_logits;
+  float* d_sh;
+};
+
+inline unsigned grid_for(int64_t n, int block) { return (unsigned)((n + block - 1) / block); }
+
+// Process-wide count of kernel launches (see gs_debug_kernel_launches).
+void count_launches(int n);
+int64_t kernel_launches();
+
+// preprocess.cu
+cudaError_t launch_preprocess(const Params& p, const DevCam& cam, const Records& out,
+                              cudaStream_t s);
+cudaError_t launch_preprocess_bwd(const Params& p, const uint8_t* mask, const DevCam& cam,
+                                  const Records& in, const float4* grad2d, const Grads& g,
+                                  cudaStream_t s);
+
+// cull.cu
+size_t cull_workspace_bytes(int64_t N);
+cudaError_t launch_cull(const float* means, const float* importance, int64_t N, const DevCam& cam,
+                        float lod_dist, float q, uint8_t* mask, int32_t* active_idx,
+                        int32_t* n_active, void* ws, cudaStream_t s);
+
+// binsort.cu
+struct BinSortPlan {
+  int64_t n, capacity, tiles;
+  int passes, tile_bits;
+  size_t bytes;
+};
+BinSortPlan binsort_plan(int64_t n, int64_t capacity, int64_t tiles);
+cudaError_t launch_scan_tiles(const int32_t* tiles, int64_t n, int32_t* offsets, void* ws,
+                              const BinSortPlan& plan, cudaStream_t s);
+const int64_t* binsort_total_ptr(void* ws, const BinSortPlan& plan);
+const int32_t* binsort_status_ptr(void* ws, const BinSortPlan& plan);
+cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const int32_t* offsets,
+                                    const DevCam& cam, int64_t n_inst, uint64_t* keys,
+                                    uint32_t* vals, uint32_t* ranges, void* ws,
+                                    const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s);
+
+// raster.cu
+cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
+                              const DevCam& cam, const float bg[3], float* image, float* final_T,
+                              int32_t* n_contrib, int32_t* last, cudaStream_t s);
+cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
+                              const DevCam& cam, const float bg[3], const float* final_T,
+                              const int32_t* last, const float* dL_dimage, float4* grad2d,
+                              int64_t n_records, cudaStream_t s);
+
+}  // namespace gs

@@ -1,0 +1,226 @@
+"""ctypes binding of libgs.so (include/gs.h), argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+CUDA tensors (or None where the C argument may be NULL) and raises GsError on
+a non-zero status. No computation happens in Python; there is no fallback:
+if the library is missing, loading raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import _build
+
+GS_OK = 0
+GS_ERR_INVALID_ARGUMENT = 1
+GS_ERR_CAPACITY = 2
+GS_ERR_CUDA = 3
+GS_ERR_DEVICE_TIMEOUT = 4
+GS_ERR_UNSUPPORTED = 5
+
+EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_bin_sort",
+            "gs_rasterize_fwd", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
+            "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches"]
+
+
+class GsError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: status {status} ({msg})")
+        self.status = status
+
+
+class GsCamera(ctypes.Structure):
+    _fields_ = [("R", ctypes.c_float * 9), ("t", ctypes.c_float * 3),
+                ("campos", ctypes.c_float * 3), ("fx", ctypes.c_float), ("fy", ctypes.c_float),
+                ("cx", ctypes.c_float), ("cy", ctypes.c_float), ("near_z", ctypes.c_float),
+                ("width", ctypes.c_int32), ("height", ctypes.c_int32)]
+
+
+class GsProjected(ctypes.Structure):
+    _fields_ = [("xyzo", ctypes.c_void_p), ("conic", ctypes.c_void_p), ("rgb", ctypes.c_void_p),
+                ("radius", ctypes.c_void_p), ("rect", ctypes.c_void_p),
+                ("tiles_touched", ctypes.c_void_p)]
+
+
+_LIB = None
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+PI64 = ctypes.POINTER(ctypes.c_int64)
+PSZ = ctypes.POINTER(ctypes.c_size_t)
+PCAM = ctypes.POINTER(GsCamera)
+PPROJ = ctypes.POINTER(GsProjected)
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libgs.so (building it first if it is absent and nvcc is available)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(_build.LIB):
+            if not build_if_missing:
+                raise OSError(f"libgs.so not built: {_build.LIB}")
+            _build.build()
+        L = ctypes.CDLL(_build.LIB)
+        L.gs_version.restype = ctypes.c_int
+        L.gs_status_string.restype = ctypes.c_char_p
+        L.gs_status_string.argtypes = [ctypes.c_int]
+        L.gs_cull.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P, PSZ, P]
+        L.gs_preprocess.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, PCAM, PPROJ, P]
+        L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
+        L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P]
+        L.gs_rasterize_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P, P, P,
+                                       P, P, P, P, P, P, P, P, P, P]
+        L.gs_preprocess_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P,
+                                        P, P, P, P, P, P]
+        L.gs_rasterize_bwd_2d.argtypes = [PPROJ, I64, P, P, PCAM, P, P, P, P, P, P]
+        L.gs_debug_kernel_launches.restype = ctypes.c_int64
+        L.gs_debug_kernel_launches.argtypes = []
+        L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
+        L.gs_debug_set_stalled_sort_tile.restype = None
+        for name in ["gs_cull", "gs_preprocess", "gs_bin_sort", "gs_rasterize_fwd",
+                     "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
+            getattr(L, name).restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def _check(fn: str, status: int):
+    if status != GS_OK:
+        raise GsError(fn, status, load().gs_status_string(status).decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def camera(cam) -> GsCamera:
+    """gs_camera from any object with R, t, campos, fx, fy, cx, cy, width, height, near_z."""
+    c = GsCamera()
+    R = [float(v) for v in torch.as_tensor(cam.R, dtype=torch.float32).reshape(9).tolist()]
+    c.R[:] = R
+    c.t[:] = [float(v) for v in torch.as_tensor(cam.t, dtype=torch.float32).reshape(3).tolist()]
+    c.campos[:] = [float(v) for v in torch.as_tensor(cam.campos, dtype=torch.float32).reshape(3).tolist()]
+    c.fx, c.fy, c.cx, c.cy = float(cam.fx), float(cam.fy), float(cam.cx), float(cam.cy)
+    c.near_z = float(cam.near_z)
+    c.width, c.height = int(cam.width), int(cam.height)
+    return c
+
+
+def projected(rec: dict) -> GsProjected:
+    """gs_projected from a dict of record tensors (see Records in pipeline.py)."""
+    return GsProjected(_p(rec["xyzo"]), _p(rec["conic"]), _p(rec["rgb"]), _p(rec["radius"]),
+                       _p(rec["rect"]), _p(rec["tiles"]))
+
+
+def version() -> int:
+    return load().gs_version()
+
+
+def gs_cull(means, importance, N, cam: GsCamera, lod_dist, importance_q, mask, active_idx,
+            n_active, workspace, stream=None):
+    nbytes = ctypes.c_size_t(0 if workspace is None else workspace.numel() * workspace.element_size())
+    _check("gs_cull", load().gs_cull(_p(means), _p(importance), int(N), ctypes.byref(cam),
+                                     float(lod_dist), float(importance_q), _p(mask), _p(active_idx),
+                                     _p(n_active), _p(workspace), ctypes.byref(nbytes), _stream(stream)))
+    return nbytes.value
+
+
+def gs_cull_workspace(N, cam: GsCamera) -> int:
+    nbytes = ctypes.c_size_t(0)
+    _check("gs_cull", load().gs_cull(None, None, int(N), ctypes.byref(cam), 0.0, 0.0, None, None, None,
+                                     None, ctypes.byref(nbytes), None))
+    return nbytes.value
+
+
+def gs_preprocess(means, log_scales, quats, opacity_logits, sh, sh_degree, N, active_idx, n_active,
+                  cam: GsCamera, out: GsProjected, stream=None):
+    _check("gs_preprocess", load().gs_preprocess(
+        _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
+        _p(active_idx), _p(n_active), ctypes.byref(cam), ctypes.byref(out), _stream(stream)))
+
+
+def gs_bin_sort_workspace(n, cam: GsCamera, capacity) -> int:
+    nbytes = ctypes.c_size_t(0)
+    ni = ctypes.c_int64(0)
+    _check("gs_bin_sort", load().gs_bin_sort(None, int(n), ctypes.byref(cam), None, None, None,
+                                             int(capacity), None, ctypes.byref(ni), None,
+                                             ctypes.byref(nbytes), None))
+    return nbytes.value
+
+
+def gs_bin_sort(rec: GsProjected, n, cam: GsCamera, offsets, keys, vals, capacity, tile_ranges,
+                workspace, stream=None, raise_on_capacity=True):
+    """Returns (status, n_instances). Raises on errors other than GS_ERR_CAPACITY."""
+    nbytes = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    ni = ctypes.c_int64(0)
+    st = load().gs_bin_sort(ctypes.byref(rec), int(n), ctypes.byref(cam), _p(offsets), _p(keys),
+                            _p(vals), int(capacity), _p(tile_ranges), ctypes.byref(ni), _p(workspace),
+                            ctypes.byref(nbytes), _stream(stream))
+    if st == GS_ERR_CAPACITY and not raise_on_capacity:
+        return st, ni.value
+    _check("gs_bin_sort", st)
+    return st, ni.value
+
+
+def gs_rasterize_fwd(rec: GsProjected, vals, tile_ranges, cam: GsCamera, bg, image, final_T,
+                     n_contrib, last, stream=None):
+    bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
+    _check("gs_rasterize_fwd", load().gs_rasterize_fwd(
+        ctypes.byref(rec), _p(vals), _p(tile_ranges), ctypes.byref(cam), ctypes.cast(bgv, P),
+        _p(image), _p(final_T), _p(n_contrib), _p(last), _stream(stream)))
+
+
+def gs_rasterize_bwd(means, log_scales, quats, opacity_logits, sh, sh_degree, N, active_idx, n_active,
+                     mask, cam: GsCamera, rec: GsProjected, vals, tile_ranges, bg, final_T, last,
+                     dL_dimage, grad2d, d_means, d_log_scales, d_quats, d_opacity_logits, d_sh,
+                     stream=None):
+    bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
+    _check("gs_rasterize_bwd", load().gs_rasterize_bwd(
+        _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
+        _p(active_idx), _p(n_active), _p(mask), ctypes.byref(cam), ctypes.byref(rec), _p(vals),
+        _p(tile_ranges), ctypes.cast(bgv, P), _p(final_T), _p(last), _p(dL_dimage), _p(grad2d),
+        _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
+
+
+def gs_rasterize_bwd_2d(rec: GsProjected, n_records, vals, tile_ranges, cam: GsCamera, bg, final_T, last,
+                        dL_dimage, grad2d, stream=None):
+    bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
+    _check("gs_rasterize_bwd_2d", load().gs_rasterize_bwd_2d(
+        ctypes.byref(rec), int(n_records), _p(vals), _p(tile_ranges), ctypes.byref(cam),
+        ctypes.cast(bgv, P), _p(final_T), _p(last), _p(dL_dimage), _p(grad2d), _stream(stream)))
+
+
+def gs_debug_kernel_launches() -> int:
+    return int(load().gs_debug_kernel_launches())
+
+
+def gs_preprocess_bwd(means, log_scales, quats, opacity_logits, sh, sh_degree, N, active_idx, n_active,
+                      mask, cam: GsCamera, rec: GsProjected, grad2d, d_means, d_log_scales, d_quats,
+                      d_opacity_logits, d_sh, stream=None):
+    _check("gs_preprocess_bwd", load().gs_preprocess_bwd(
+        _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
+        _p(active_idx), _p(n_active), _p(mask), ctypes.byref(cam), ctypes.byref(rec), _p(grad2d),
+        _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
+
+
+def gs_debug_set_stalled_sort_tile(tile: int):
+    load().gs_debug_set_stalled_sort_tile(int(tile))

@@ -1,0 +1,244 @@
+"""The rasterizer's public Python API: one view forward and backward through
+the five C entry points (gs_cull, gs_preprocess, gs_bin_sort,
+gs_rasterize_fwd, gs_rasterize_bwd). Torch only allocates device memory and
+supplies the stream; every stage runs in libgs.so.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import gs
+
+
+@dataclasses.dataclass
+class GaussianParams:
+    """Device-resident parameters in the library's SoA layout."""
+    means: torch.Tensor        # [3][N]
+    log_scales: torch.Tensor   # [3][N]
+    quats: torch.Tensor        # [4][N]
+    opacity_logits: torch.Tensor  # [N]
+    sh: torch.Tensor           # [K*3][N]
+    sh_degree: int
+    importance: Optional[torch.Tensor] = None  # [N]
+
+    @property
+    def N(self) -> int:
+        return int(self.opacity_logits.shape[0])
+
+    @property
+    def K(self) -> int:
+        return (self.sh_degree + 1) ** 2
+
+    @staticmethod
+    def from_scene(scene, device="cuda") -> "GaussianParams":
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        return GaussianParams(t(scene.means), t(scene.log_scales), t(scene.quats),
+                              t(scene.opacity_logits), t(scene.sh), scene.sh_degree,
+                              None if scene.importance is None else t(scene.importance))
+
+    @staticmethod
+    def empty_like_host(scene, pin=True):
+        """Pinned host copies of a scene's parameters (for host-buffer calls)."""
+        f = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory() if pin else torch.from_numpy(a)
+        return {k: f(getattr(scene, k)) for k in ("means", "log_scales", "quats", "opacity_logits", "sh")}
+
+
+class _NoTimer:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+class _StageTimer:
+    def __init__(self, store):
+        self.store = store
+
+    def __enter__(self):
+        self.start = torch.cuda.Event(enable_timing=True)
+        self.end = torch.cuda.Event(enable_timing=True)
+        self.start.record()
+        return self
+
+    def __exit__(self, *a):
+        self.end.record()
+        self.store.append((self.start, self.end))
+        return False
+
+
+def _u8(n, dev):
+    return torch.empty(max(int(n), 1), dtype=torch.uint8, device=dev)
+
+
+class Rasterizer:
+    """Buffers and calls for rendering one view of N Gaussians at W x H.
+
+    forward() runs cull -> preprocess -> bin_sort -> rasterize_fwd and keeps
+    what backward() needs; backward() runs rasterize_bwd. Buffers are
+    allocated once (the instance capacity grows when gs_bin_sort reports it
+    is too small) and reused across calls.
+    """
+
+    def __init__(self, N: int, sh_degree: int, width: int, height: int, device=None,
+                 capacity: Optional[int] = None):
+        self.dev = torch.device(device or "cuda")
+        self.N, self.sh_degree, self.W, self.H = int(N), int(sh_degree), int(width), int(height)
+        self.K = (sh_degree + 1) ** 2
+        self.TW, self.TH = (width + 15) // 16, (height + 15) // 16
+        self.TT = self.TW * self.TH
+        n, d = max(self.N, 1), self.dev
+        f32 = dict(dtype=torch.float32, device=d)
+        i32 = dict(dtype=torch.int32, device=d)
+        self.rec = {"xyzo": torch.empty((n, 4), **f32), "conic": torch.empty((n, 4), **f32),
+                    "rgb": torch.empty((n, 4), **f32), "radius": torch.empty(n, **i32),
+                    "rect": torch.empty((n, 4), dtype=torch.int16, device=d),
+                    "tiles": torch.empty(n, **i32)}
+        self.offsets = torch.empty(n, **i32)
+        self.mask = torch.empty(n, dtype=torch.uint8, device=d)
+        self.active_idx = torch.empty(n, **i32)
+        self.n_active = torch.zeros(1, **i32)
+        self.image = torch.empty((3, height, width), **f32)
+        self.final_T = torch.empty((height, width), **f32)
+        self.n_contrib = torch.empty((height, width), **i32)
+        self.last = torch.empty((height, width), **i32)
+        self.ranges = torch.empty((self.TT, 2), **i32)
+        self.grad2d = torch.empty((n, 12), **f32)
+        self.grads = {"means": torch.empty((3, n), **f32), "log_scales": torch.empty((3, n), **f32),
+                      "quats": torch.empty((4, n), **f32), "opacity_logits": torch.empty(n, **f32),
+                      "sh": torch.empty((3 * self.K, n), **f32)}
+        self._proj = gs.projected(self.rec)
+        self.capacity = 0
+        self.keys = self.vals = self.sort_ws = None
+        self._cam_wh = None
+        self._ensure_capacity(capacity if capacity is not None else max(4 * self.N, 1024))
+        cam_probe = gs.GsCamera()
+        cam_probe.width, cam_probe.height = width, height
+        self.cull_ws = _u8(gs.gs_cull_workspace(self.N, cam_probe), d)
+        self.n_instances = 0
+        self.params = None
+        self.cam = None
+        self.bg = (0.0, 0.0, 0.0)
+        self.culled = False
+        # Optional per-stage CUDA-event timing: {stage: [(start, end), ...]}.
+        self.stage_events = None
+
+    def _timed(self, stage):
+        ev = self.stage_events
+        if ev is None:
+            return _NoTimer()
+        return _StageTimer(ev.setdefault(stage, []))
+
+    def _ensure_capacity(self, cap: int):
+        if cap <= self.capacity:
+            return
+        cap = int(cap)
+        self.keys = torch.empty(max(cap, 1), dtype=torch.int64, device=self.dev)
+        self.vals = torch.empty(max(cap, 1), dtype=torch.int32, device=self.dev)
+        probe = gs.GsCamera()
+        probe.width, probe.height = self.W, self.H
+        self.sort_ws = _u8(gs.gs_bin_sort_workspace(self.N, probe, cap), self.dev)
+        self.capacity = cap
+
+    # ------------------------------------------------------------------ stages
+    def cull(self, params: GaussianParams, cam: gs.GsCamera, lod_dist=0.0, importance_q=0.0):
+        with self._timed("cull"):
+            gs.gs_cull(params.means, params.importance if importance_q > 0 else None, self.N, cam,
+                       lod_dist, importance_q, self.mask, self.active_idx, self.n_active, self.cull_ws)
+        self.culled = True
+
+    def preprocess(self, params: GaussianParams, cam: gs.GsCamera):
+        act = self.active_idx if self.culled else None
+        na = self.n_active if self.culled else None
+        with self._timed("preprocess"):
+            gs.gs_preprocess(params.means, params.log_scales, params.quats, params.opacity_logits,
+                             params.sh, params.sh_degree, self.N, act, na, cam, self._proj)
+
+    def bin_sort(self, cam: gs.GsCamera) -> int:
+        with self._timed("bin_sort"):
+            return self._bin_sort(cam)
+
+    def _bin_sort(self, cam: gs.GsCamera) -> int:
+        st, ni = gs.gs_bin_sort(self._proj, self.N, cam, self.offsets, self.keys, self.vals, self.capacity,
+                                self.ranges, self.sort_ws, raise_on_capacity=False)
+        if st == gs.GS_ERR_CAPACITY:
+            self._ensure_capacity(int(ni * 1.25) + 1024)
+            st, ni = gs.gs_bin_sort(self._proj, self.N, cam, self.offsets, self.keys, self.vals,
+                                    self.capacity, self.ranges, self.sort_ws)
+        self.n_instances = ni
+        return ni
+
+    def raster_fwd(self, cam: gs.GsCamera, bg):
+        with self._timed("raster_fwd"):
+            gs.gs_rasterize_fwd(self._proj, self.vals, self.ranges, cam, bg, self.image, self.final_T,
+                                self.n_contrib, self.last)
+
+    # ------------------------------------------------------------------ public
+    def forward(self, params: GaussianParams, cam, bg=(0.0, 0.0, 0.0), lod_dist=0.0,
+                importance_q=0.0) -> torch.Tensor:
+        c = cam if isinstance(cam, gs.GsCamera) else gs.camera(cam)
+        if (c.width, c.height) != (self.W, self.H):
+            raise ValueError("camera size differs from the rasterizer's")
+        self.params, self.cam, self.bg = params, c, tuple(float(b) for b in bg)
+        self.cull(params, c, lod_dist, importance_q)
+        self.preprocess(params, c)
+        self.bin_sort(c)
+        self.raster_fwd(c, self.bg)
+        return self.image
+
+    def backward(self, dL_dimage: torch.Tensor) -> dict:
+        p, c = self.params, self.cam
+        act = self.active_idx if self.culled else None
+        na = self.n_active if self.culled else None
+        mask = self.mask if self.culled else None
+        g = self.grads
+        if self.stage_events is None:
+            gs.gs_rasterize_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
+                                self.N, act, na, mask, c, self._proj, self.vals, self.ranges, self.bg,
+                                self.final_T, self.last, dL_dimage, self.grad2d, g["means"],
+                                g["log_scales"], g["quats"], g["opacity_logits"], g["sh"])
+            return g
+        # the same two parts as separate calls, so each can be timed
+        with self._timed("raster_bwd"):
+            gs.gs_rasterize_bwd_2d(self._proj, self.N, self.vals, self.ranges, c, self.bg, self.final_T,
+                                   self.last, dL_dimage, self.grad2d)
+        with self._timed("preprocess_bwd"):
+            gs.gs_preprocess_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
+                                 self.N, act, na, mask, c, self._proj, self.grad2d, g["means"],
+                                 g["log_scales"], g["quats"], g["opacity_logits"], g["sh"])
+        return g
+
+    def work_counts(self) -> dict:
+        """Per-view work of the last forward (device reductions, then one sync):
+        visible Gaussians V, instances I, forward-evaluated pairs E (pairs of a
+        pixel and an entry of its tile's list up to the pixel's stop), backward
+        pairs E_bwd (entries before each pixel's last blend) and blends B."""
+        H, W = self.H, self.W
+        lens = (self.ranges[:, 1] - self.ranges[:, 0]).to(torch.int64)
+        ty = torch.arange(H, device=self.dev) // 16
+        tx = torch.arange(W, device=self.dev) // 16
+        tile = (ty[:, None] * self.TW + tx[None, :]).reshape(-1)
+        plen = lens[tile].reshape(H, W)
+        last = self.last.to(torch.int64)
+        stopped = self.final_T < 1e-4
+        E = torch.where(stopped, last, plen).sum()
+        out = torch.stack([(self.rec["tiles"] > 0).sum().to(torch.int64), E, last.sum(),
+                           self.n_contrib.to(torch.int64).sum()]).cpu().tolist()
+        return {"V": out[0], "I": self.n_instances, "E": out[1], "E_bwd": out[2], "B": out[3]}
+
+    def records_numpy(self) -> dict:
+        r = {k: v.cpu().numpy() for k, v in self.rec.items()}
+        r["rect"] = r["rect"].view(np.uint16)
+        return r
+
+    def bins_numpy(self) -> dict:
+        I = self.n_instances
+        return {"keys": self.keys[:I].cpu().numpy().view(np.uint64),
+                "vals": self.vals[:I].cpu().numpy().view(np.uint32),
+                "ranges": self.ranges.cpu().numpy().view(np.uint32),
+                "offsets": self.offsets.cpu().numpy(), "n_instances": I}

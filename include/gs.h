@@ -1,0 +1,230 @@
+/*
+ * gs.h -- C ABI of the B200 differentiable tile rasterizer for 3D Gaussian
+ * splats (libgs.so).
+ *
+ * The method: a per-view active-set cull, per-Gaussian EWA projection with
+ * spherical-harmonic colour, binning of (Gaussian, tile) pairs by a 64-bit
+ * key (tile_id << 32 | depth bits) with a stable radix sort, per-tile range
+ * extraction, front-to-back alpha compositing per pixel over 16x16 tiles,
+ * and the matching backward pass.
+ *
+ * Sources on the pages this library follows:
+ *  - BlitzGS (CVPR 2026) write-up, section 2.3 "视图层级精细化修剪": per-view
+ *    active set from a distance-LOD gate and an importance cull mask.
+ *  - 4D-GS release page ("VisionTech 发布并开源 ... 120fps 实时渲染"), section
+ *    "技术架构与关键机制": tiled rasterization with per-pixel alpha blending.
+ *  - "像素扩散与CUDA内核优化" (Gsplat part), section 三.2: projection stages
+ *    as separate parallel blocks; spatially local data staged in shared memory.
+ *  - Spirula Studio quantised-training page, sections "先算一笔账" (full SH3
+ *    colour, 45 coefficients per Gaussian) and "实测" (64-bit element addressing
+ *    once element counts pass 2^31).
+ *
+ * Conventions for every entry point
+ *  - Pointers marked [device] are CUDA device pointers owned by the caller;
+ *    the library never allocates, frees or retains them. Pointers marked
+ *    [host] are read during the call only.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *    stream. Work is enqueued asynchronously on it unless stated otherwise.
+ *  - Calls that need scratch memory take (workspace, workspace_bytes). With
+ *    workspace == NULL the call only stores the required size in
+ *    *workspace_bytes and returns GS_OK. The workspace must be 256-byte
+ *    aligned and not shared by calls in flight at the same time.
+ *  - Parameters use structure-of-arrays planes of float32, element counts in
+ *    int64 (SH planes hold 48*N floats, past 2^31 elements at 45M Gaussians).
+ *      means [3][N], log_scales [3][N], quats [4][N] as (w, x, y, z),
+ *      opacity_logits [N], sh [K*3][N] with plane index k*3 + channel,
+ *      K = (sh_degree + 1)^2.
+ *  - Images are channel-planar: image [3][H][W]; per-pixel maps are [H][W].
+ *    Pixel (u, v) is sampled at (u + 0.5, v + 0.5); tiles are 16x16 pixels,
+ *    TW = ceil(W/16), TH = ceil(H/16), tile id = ty*TW + tx.
+ *  - Return values are GS_* codes below; on an error the outputs are
+ *    unspecified. GS_ERR_CUDA means a CUDA runtime call failed (the CUDA error
+ *    is left for the caller to query with cudaGetLastError).
+ *  - Arithmetic follows a fixed fp32 specification (operation order, explicit
+ *    fused multiply-adds, a software exp2) so that every discrete result --
+ *    cull masks, radii, tile rects, keys, sorted order, ranges and per-pixel
+ *    contributor counts -- is reproducible bit for bit by an independent CPU
+ *    implementation.
+ */
+#ifndef GS_H_
+#define GS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GS_API __attribute__((visibility("default")))
+
+enum {
+  GS_OK = 0,
+  GS_ERR_INVALID_ARGUMENT = 1, /* null pointer, negative size, bad camera, ...  */
+  GS_ERR_CAPACITY = 2,         /* more (Gaussian, tile) instances than capacity */
+  GS_ERR_CUDA = 3,             /* a CUDA runtime call failed                    */
+  GS_ERR_DEVICE_TIMEOUT = 4,   /* a bounded device-side wait gave up            */
+  GS_ERR_UNSUPPORTED = 5       /* e.g. sh_degree > 3                            */
+};
+
+/* Pinhole camera, OpenCV axes (x right, y down, z forward). */
+typedef struct gs_camera {
+  float R[9];      /* world -> camera rotation, row-major                        */
+  float t[3];      /* world -> camera translation: t_cam = R mu + t              */
+  float campos[3]; /* camera centre in world coordinates (SH direction, LOD)     */
+  float fx, fy, cx, cy; /* intrinsics in pixels                                   */
+  float near_z;    /* Gaussians with camera-space z <= near_z are culled; >= 0    */
+  int32_t width, height; /* image size in pixels, each in [1, 65535*16]          */
+} gs_camera;
+
+/* Projected records, one per active position (structure of small vectors).
+ * A record is written in full only for a visible Gaussian (tiles_touched > 0);
+ * all fields of other records are zero. */
+typedef struct gs_projected {
+  float* xyzo;            /* [device] [cap][4]: px, py, depth (camera z), opacity */
+  float* conic;           /* [device] [cap][4]: A, B, C of Sigma'^-1, 0           */
+  float* rgb;             /* [device] [cap][4]: r, g, b, 0                        */
+  int32_t* radius;        /* [device] [cap]: ceil(3 sqrt(lambda_max(Sigma')))     */
+  uint16_t* rect;         /* [device] [cap][4]: x0, y0, x1, y1 tile rect, end-excl*/
+  int32_t* tiles_touched; /* [device] [cap]: (x1 - x0) * (y1 - y0)                */
+} gs_projected;
+
+GS_API int gs_version(void);
+GS_API const char* gs_status_string(int status);
+
+/* Per-view active-set cull (BlitzGS write-up, section 2.3: distance-LOD gate
+ * and importance cull mask).
+ *   keep(g) = [lod_dist <= 0 or |mu_g - campos|^2 <= lod_dist^2]
+ *           and [importance_q == 0 or importance[g] >= tau]
+ * with the squared distance in fp32 as ((dx*dx + dy*dy) + dz*dz) and tau the
+ * value of rank floor(q*N) (0-based, ascending, total order on the fp32 bit
+ * patterns) among all N weights. Then order-preserving compaction.
+ *   means        [device] [3][N]
+ *   importance   [device] [N], may be NULL when importance_q == 0
+ *   N            number of Gaussians, 0 <= N < 2^31
+ *   cam          [host] camera (campos is used)
+ *   importance_q in [0, 1)
+ *   mask         [device] [N] u8 out: 1 kept, 0 culled
+ *   active_idx   [device] [N] i32 out: kept indices in increasing order
+ *   n_active     [device] i32 out: number of kept Gaussians
+ *   workspace    [device] scratch, see conventions
+ * Asynchronous. */
+GS_API int gs_cull(const float* means, const float* importance, int64_t N, const gs_camera* cam,
+                   float lod_dist, float importance_q, uint8_t* mask, int32_t* active_idx,
+                   int32_t* n_active, void* workspace, size_t* workspace_bytes, void* stream);
+
+/* Projection of every active Gaussian into records (EWA splatting):
+ *   t = R mu + t, culled unless t.z > near_z; s = exp(log_s); q normalised;
+ *   Sigma = Rq S S^T Rq^T; J = d(pinhole)/dt at t;
+ *   Sigma' = J R Sigma R^T J^T + 0.3 I; culled unless det(Sigma') > 0;
+ *   conic = Sigma'^-1; radius = ceil(3 sqrt(lambda_max)); centre
+ *   (fx tx/tz + cx, fy ty/tz + cy); tile rect of the radius square clamped to
+ *   the grid, culled if empty; opacity = 1/(1 + exp(-logit));
+ *   colour = max(0, sum_k Y_k(dir) sh_k + 0.5) with dir = (mu - campos)/|.|
+ *   and Y the real orthonormal SH basis (Condon-Shortley phase), l <= sh_degree.
+ * Non-finite means, log-scales, quaternions or logits, and zero quaternions,
+ * cull the Gaussian.
+ *   active_idx   [device] [N] or NULL (record i is Gaussian i)
+ *   n_active     [device] i32 or NULL (then N). Records i >= n_active get
+ *                tiles_touched = 0.
+ *   out          [host] struct of [device] arrays with capacity N
+ * Asynchronous. */
+GS_API int gs_preprocess(const float* means, const float* log_scales, const float* quats,
+                         const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                         const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
+                         const gs_projected* out, void* stream);
+
+/* Tile binning: exclusive scan of tiles_touched into offsets, emission of one
+ * (key, value) per (Gaussian, tile) with key = (tile_id << 32) | bits(depth),
+ * value = record index, tiles in row-major order within the rect; stable LSD
+ * radix sort (8-bit digits, onesweep with decoupled look-back) over the key
+ * bits [0, 32 + ceil(log2(TW*TH))); then [start, end) per tile into
+ * tile_ranges (empty tiles [0, 0)).
+ *   in           [host] struct of [device] records, n entries
+ *   offsets      [device] [n] i32 out
+ *   keys, vals   [device] [capacity] out, sorted
+ *   capacity     size of keys/vals, < 2^30
+ *   tile_ranges  [device] [TW*TH][2] u32 out
+ *   n_instances  [host] out: number of instances I
+ * Synchronous: waits on `stream` once to read I and once at the end to read
+ * the device status. Returns GS_ERR_CAPACITY (with *n_instances set, nothing
+ * sorted) when I > capacity, GS_ERR_DEVICE_TIMEOUT if a look-back wait hit its
+ * iteration limit. */
+GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
+                       uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
+                       int64_t* n_instances, void* workspace, size_t* workspace_bytes,
+                       void* stream);
+
+/* Forward compositing (tiled rasterization with alpha blending). For each
+ * pixel, over its tile's sorted list: alpha = min(0.99, o exp(p)) with
+ * p = -1/2 (A dx^2 + C dy^2) - B dx dy, (dx, dy) = (px - u - 0.5, py - v - 0.5);
+ * skip alpha < 1/255; C += T alpha c; T *= 1 - alpha; stop once T < 1e-4
+ * (the crossing Gaussian is blended). out = C + T bg.
+ *   vals, tile_ranges [device] from gs_bin_sort
+ *   bg           [host] 3 floats
+ *   image        [device] [3][H][W] out
+ *   final_T      [device] [H][W] out
+ *   n_contrib    [device] [H][W] i32 out: blended Gaussians
+ *   last         [device] [H][W] i32 out: 1 + list offset of the last blend
+ * Asynchronous. */
+GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
+                            const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                            float* image, float* final_T, int32_t* n_contrib, int32_t* last,
+                            void* stream);
+
+/* Backward pass: exact derivatives of the forward with every discrete decision
+ * held fixed (visibility, tile lists, skips, the 0.99 clamp -- zero gradient
+ * through a clamped alpha -- colour clamps, stop points).
+ * Part 1 replays each pixel back to front and accumulates per-record 2-D
+ * gradients into grad2d; part 2 chains them to the parameters.
+ *   params, sh_degree, N, active_idx, n_active: as given to gs_preprocess
+ *   mask         [device] [N] u8 from gs_cull or NULL (all active)
+ *   in           records from gs_preprocess
+ *   final_T, last from gs_rasterize_fwd; dL_dimage [device] [3][H][W]
+ *   grad2d       [device] [N][12] f32 out: (dpx, dpy, dopacity, 0,
+ *                dA, dB, dC, 0, dr, dg, db, 0) per record
+ *   d_*          [device] out, same layouts as the parameters; overwritten,
+ *                zero for Gaussians that are culled or not visible
+ * Asynchronous. */
+GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const float* quats,
+                            const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                            const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
+                            const gs_camera* cam, const gs_projected* in, const uint32_t* vals,
+                            const uint32_t* tile_ranges, const float* bg, const float* final_T,
+                            const int32_t* last, const float* dL_dimage, float* grad2d,
+                            float* d_means, float* d_log_scales, float* d_quats,
+                            float* d_opacity_logits, float* d_sh, void* stream);
+
+/* Part 1 of gs_rasterize_bwd alone: the back-to-front replay that writes the
+ * per-record 2-D gradients grad2d [device] [N][12] (zeroed first), without
+ * chaining them to the parameters. Same arguments as the corresponding ones
+ * of gs_rasterize_bwd; n_records = N. Asynchronous. */
+GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,
+                               const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                               const float* final_T, const int32_t* last, const float* dL_dimage,
+                               float* grad2d, void* stream);
+
+/* Part 2 of gs_rasterize_bwd alone: parameter gradients from given per-record
+ * 2-D gradients grad2d [device] [N][12] (input). Same outputs. Asynchronous. */
+GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const float* quats,
+                             const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                             const int32_t* active_idx, const int32_t* n_active,
+                             const uint8_t* mask, const gs_camera* cam, const gs_projected* in,
+                             const float* grad2d, float* d_means, float* d_log_scales,
+                             float* d_quats, float* d_opacity_logits, float* d_sh, void* stream);
+
+/* Number of kernels this library has launched in the process so far (all
+ * devices, all streams). Host-side counter, for accounting in benchmarks. */
+GS_API int64_t gs_debug_kernel_launches(void);
+
+/* Fault-injection hook for tests of the bounded look-back wait: while set to
+ * k >= 0, tile k of every radix-sort pass never publishes its counts, so its
+ * successor's wait runs out and gs_bin_sort returns GS_ERR_DEVICE_TIMEOUT.
+ * -1 (the default) disables it. Host-side state, not thread-safe. */
+GS_API void gs_debug_set_stalled_sort_tile(int64_t tile);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GS_H_ */

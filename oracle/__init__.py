@@ -75,7 +75,8 @@ def _declare(L):
                                      P, P, P, P, P, P, P, P, P]
     L.or_loss_frozen_f64.restype = ctypes.c_double
     L.or_backward_f64.argtypes = [P, P, P, P, P, I32, I64, P, I64, P, I32, I32,
-                                  P, P, P, P, P, P, P, P, P, P] + [P] * 10
+                                  P, P, P, P, P, P, P, P, P, P] + [P] * 10 + [P, I64]
+    L.or_num_threads.restype = ctypes.c_int
     L.or_preprocess_bwd_f64.argtypes = [P, P, P, P, P, I32, I64, P, I64, P, I32, I32,
                                         P, P, P] + [P] * 10
     L.or_project_f64.argtypes = [P, P, P, P, P, I32, I64, P, I32, I32, P, P, P]
@@ -238,7 +239,11 @@ def loss_frozen(params64, scene, cam, rec, bins, dL_dimage, want_image=False):
     return (loss, img) if want_image else loss
 
 
-def backward(scene, cam, rec, bins, dL_dimage, params3d=True):
+def num_threads() -> int:
+    return int(lib().or_num_threads())
+
+
+def backward(scene, cam, rec, bins, dL_dimage, params3d=True, tile_subset=None):
     """Reference gradients (fp64, fp32 decisions) with magnitude bounds."""
     N, K = scene.N, scene.K
     na = rec["n_active"]
@@ -257,7 +262,9 @@ def backward(scene, cam, rec, bins, dL_dimage, params3d=True):
         _p(cam_array(cam)), cam.width, cam.height, _p(rec["xyzo"]), _p(rec["conic"]),
         _p(rec["rgb"]), _p(rec["tiles"]), _p(vals), _p(_c(bins["ranges"], np.uint32)),
         _p(_c(scene.bg, np.float32)), _p(_c(dL_dimage, np.float32)), _p(g2), _p(s2),
-        *[_p(a) for a in d], *[_p(a) for a in m])
+        *[_p(a) for a in d], *[_p(a) for a in m],
+        _p(None if tile_subset is None else _c(tile_subset, np.int32)),
+        0 if tile_subset is None else len(tile_subset))
     if params3d:
         names = ["means", "log_scales", "quats", "opacity_logits", "sh"]
         out.update({"d_" + k: v for k, v in zip(names, d)})

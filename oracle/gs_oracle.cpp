@@ -53,6 +53,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <limits>
+#include <type_traits>
 #include <vector>
 #ifdef _OPENMP
 #include <omp.h>
@@ -221,6 +222,45 @@ void sh_basis_grad(double x, double y, double z, int K, double G[16][3]) {
   G[14][0] = c[14] * 2.0 * x * z; G[14][1] = c[14] * (-2.0 * y * z);
   G[14][2] = c[14] * (xx - yy);
   G[15][0] = c[15] * (3.0 * xx - 3.0 * yy); G[15][1] = c[15] * (-6.0 * x * y);
+}
+
+// Magnitude versions of the basis and its gradient: every polynomial
+// evaluated on |x|, |y|, |z| with its subtractions turned into additions and
+// |constant|. They bound the size of the terms an fp32 evaluation sums, which
+// sets its rounding error where a polynomial nearly cancels.
+void sh_basis_abs(double x, double y, double z, int K, double Y[16]) {
+  x = std::fabs(x); y = std::fabs(y); z = std::fabs(z);
+  const double* c = KC.shd;
+  double a[16];
+  for (int k = 0; k < 16; ++k) a[k] = std::fabs(c[k]);
+  const double xx = x * x, yy = y * y, zz = z * z;
+  Y[0] = a[0];
+  Y[1] = a[1] * y; Y[2] = a[2] * z; Y[3] = a[3] * x;
+  Y[4] = a[4] * x * y; Y[5] = a[5] * y * z; Y[6] = a[6] * (2 * zz + xx + yy);
+  Y[7] = a[7] * x * z; Y[8] = a[8] * (xx + yy);
+  Y[9] = a[9] * y * (3 * xx + yy); Y[10] = a[10] * x * y * z;
+  Y[11] = a[11] * y * (4 * zz + xx + yy); Y[12] = a[12] * z * (2 * zz + 3 * xx + 3 * yy);
+  Y[13] = a[13] * x * (4 * zz + xx + yy); Y[14] = a[14] * z * (xx + yy);
+  Y[15] = a[15] * x * (xx + 3 * yy);
+  for (int k = K; k < 16; ++k) Y[k] = 0.0;
+}
+
+void sh_basis_grad_abs(double x, double y, double z, int K, double G[16][3]) {
+  sh_basis_grad(std::fabs(x), std::fabs(y), std::fabs(z), K, G);
+  for (int k = 0; k < 16; ++k)
+    for (int m = 0; m < 3; ++m) G[k][m] = std::fabs(G[k][m]);
+  if (K <= 9) return;
+  x = std::fabs(x); y = std::fabs(y); z = std::fabs(z);
+  const double xx = x * x, yy = y * y, zz = z * z;
+  const double* c = KC.shd;
+  G[9][1] = std::fabs(c[9]) * (3 * xx + 3 * yy);
+  G[11][1] = std::fabs(c[11]) * (4 * zz + xx + 3 * yy);
+  G[12][2] = std::fabs(c[12]) * (6 * zz + 3 * xx + 3 * yy);
+  G[13][0] = std::fabs(c[13]) * (4 * zz + 3 * xx + yy);
+  G[14][2] = std::fabs(c[14]) * (xx + yy);
+  G[15][0] = std::fabs(c[15]) * (3 * xx + 3 * yy);
+  G[6][2] = std::fabs(c[6]) * 4 * z;
+  G[8][0] = std::fabs(c[8]) * 2 * x;
 }
 
 // ------------------------------------------------------------- projection
@@ -439,6 +479,14 @@ int64_t tile_count(int W, int H) { return (int64_t)((W + 15) / 16) * ((H + 15) /
 
 // Library self-description and constants used by the pins.
 OR_API int or_version(void) { return 1; }
+
+OR_API int or_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
 
 OR_API void or_constants(float* out /* 32 */) {
   for (int k = 0; k < 8; ++k) out[k] = KC.e2c[k];
@@ -779,8 +827,13 @@ void preprocess_bwd_one(const Cam& cam, const double mu[3], const double ls[3], 
   const double nd = std::sqrt(dv[0] * dv[0] + dv[1] * dv[1] + dv[2] * dv[2]);
   const double dir[3] = {dv[0] / nd, dv[1] / nd, dv[2] / nd};
   double Y[16], DY[16][3];
-  sh_basis<double>(dir[0], dir[1], dir[2], K, Y);
-  sh_basis_grad(dir[0], dir[1], dir[2], K, DY);
+  if (std::is_same<G, Mag>::value) {
+    sh_basis_abs(dir[0], dir[1], dir[2], K, Y);
+    sh_basis_grad_abs(dir[0], dir[1], dir[2], K, DY);
+  } else {
+    sh_basis<double>(dir[0], dir[1], dir[2], K, Y);
+    sh_basis_grad(dir[0], dir[1], dir[2], K, DY);
+  }
   G gv[3];
   for (int ch = 0; ch < 3; ++ch) gv[ch] = clamped[ch] ? gz<G>() : g2[6 + ch];
   G gdir[3] = {gz<G>(), gz<G>(), gz<G>()};
@@ -924,7 +977,8 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
                            const float* bg, const float* dL_dimage, double* g2d, double* s2d,
                            double* d_means, double* d_log_scales, double* d_quats, double* d_logits,
                            double* d_sh, double* m_means, double* m_log_scales, double* m_quats,
-                           double* m_logits, double* m_sh) {
+                           double* m_logits, double* m_sh, const int32_t* tile_subset,
+                           int64_t n_subset) {
   const int K = (sh_degree + 1) * (sh_degree + 1);
   const Cam cam = make_cam(camv, width, height);
   // fp64 copies of the parameters
@@ -943,8 +997,10 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
   const int TW = cam.TW;
   const int64_t TT = tile_count(width, height);
   const size_t NP = (size_t)width * height;
+  const int64_t nt = tile_subset ? n_subset : TT;
 #pragma omp parallel for schedule(dynamic, 4)
-  for (int64_t tile = 0; tile < TT; ++tile) {
+  for (int64_t s = 0; s < nt; ++s) {
+    const int64_t tile = tile_subset ? tile_subset[s] : s;
     const int tx = (int)(tile % TW), ty = (int)(tile / TW);
     const uint32_t start = ranges[2 * tile], end = ranges[2 * tile + 1];
     std::vector<Blend> bl;

@@ -1,0 +1,58 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every
+entry point that include/gs.h declares (no compute calls here)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from differentiable_tile_rasterizer_b200 import _build, gs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "gs.h")).read()
+    return sorted(set(re.findall(r"GS_API\s+[\w\s\*]+?\b(gs_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_five_stages():
+    names = _declared()
+    for n in ["gs_cull", "gs_preprocess", "gs_bin_sort", "gs_rasterize_fwd", "gs_rasterize_bwd",
+              "gs_status_string"]:
+        assert n in names
+    assert set(names) == set(gs.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    path = _build.build()
+    lib = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(gs_\w+)", out))
+    assert set(_declared()) <= exported
+    # nothing else with the public prefix leaks out
+    assert exported == set(_declared())
+
+
+def test_status_strings_and_version():
+    L = gs.load()
+    assert gs.version() == 1
+    assert L.gs_status_string(0) == b"ok"
+    assert L.gs_status_string(4).startswith(b"bounded")
+
+
+def test_workspace_queries_need_no_gpu():
+    cam = gs.GsCamera()
+    cam.width, cam.height = 1920, 1080
+    assert gs.gs_cull_workspace(1_000_000, cam) > 0
+    small = gs.gs_bin_sort_workspace(1000, cam, 10_000)
+    big = gs.gs_bin_sort_workspace(1000, cam, 10_000_000)
+    assert big > small > 12 * 10_000
+    cam.width = 0
+    with pytest.raises(gs.GsError):
+        gs.gs_cull_workspace(10, cam)
+

@@ -1,0 +1,281 @@
+"""CUDA path against the oracle, element by element, through the C ABI.
+
+Integer results (cull mask, active list, radius, rect, tiles, offsets, keys,
+sorted values, ranges, contributor counts, last index) must be bit-exact.
+Floats of the fp32 specification (records, image, transmittance) are
+compared within 1e-4 absolute and are expected to be bit-equal too.
+Gradients: |g - g_ref| <= 1e-3 |g_ref| + 1e-4 S, where g_ref is the oracle's
+float64 gradient and S the sum of the absolute per-pixel contributions to
+that element (propagated through the projection backward by magnitudes).
+The S term covers fp32 accumulation and the division-based recovery of T,
+whose relative error grows with the number of blends behind a pixel.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from differentiable_tile_rasterizer_b200 import gs, synthetic as S
+from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, Rasterizer
+from tests._helpers import make_scene, simple_camera
+from tests.gpu_helpers import (assert_bits, bits_equal, fwd_numpy, gpu_forward, grad_tol_check,
+                               load_bins, load_records)
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ["means", "log_scales", "quats", "opacity_logits", "sh"]
+
+
+def _scenes():
+    yield "tiny", S.make_config(0)
+    yield "ragged_sh1", S.random_scene(700, 83, 37, sh_degree=1, seed=31, bg=(0.1, 0.3, 0.2))
+    yield "ragged_sh2", S.random_scene(900, 130, 75, sh_degree=2, seed=32, n_poses=2)
+    yield "sh3_rot", S.random_scene(1500, 200, 120, sh_degree=3, seed=33, n_poses=3)
+    yield "one_pixel", S.random_scene(50, 1, 1, sh_degree=0, seed=34, mean_box=0.05)
+    yield "thin_strip", S.random_scene(400, 300, 7, sh_degree=1, seed=35)
+
+
+SCENES = dict(_scenes())
+
+
+def _full_compare(scene, pose=0):
+    R = gpu_forward(scene, pose)
+    ref = oracle.render(scene, pose)
+    rec = R.records_numpy()
+    o = ref["rec"]
+    for k in ("xyzo", "conic", "rgb", "radius", "rect", "tiles"):
+        assert_bits(rec[k], o[k], k)
+    b = R.bins_numpy()
+    assert b["n_instances"] == ref["bins"]["n_instances"]
+    assert_bits(b["offsets"], ref["bins"]["offsets"], "offsets")
+    assert_bits(b["keys"], ref["bins"]["keys"], "keys")
+    assert_bits(b["vals"], ref["bins"]["vals"], "vals")
+    assert_bits(b["ranges"], ref["bins"]["ranges"], "ranges")
+    f = fwd_numpy(R)
+    for k in ("n_contrib", "last"):
+        assert_bits(f[k], ref["fwd"][k], k)
+    for k in ("image", "final_T"):
+        assert np.abs(f[k] - ref["fwd"][k]).max() <= 1e-4, k
+        assert bits_equal(f[k], ref["fwd"][k])[0], k
+    return R, ref
+
+
+@pytest.mark.parametrize("name", list(SCENES))
+def test_forward_pipeline_bitexact(name):
+    sc = SCENES[name]
+    for pose in range(len(sc.cameras)):
+        _full_compare(sc, pose)
+
+
+def test_forward_config1_bitexact():
+    _full_compare(S.make_config(1))
+
+
+def test_stagewise_sort_and_raster_from_oracle_records():
+    sc = S.random_scene(2000, 160, 144, sh_degree=2, seed=36)
+    cam = sc.cameras[0]
+    ref = oracle.render(sc)
+    R = Rasterizer(sc.N, sc.sh_degree, cam.width, cam.height)
+    load_records(R, ref["rec"])
+    c = gs.camera(cam)
+    R.bin_sort(c)
+    b = R.bins_numpy()
+    for k in ("keys", "vals", "ranges", "offsets"):
+        assert_bits(b[k], ref["bins"][k], k)
+    load_bins(R, ref["bins"])
+    R.raster_fwd(c, sc.bg)
+    f = fwd_numpy(R)
+    for k in ("n_contrib", "last", "image", "final_T"):
+        assert_bits(f[k], ref["fwd"][k], k)
+
+
+def test_preprocess_edge_cases():
+    cam = simple_camera(64, 64, 50.0, near=0.2)
+    means = np.array([[0, 0, 0, 0, 0, 100, 0, np.nan, 0.01],
+                      [0, 0, 0, 0, 0, 0, 0, 0, 0.02],
+                      [0.2, np.nextafter(np.float32(0.2), np.float32(1)), 1.0, 1.0, -1.0, 1.0, 2.0, 2.0, 0.25]],
+                     np.float32)
+    N = means.shape[1]
+    ls = np.full((3, N), -3.0, np.float32)
+    ls[:, 8] = 4.0  # huge Gaussian close to the camera: covers every tile
+    q = np.tile(np.array([[1], [0], [0], [0]], np.float32), (1, N))
+    q[:, 3] = 0.0
+    lg = np.zeros(N, np.float32)
+    lg[6] = np.inf
+    sc = make_scene(means, ls, q, lg, np.ones((3, N)), 0, [cam])
+    R, ref = _full_compare(sc)
+    assert list(ref["rec"]["tiles"] > 0) == [False, True, True, False, False, False, False, False, True]
+    assert ref["rec"]["tiles"][8] == 16
+
+
+def test_empty_scene_and_nothing_visible():
+    cam = simple_camera(40, 24, 30.0)
+    sc = make_scene(np.array([[0.0], [0.0], [-5.0]]), np.zeros((3, 1)), [[1], [0], [0], [0]], [0.0],
+                    np.zeros((3, 1)), 0, [cam], bg=(0.25, 0.5, 0.75))
+    R, ref = _full_compare(sc)
+    assert R.n_instances == 0
+    img = R.image.cpu().numpy()
+    assert np.all(img[0] == 0.25) and np.all(img[2] == 0.75)
+
+
+def test_capacity_growth_and_error():
+    sc = S.random_scene(3000, 128, 128, sh_degree=0, seed=37, log_scale=(-1.5, 0.3))
+    cam = sc.cameras[0]
+    R = gpu_forward(sc, capacity=16)  # forces the capacity error, then a resize
+    ref = oracle.render(sc)
+    assert R.n_instances == ref["bins"]["n_instances"] > 16
+    assert_bits(fwd_numpy(R)["n_contrib"], ref["fwd"]["n_contrib"], "n_contrib")
+    # the raw entry point reports GS_ERR_CAPACITY with the required count
+    R2 = Rasterizer(sc.N, 0, cam.width, cam.height, capacity=8)
+    R2.forward  # buffers only
+    params = GaussianParams.from_scene(sc)
+    c = gs.camera(cam)
+    R2.cull(params, c)
+    R2.preprocess(params, c)
+    st, ni = gs.gs_bin_sort(R2._proj, R2.N, c, R2.offsets, R2.keys, R2.vals, 8, R2.ranges, R2.sort_ws,
+                            raise_on_capacity=False)
+    assert st == gs.GS_ERR_CAPACITY and ni == ref["bins"]["n_instances"]
+
+
+def test_cull_bitexact():
+    rng = np.random.default_rng(5)
+    N = 300_000
+    means = rng.uniform(-200, 200, (3, N)).astype(np.float32)
+    imp = rng.exponential(1.0, N).astype(np.float32)
+    imp[:1000] = imp[1000]  # ties at tau candidates
+    cam = simple_camera(96, 64, 80.0)
+    cam.campos = np.array([3.0, -2.0, 1.0], np.float32)
+    base = dict(log_scales=np.full((3, N), -2.0), quats=np.tile([[1], [0], [0], [0]], (1, N)),
+                logits=np.zeros(N), sh=np.zeros((3, N)))
+    for lod, q in [(150.0, 0.3), (0.0, 0.3), (150.0, 0.0), (0.0, 0.0), (1e-3, 0.9), (250.0, 0.999),
+                   (150.0, 1e-7)]:
+        sc = make_scene(means, base["log_scales"], base["quats"], base["logits"], base["sh"], 0, [cam],
+                        importance=imp, lod_dist=lod, importance_q=q)
+        ref = oracle.cull(sc, cam)
+        params = GaussianParams.from_scene(sc)
+        R = Rasterizer(N, 0, cam.width, cam.height)
+        R.cull(params, gs.camera(cam), lod, q)
+        torch.cuda.synchronize()
+        na = int(R.n_active.item())
+        assert na == ref["n_active"], (lod, q)
+        assert_bits(R.mask.cpu().numpy(), ref["mask"], "mask")
+        assert_bits(R.active_idx[:na].cpu().numpy(), ref["active_idx"], "active_idx")
+
+
+def test_cull_then_render_city_like():
+    rng = np.random.default_rng(6)
+    sc = S.random_scene(20000, 192, 128, sh_degree=3, seed=38, mean_box=3.0, cam_dist=6.0,
+                        with_importance=True, lod_dist=6.5, importance_q=0.3)
+    R, ref = _full_compare(sc)
+    assert 0 < ref["cull"]["n_active"] < sc.N
+    assert_bits(R.mask.cpu().numpy(), ref["cull"]["mask"], "mask")
+
+
+def _backward_compare(scene, pose=0):
+    cam = scene.cameras[pose]
+    R = gpu_forward(scene, pose)
+    ref = oracle.render(scene, pose)
+    g = scene.grad_image(pose)
+    R.backward(torch.from_numpy(g).cuda())
+    torch.cuda.synchronize()
+    ob = oracle.backward(scene, cam, ref["rec"], ref["bins"], g)
+    na = ref["rec"]["n_active"]
+    g2 = R.grad2d.cpu().numpy()[:na]
+    cols = [0, 1, 4, 5, 6, 2, 8, 9, 10]  # GPU layout -> oracle order px py A B C o r g b
+    grad_tol_check(g2[:, cols], ob["g2d"], ob["s2d"], what="grad2d")
+    for n in NAMES:
+        got = R.grads[n].cpu().numpy()
+        grad_tol_check(got, ob["d_" + n], ob["m_" + n], what=n)
+    return R, ref, ob
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged_sh1", "ragged_sh2", "sh3_rot", "one_pixel"])
+def test_backward_against_oracle(name):
+    sc = SCENES[name]
+    for pose in range(len(sc.cameras)):
+        _backward_compare(sc, pose)
+
+
+def test_backward_config1():
+    _backward_compare(S.make_config(1))
+
+
+def test_backward_with_cull_zeroes_inactive():
+    sc = S.random_scene(5000, 128, 96, sh_degree=2, seed=39, mean_box=2.0, cam_dist=4.0,
+                        with_importance=True, lod_dist=4.2, importance_q=0.25)
+    R, ref, ob = _backward_compare(sc)
+    mask = ref["cull"]["mask"].astype(bool)
+    assert (~mask).any()
+    for n in NAMES:
+        assert not R.grads[n].cpu().numpy()[..., ~mask].any()
+
+
+def test_backward_clamped_alpha_and_colour():
+    sc = S.random_scene(300, 96, 80, sh_degree=1, seed=40)
+    sc.opacity_logits[:100] = 8.0
+    sc.sh[0:3, 100:150] = -5.0
+    _backward_compare(sc)
+
+
+def test_preprocess_backward_stagewise():
+    sc = S.random_scene(4000, 256, 192, sh_degree=3, seed=41, n_poses=2)
+    cam = sc.cameras[1]
+    ref = oracle.render(sc, 1)
+    rng = np.random.default_rng(0)
+    na = ref["rec"]["n_active"]
+    g2 = rng.standard_normal((na, 9)).astype(np.float32).astype(np.float64)
+    ob = oracle.preprocess_bwd(sc, cam, ref["rec"], g2)
+    R = Rasterizer(sc.N, 3, cam.width, cam.height)
+    load_records(R, ref["rec"])
+    grad2d = np.zeros((sc.N, 12), np.float32)
+    grad2d[:na, [0, 1, 4, 5, 6, 2, 8, 9, 10]] = g2
+    gd = torch.from_numpy(grad2d).cuda()
+    params = GaussianParams.from_scene(sc)
+    g = R.grads
+    gs.gs_preprocess_bwd(params.means, params.log_scales, params.quats, params.opacity_logits, params.sh,
+                         3, sc.N, None, None, None, gs.camera(cam), R._proj, gd, g["means"],
+                         g["log_scales"], g["quats"], g["opacity_logits"], g["sh"])
+    torch.cuda.synchronize()
+    for n in NAMES:
+        grad_tol_check(g[n].cpu().numpy(), ob["d_" + n], ob["m_" + n], rtol=1e-4, mtol=1e-5, what=n)
+
+
+def test_sort_lookback_timeout_is_reported_and_recoverable():
+    sc = S.random_scene(3000, 256, 256, sh_degree=0, seed=42, log_scale=(-1.0, 0.3))
+    cam = sc.cameras[0]
+    R = gpu_forward(sc)
+    assert R.n_instances > 3 * 4096  # several sort tiles per pass
+    c = gs.camera(cam)
+    gs.gs_debug_set_stalled_sort_tile(1)
+    try:
+        with pytest.raises(gs.GsError) as ei:
+            R.bin_sort(c)
+        assert ei.value.status == gs.GS_ERR_DEVICE_TIMEOUT
+        assert not R.ranges.any()
+    finally:
+        gs.gs_debug_set_stalled_sort_tile(-1)
+    R.bin_sort(c)
+    ref = oracle.render(sc)
+    assert_bits(R.bins_numpy()["keys"], ref["bins"]["keys"], "keys after recovery")
+
+
+def test_invalid_arguments_rejected():
+    cam = simple_camera(32, 32, 30.0)
+    c = gs.camera(cam)
+    bad = gs.camera(cam)
+    bad.width = 0
+    R = Rasterizer(10, 0, 32, 32)
+    params = GaussianParams.from_scene(S.random_scene(10, 32, 32, seed=1))
+    with pytest.raises(gs.GsError) as ei:
+        gs.gs_preprocess(params.means, params.log_scales, params.quats, params.opacity_logits, params.sh,
+                         4, 10, None, None, c, R._proj)
+    assert ei.value.status == gs.GS_ERR_UNSUPPORTED
+    with pytest.raises(gs.GsError) as ei:
+        gs.gs_preprocess(params.means, params.log_scales, params.quats, params.opacity_logits, params.sh,
+                         0, 10, None, None, bad, R._proj)
+    assert ei.value.status == gs.GS_ERR_INVALID_ARGUMENT
+    with pytest.raises(gs.GsError):
+        gs.gs_cull(params.means, None, 10, c, 0.0, 0.5, R.mask, R.active_idx, R.n_active, R.cull_ws)

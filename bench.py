@@ -67,7 +67,7 @@ class ClockSampler:
             sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", sel, f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except Exception:
@@ -301,7 +301,7 @@ def run_ours(args):
         line["e2e"] = e2e(args, scene, R, gimg, cams, bg, world)
     if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
-        cs = cpu_sample(scene, tile_stride=args.ref_tile_stride)
+        cs = cpu_sample(scene, tile_stride=args.cpu_tile_stride)
         line["cpu_baseline"] = {"value": 1.0 / cs["frame_s"], "unit": "frames/s", "cores": oracle.num_threads(),
                                 "kind": "oracle",
                                 "sample": f"1 pose: preprocess and bin/sort in full, forward + backward on "
@@ -360,12 +360,15 @@ def e2e(args, scene, R, gimg, cams, bg, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--ref-tile-stride", type=int, default=32)
+    ap.add_argument("--ref-tile-stride", type=int, default=32,
+                    help="reference arm: sample every n-th tile per step")
+    ap.add_argument("--cpu-tile-stride", type=int, default=8,
+                    help="cpu_baseline: sample every n-th tile")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

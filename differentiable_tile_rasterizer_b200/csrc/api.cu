@@ -117,12 +117,11 @@ GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, 
   }
   if (*workspace_bytes < plan.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return GS_ERR_INVALID_ARGUMENT;
-  if (!records_ok(in) || !n_instances || !tile_ranges || (n > 0 && !offsets) ||
-      (capacity > 0 && (!keys || !vals)))
+  if (!records_ok(in) || !n_instances || !tile_ranges || (capacity > 0 && (!keys || !vals)))
     return GS_ERR_INVALID_ARGUMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Records rec = to_records(in);
-  cudaError_t e = launch_scan_tiles(rec.tiles, n, offsets, workspace, plan, s);
+  cudaError_t e = launch_depth_order(rec, n, offsets, workspace, plan, g_stall_tile, s);
   if (e != cudaSuccess) return GS_ERR_CUDA;
   int64_t total = 0;
   e = cudaMemcpyAsync(&total, binsort_total_ptr(workspace, plan), sizeof(int64_t), cudaMemcpyDeviceToHost, s);
@@ -130,8 +129,7 @@ GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, 
   if (e != cudaSuccess) return GS_ERR_CUDA;
   *n_instances = total;
   if (total > capacity) return GS_ERR_CAPACITY;
-  e = launch_emit_sort_ranges(rec, n, offsets, dc, total, keys, vals, tile_ranges, workspace, plan,
-                              g_stall_tile, s);
+  e = launch_emit_sort_ranges(rec, n, dc, total, keys, vals, tile_ranges, workspace, plan, g_stall_tile, s);
   if (e != cudaSuccess) return GS_ERR_CUDA;
   int32_t status = 0;
   e = cudaMemcpyAsync(&status, binsort_status_ptr(workspace, plan), sizeof(int32_t), cudaMemcpyDeviceToHost, s);

@@ -84,13 +84,14 @@ struct BinSortPlan {
   size_t bytes;
 };
 BinSortPlan binsort_plan(int64_t n, int64_t capacity, int64_t tiles);
-cudaError_t launch_scan_tiles(const int32_t* tiles, int64_t n, int32_t* offsets, void* ws,
-                              const BinSortPlan& plan, cudaStream_t s);
+// Sorts the records by (depth, index) and scans their tiles_touched in that
+// order (total at binsort_total_ptr); also the record-order offsets if given.
+cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, void* ws,
+                               const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s);
 const int64_t* binsort_total_ptr(void* ws, const BinSortPlan& plan);
 const int32_t* binsort_status_ptr(void* ws, const BinSortPlan& plan);
-cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const int32_t* offsets,
-                                    const DevCam& cam, int64_t n_inst, uint64_t* keys,
-                                    uint32_t* vals, uint32_t* ranges, void* ws,
+cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam& cam, int64_t n_inst,
+                                    uint64_t* keys, uint32_t* vals, uint32_t* ranges, void* ws,
                                     const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s);
 
 // raster.cu

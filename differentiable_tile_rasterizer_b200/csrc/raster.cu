@@ -30,6 +30,38 @@ __device__ __forceinline__ void tile_pixel(int tid, int& du, int& dv) {
   dv = (w >> 1) * 4 + (l >> 3);
 }
 
+// Conservative screen box of the pixel centres at which the fp32 pair
+// arithmetic can give alpha >= 1/255 (a warp whose pixels all lie outside
+// may skip the Gaussian: the per-pixel result is the same).
+// With d = (px - x, py - y) the exact quadratic is p2(d) = -d^T M d,
+// M = [[-a2, -b2/2], [-b2/2, -c2]] positive definite. Evaluated in fp32 as
+// specified it is off by at most ~7 eps (|a2| dx^2 + |b2| |dx dy| + |c2| dy^2)
+// <= sl |d|^2 with sl = 1e-6 K, K = max(|a2|, |c2|) + |b2|/2, so the
+// computed value is <= -d^T (M - sl I) d. A blend needs o exp2(p2) >= 1/255
+// up to ~2 ulp, i.e. p2 >= -log2(255 o) - 1e-3. Hence every blending pixel
+// lies in the ellipse d^T (M - sl I) d <= log2(255 o) + 1e-3, whose bounding
+// box is returned, widened by 2% plus 0.05 px to cover the rounding of this
+// computation. Returns an empty box if the Gaussian can never blend and an
+// unbounded one if (M - sl I) is not safely positive definite.
+__device__ __forceinline__ float4 blend_box(float px, float py, float a2, float b2, float c2, float o) {
+  const float kInf = __int_as_float(0x7f800000);
+  const float rho2 = __log2f(255.0f * o) + 1e-3f;
+  if (!(rho2 > 0.0f)) return make_float4(kInf, -kInf, kInf, -kInf);
+  const float K = fmaxf(fabsf(a2), fabsf(c2)) + 0.5f * fabsf(b2);
+  const float sl = 1e-6f * K;
+  const float m00 = -a2 - sl, m11 = -c2 - sl, m01 = -0.5f * b2;
+  const float det = m00 * m11 - m01 * m01;
+  if (!(m00 > 0.0f) || !(m11 > 0.0f) || !(det > 1e-3f * (m00 * m11)))
+    return make_float4(-kInf, kInf, -kInf, kInf);
+  const float hx = sqrtf(rho2 * m11 / det) * 1.02f + 0.05f + 1e-6f * fabsf(px);
+  const float hy = sqrtf(rho2 * m00 / det) * 1.02f + 0.05f + 1e-6f * fabsf(py);
+  return make_float4(px - hx, px + hx, py - hy, py + hy);
+}
+
+__device__ __forceinline__ bool box_hits(const float4 b, float x0, float x1, float y0, float y1) {
+  return b.x <= x1 && b.y >= x0 && b.z <= y1 && b.w >= y0;
+}
+
 struct FwdArgs {
   const float4* xyzo;
   const float4* conic;
@@ -48,13 +80,18 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
   __shared__ float4 s_geo[kBlock];  // px, py, a2, b2
   __shared__ float2 s_co[kBlock];   // c2, opacity
   __shared__ float4 s_rgb[kBlock];
+  __shared__ float4 s_box[kBlock];
   const int tile = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int du, dv;
   tile_pixel(tid, du, dv);
-  const int u = (tile % a.TW) * kTile + du, v = (tile / a.TW) * kTile + dv;
+  const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
+  const int u = tx0 + du, v = ty0 + dv;
   const bool inside = u < a.W && v < a.H;
   const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
+  // pixel-centre extent of this warp's 8x4 block
+  const float wx0 = (float)(tx0 + (warp & 1) * 8) + 0.5f, wx1 = wx0 + 7.0f;
+  const float wy0 = (float)(ty0 + (warp >> 1) * 4) + 0.5f, wy1 = wy0 + 3.0f;
   const uint2 range = a.ranges[tile];
   const int n = (int)(range.y - range.x);
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
@@ -66,14 +103,24 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
       const uint32_t i = a.vals[range.x + base + tid];
       const float4 g = a.xyzo[i];
       const float4 q = a.conic[i];
-      s_geo[tid] = make_float4(g.x, g.y, __fmul_rn(q.x, kHalfNegLog2e), __fmul_rn(q.y, kNegLog2e));
-      s_co[tid] = make_float2(__fmul_rn(q.z, kHalfNegLog2e), g.w);
+      const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
+                  c2 = __fmul_rn(q.z, kHalfNegLog2e);
+      s_geo[tid] = make_float4(g.x, g.y, a2, b2);
+      s_co[tid] = make_float2(c2, g.w);
       s_rgb[tid] = a.rgb[i];
+      s_box[tid] = blend_box(g.x, g.y, a2, b2, c2, g.w);
     }
     __syncthreads();
-    if (!done) {
-      const int m = min(kBlock, n - base);
-      for (int k = 0; k < m; ++k) {
+    const int m = min(kBlock, n - base);
+    for (int c0 = 0; c0 < m; c0 += 32) {
+      if (__all_sync(0xffffffffu, done)) break;
+      const int j = c0 + lane;
+      const bool rel = j < m && box_hits(s_box[j], wx0, wx1, wy0, wy1);
+      unsigned msk = __ballot_sync(0xffffffffu, rel);
+      while (msk) {
+        const int k = c0 + __ffs(msk) - 1;
+        msk &= msk - 1;
+        if (done) continue;
         const float4 g = s_geo[k];
         const float2 co = s_co[k];
         const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
@@ -93,10 +140,7 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
         T = __fmul_rn(T, __fsub_rn(1.0f, alpha));
         ++cnt;
         lst = base + k + 1;
-        if (T < kTMin) {
-          done = true;
-          break;
-        }
+        if (T < kTMin) done = true;
       }
     }
   }
@@ -125,26 +169,76 @@ struct BwdArgs {
   float4* grad2d;  // [n][3]
 };
 
-__device__ __forceinline__ float warp_sum(float v) {
+// Where the multi-value butterfly below leaves its results: lane `lane` ends
+// up holding the warp total of value `idx`, and it is the lane that reports
+// it if `owner` (one lane per value 0..8).
+struct Reduce9Slot {
+  int idx;
+  bool owner;
+};
+__device__ __forceinline__ Reduce9Slot reduce9_slot(int lane) {
+  // Split tree over the value index range: 9 -> (5 | 4), 5 -> (3 | 2), 3 -> (2 | 1),
+  // 2 -> (1 | 1); lanes with the offset bit set take the upper part.
+  int b = 0, hi = 9;
+  const int n1[4] = {5, 3, 2, 1};
+  const int off[4] = {16, 8, 4, 2};
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+  for (int l = 0; l < 4; ++l) {
+    if (lane & off[l]) b += n1[l];
+    else hi = min(hi, b + n1[l]);
+  }
+  return Reduce9Slot{b, b < hi && (lane & 1) == 0};
+}
+
+// Sum v[0..8] over the warp with 12 shuffles (instead of 45): at each level a
+// lane keeps one half of its values and trades the other half with its
+// partner. Returns the total of value reduce9_slot(lane).idx.
+__device__ __forceinline__ float warp_reduce9(const float v[9], int lane) {
+  const bool u1 = lane & 16, u2 = lane & 8, u3 = lane & 4, u4 = lane & 2;
+  float w1[5];
+#pragma unroll
+  for (int j = 0; j < 5; ++j) {
+    const float lo = v[j], up = j + 5 < 9 ? v[j + 5] : 0.0f;
+    const float r = __shfl_xor_sync(0xffffffffu, u1 ? lo : up, 16);
+    w1[j] = (u1 ? up : lo) + r;
+  }
+  float w2[3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const float lo = w1[j], up = j + 3 < 5 ? w1[j + 3] : 0.0f;
+    const float r = __shfl_xor_sync(0xffffffffu, u2 ? lo : up, 8);
+    w2[j] = (u2 ? up : lo) + r;
+  }
+  float w3[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float lo = w2[j], up = j + 2 < 3 ? w2[j + 2] : 0.0f;
+    const float r = __shfl_xor_sync(0xffffffffu, u3 ? lo : up, 4);
+    w3[j] = (u3 ? up : lo) + r;
+  }
+  const float r4 = __shfl_xor_sync(0xffffffffu, u4 ? w3[0] : w3[1], 2);
+  const float w4 = (u4 ? w3[1] : w3[0]) + r4;
+  return w4 + __shfl_xor_sync(0xffffffffu, w4, 1);
 }
 
 __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
   __shared__ float4 s_geo[kBlock];  // px, py, a2, b2
   __shared__ float4 s_co[kBlock];   // c2, opacity, A, B
   __shared__ float4 s_rgb[kBlock];  // r, g, b, C
+  __shared__ float4 s_box[kBlock];
+  __shared__ float s_acc[kBlock][9];  // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
   __shared__ uint32_t s_idx[kBlock];
   __shared__ int s_maxlast;
   const int tile = blockIdx.x;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int du, dv;
   tile_pixel(tid, du, dv);
-  const int u = (tile % a.TW) * kTile + du, v = (tile / a.TW) * kTile + dv;
+  const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
+  const int u = tx0 + du, v = ty0 + dv;
   const bool inside = u < a.W && v < a.H;
   const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
+  const float wx0 = (float)(tx0 + (warp & 1) * 8) + 0.5f, wx1 = wx0 + 7.0f;
+  const float wy0 = (float)(ty0 + (warp >> 1) * 4) + 0.5f, wy1 = wy0 + 3.0f;
   const uint2 range = a.ranges[tile];
   const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
   float T = 1.0f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
@@ -156,14 +250,16 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
     g1 = a.dL_dimage[P + pix];
     g2 = a.dL_dimage[2 * P + pix];
   }
+  const int warp_last = __reduce_max_sync(0xffffffffu, my_last);
+  const Reduce9Slot slot = reduce9_slot(lane);
   float R0 = a.bg0, R1 = a.bg1, R2 = a.bg2;
   if (tid == 0) s_maxlast = 0;
   __syncthreads();
-  if (my_last > 0) atomicMax(&s_maxlast, my_last);
+  if (lane == 0 && warp_last > 0) atomicMax(&s_maxlast, warp_last);
   __syncthreads();
   const int n = s_maxlast;  // list offsets [0, n) can hold a blend
   for (int done = 0; done < n; done += kBlock) {
-    // this batch covers list offsets n-1-done down to max(0, n-done-kBlock)
+    // slot k of this batch holds list offset n - 1 - done - k (back to front)
     __syncthreads();
     const int off = n - 1 - done - tid;
     if (off >= 0) {
@@ -171,70 +267,85 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
       const float4 g = a.xyzo[i];
       const float4 q = a.conic[i];
       const float4 c = a.rgb[i];
-      s_geo[tid] = make_float4(g.x, g.y, __fmul_rn(q.x, kHalfNegLog2e), __fmul_rn(q.y, kNegLog2e));
-      s_co[tid] = make_float4(__fmul_rn(q.z, kHalfNegLog2e), g.w, q.x, q.y);
+      const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
+                  c2 = __fmul_rn(q.z, kHalfNegLog2e);
+      s_geo[tid] = make_float4(g.x, g.y, a2, b2);
+      s_co[tid] = make_float4(c2, g.w, q.x, q.y);
       s_rgb[tid] = make_float4(c.x, c.y, c.z, q.z);
+      s_box[tid] = blend_box(g.x, g.y, a2, b2, c2, g.w);
       s_idx[tid] = i;
     }
+#pragma unroll
+    for (int j = 0; j < 9; ++j) s_acc[tid][j] = 0.0f;
     __syncthreads();
     const int m = min(kBlock, n - done);
-    for (int k = 0; k < m; ++k) {
-      const int offk = n - 1 - done - k;
-      bool contrib = offk < my_last;
-      float dpx = 0.f, dpy = 0.f, dop = 0.f, dA = 0.f, dB = 0.f, dC = 0.f, dr = 0.f, dg = 0.f, db = 0.f;
-      if (contrib) {
-        const float4 g = s_geo[k];
-        const float4 co = s_co[k];
-        const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
-        float qv = __fmul_rn(g.z, dx);
-        qv = __fmaf_rn(g.w, dy, qv);
-        float p2 = __fmul_rn(dx, qv);
-        const float wv = __fmul_rn(co.x, dy);
-        p2 = __fmaf_rn(wv, dy, p2);
-        const float e = exp2_raster(p2);
-        const float vv = __fmul_rn(co.y, e);
-        const float alpha = fminf(vv, kAlphaMax);
-        contrib = alpha >= kAlphaMin;
-        if (contrib) {
-          const float4 c = s_rgb[k];
-          const float oma = 1.0f - alpha;
-          T = T / oma;  // transmittance in front of this Gaussian
-          const float wgt = alpha * T;
-          dr = g0 * wgt;
-          dg = g1 * wgt;
-          db = g2 * wgt;
-          const float Gk = T * (g0 * (c.x - R0) + g1 * (c.y - R1) + g2 * (c.z - R2));
-          if (vv < kAlphaMax) {
-            dop = Gk * e;
-            const float dp = Gk * alpha;
-            const float A = co.z, B = co.w, Cc = c.w;
-            dpx = -dp * fmaf(A, dx, B * dy);
-            dpy = -dp * fmaf(B, dx, Cc * dy);
-            dA = -0.5f * dp * dx * dx;
-            dB = -dp * dx * dy;
-            dC = -0.5f * dp * dy * dy;
+    for (int c0 = 0; c0 < m; c0 += 32) {
+      const int j = c0 + lane;
+      const bool rel = j < m && (n - 1 - done - j) < warp_last && box_hits(s_box[j], wx0, wx1, wy0, wy1);
+      unsigned msk = __ballot_sync(0xffffffffu, rel);
+      while (msk) {
+        const int k = c0 + __ffs(msk) - 1;
+        msk &= msk - 1;
+        const int offk = n - 1 - done - k;
+        float gv[9] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        bool contrib = false;
+        if (offk < my_last) {
+          const float4 g = s_geo[k];
+          const float4 co = s_co[k];
+          const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
+          float qv = __fmul_rn(g.z, dx);
+          qv = __fmaf_rn(g.w, dy, qv);
+          float p2 = __fmul_rn(dx, qv);
+          const float wv = __fmul_rn(co.x, dy);
+          p2 = __fmaf_rn(wv, dy, p2);
+          const float e = exp2_raster(p2);
+          const float vv = __fmul_rn(co.y, e);
+          const float alpha = fminf(vv, kAlphaMax);
+          contrib = alpha >= kAlphaMin;
+          if (contrib) {
+            const float4 c = s_rgb[k];
+            const float oma = 1.0f - alpha;
+            T = T / oma;  // transmittance in front of this Gaussian
+            const float wgt = alpha * T;
+            gv[6] = g0 * wgt;
+            gv[7] = g1 * wgt;
+            gv[8] = g2 * wgt;
+            const float Gk = T * (g0 * (c.x - R0) + g1 * (c.y - R1) + g2 * (c.z - R2));
+            if (vv < kAlphaMax) {
+              gv[2] = Gk * e;
+              const float dp = Gk * alpha;
+              const float A = co.z, B = co.w, Cc = c.w;
+              gv[0] = -dp * fmaf(A, dx, B * dy);
+              gv[1] = -dp * fmaf(B, dx, Cc * dy);
+              gv[3] = -0.5f * dp * dx * dx;
+              gv[4] = -dp * dx * dy;
+              gv[5] = -0.5f * dp * dy * dy;
+            }
+            R0 = fmaf(c.x, alpha, oma * R0);
+            R1 = fmaf(c.y, alpha, oma * R1);
+            R2 = fmaf(c.z, alpha, oma * R2);
           }
-          R0 = fmaf(c.x, alpha, oma * R0);
-          R1 = fmaf(c.y, alpha, oma * R1);
-          R2 = fmaf(c.z, alpha, oma * R2);
+        }
+        if (__any_sync(0xffffffffu, contrib)) {
+          const float tot = warp_reduce9(gv, lane);
+          if (slot.owner) atomicAdd(&s_acc[k][slot.idx], tot);
         }
       }
-      if (__any_sync(0xffffffffu, contrib)) {
-        dpx = warp_sum(dpx);
-        dpy = warp_sum(dpy);
-        dop = warp_sum(dop);
-        dA = warp_sum(dA);
-        dB = warp_sum(dB);
-        dC = warp_sum(dC);
-        dr = warp_sum(dr);
-        dg = warp_sum(dg);
-        db = warp_sum(db);
-        if (lane == 0) {
-          float4* dst = a.grad2d + 3 * (size_t)s_idx[k];
-          atomicAdd(dst, make_float4(dpx, dpy, dop, 0.f));
-          atomicAdd(dst + 1, make_float4(dA, dB, dC, 0.f));
-          atomicAdd(dst + 2, make_float4(dr, dg, db, 0.f));
-        }
+    }
+    __syncthreads();
+    if (tid < m) {
+      float r[9];
+      bool any = false;
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        r[j] = s_acc[tid][j];
+        any |= r[j] != 0.0f;
+      }
+      if (any) {
+        float4* dst = a.grad2d + 3 * (size_t)s_idx[tid];
+        atomicAdd(dst, make_float4(r[0], r[1], r[2], 0.f));
+        atomicAdd(dst + 1, make_float4(r[3], r[4], r[5], 0.f));
+        atomicAdd(dst + 2, make_float4(r[6], r[7], r[8], 0.f));
       }
     }
   }

@@ -127,6 +127,8 @@ class Rasterizer:
         self.culled = False
         # Optional per-stage CUDA-event timing: {stage: [(start, end), ...]}.
         self.stage_events = None
+        # Also produce the record-order scan of tiles_touched (gs_bin_sort offsets).
+        self.want_offsets = False
 
     def _timed(self, stage):
         ev = self.stage_events
@@ -164,11 +166,12 @@ class Rasterizer:
             return self._bin_sort(cam)
 
     def _bin_sort(self, cam: gs.GsCamera) -> int:
-        st, ni = gs.gs_bin_sort(self._proj, self.N, cam, self.offsets, self.keys, self.vals, self.capacity,
+        offs = self.offsets if self.want_offsets else None
+        st, ni = gs.gs_bin_sort(self._proj, self.N, cam, offs, self.keys, self.vals, self.capacity,
                                 self.ranges, self.sort_ws, raise_on_capacity=False)
         if st == gs.GS_ERR_CAPACITY:
             self._ensure_capacity(int(ni * 1.25) + 1024)
-            st, ni = gs.gs_bin_sort(self._proj, self.N, cam, self.offsets, self.keys, self.vals,
+            st, ni = gs.gs_bin_sort(self._proj, self.N, cam, offs, self.keys, self.vals,
                                     self.capacity, self.ranges, self.sort_ws)
         self.n_instances = ni
         return ni

@@ -134,14 +134,18 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
                          const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
                          const gs_projected* out, void* stream);
 
-/* Tile binning: exclusive scan of tiles_touched into offsets, emission of one
- * (key, value) per (Gaussian, tile) with key = (tile_id << 32) | bits(depth),
- * value = record index, tiles in row-major order within the rect; stable LSD
- * radix sort (8-bit digits, onesweep with decoupled look-back) over the key
- * bits [0, 32 + ceil(log2(TW*TH))); then [start, end) per tile into
- * tile_ranges (empty tiles [0, 0)).
+/* Tile binning: one (key, value) per (Gaussian, tile) instance with
+ * key = (tile_id << 32) | bits(depth) and value = record index, tiles in
+ * row-major order within the record's rect, sorted stably by key (equal keys
+ * keep record order), then [start, end) per tile into tile_ranges (empty tiles
+ * [0, 0)). The sort is an LSD radix sort with 8-bit digits (onesweep passes
+ * with decoupled look-back): the 32 depth bits are sorted once per Gaussian,
+ * the instances are emitted in that order, and only the ceil(log2(TW*TH)) tile
+ * bits are sorted over the instances, which gives the same order as sorting
+ * all key bits of every instance.
  *   in           [host] struct of [device] records, n entries
- *   offsets      [device] [n] i32 out
+ *   offsets      [device] [n] i32 out, or NULL: exclusive scan of
+ *                tiles_touched in record order
  *   keys, vals   [device] [capacity] out, sorted
  *   capacity     size of keys/vals, < 2^30
  *   tile_ranges  [device] [TW*TH][2] u32 out
@@ -149,7 +153,7 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
  * Synchronous: waits on `stream` once to read I and once at the end to read
  * the device status. Returns GS_ERR_CAPACITY (with *n_instances set, nothing
  * sorted) when I > capacity, GS_ERR_DEVICE_TIMEOUT if a look-back wait hit its
- * iteration limit. */
+ * iteration limit (tile_ranges are then all empty). */
 GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
                        uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
                        int64_t* n_instances, void* workspace, size_t* workspace_bytes,

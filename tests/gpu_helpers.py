@@ -12,6 +12,7 @@ def gpu_forward(scene, pose=0, capacity=None):
     cam = scene.cameras[pose]
     params = GaussianParams.from_scene(scene)
     R = Rasterizer(scene.N, scene.sh_degree, cam.width, cam.height, capacity=capacity)
+    R.want_offsets = True
     R.forward(params, cam, scene.bg, scene.lod_dist, scene.importance_q)
     torch.cuda.synchronize()
     return R

@@ -79,6 +79,7 @@ def test_stagewise_sort_and_raster_from_oracle_records():
     cam = sc.cameras[0]
     ref = oracle.render(sc)
     R = Rasterizer(sc.N, sc.sh_degree, cam.width, cam.height)
+    R.want_offsets = True
     load_records(R, ref["rec"])
     c = gs.camera(cam)
     R.bin_sort(c)
@@ -279,3 +280,17 @@ def test_invalid_arguments_rejected():
     assert ei.value.status == gs.GS_ERR_INVALID_ARGUMENT
     with pytest.raises(gs.GsError):
         gs.gs_cull(params.means, None, 10, c, 0.0, 0.5, R.mask, R.active_idx, R.n_active, R.cull_ws)
+
+
+def test_equal_depths_keep_record_order():
+    # every Gaussian at the same camera depth: the sort must break ties by record index
+    cam = simple_camera(160, 96, 60.0)
+    rng = np.random.default_rng(7)
+    N = 3000
+    means = np.stack([rng.uniform(-2.5, 2.5, N), rng.uniform(-1.5, 1.5, N), np.full(N, 2.0)]).astype(np.float32)
+    sc = make_scene(means, rng.normal(-3.0, 0.4, (3, N)), rng.standard_normal((4, N)), rng.normal(0, 1, N),
+                    rng.uniform(-1, 1, (3, N)), 0, [cam])
+    R, ref = _full_compare(sc)
+    depths = ref["rec"]["xyzo"][ref["rec"]["tiles"] > 0, 2]
+    assert np.unique(depths).size < 10  # mostly one depth value
+    assert R.n_instances > 2 * 4096  # several sort tiles

@@ -25,7 +25,8 @@ GS_ERR_UNSUPPORTED = 5
 
 EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_bin_sort",
             "gs_rasterize_fwd", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
-            "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches"]
+            "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
+GS_CULL_NOALLOC_MAX_N = 16777216
 
 
 class GsError(RuntimeError):
@@ -81,6 +82,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_preprocess_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P,
                                         P, P, P, P, P, P]
         L.gs_rasterize_bwd_2d.argtypes = [PPROJ, I64, P, P, PCAM, P, P, P, P, P, P]
+        L.gs_cull_noalloc.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P]
+        L.gs_cull_noalloc.restype = ctypes.c_int
         L.gs_debug_kernel_launches.restype = ctypes.c_int64
         L.gs_debug_kernel_launches.argtypes = []
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
@@ -142,6 +145,14 @@ def gs_cull(means, importance, N, cam: GsCamera, lod_dist, importance_q, mask, a
                                      float(lod_dist), float(importance_q), _p(mask), _p(active_idx),
                                      _p(n_active), _p(workspace), ctypes.byref(nbytes), _stream(stream)))
     return nbytes.value
+
+
+def gs_cull_noalloc(means, importance, N, cam: GsCamera, lod_dist, importance_q, mask, active_idx,
+                    n_active, stream=None):
+    """gs_cull with the library's own static scratch (no workspace argument)."""
+    _check("gs_cull_noalloc", load().gs_cull_noalloc(
+        _p(means), _p(importance), int(N), ctypes.byref(cam), float(lod_dist), float(importance_q),
+        _p(mask), _p(active_idx), _p(n_active), _stream(stream)))
 
 
 def gs_cull_workspace(N, cam: GsCamera) -> int:

@@ -113,6 +113,27 @@ GS_API int gs_cull(const float* means, const float* importance, int64_t N, const
                    float lod_dist, float importance_q, uint8_t* mask, int32_t* active_idx,
                    int32_t* n_active, void* workspace, size_t* workspace_bytes, void* stream);
 
+/* gs_cull without a workspace, for callers that cannot allocate device
+ * memory: a plugin inside a host application that does not own the device
+ * allocator, or a real-time loop that may not call cudaMalloc (it synchronises
+ * the whole device). The pages have no counterpart of this entry point; it is
+ * an interface convenience over gs_cull, whose results it reproduces exactly.
+ * Its scratch is a 32 KiB array in the library image, which every GPU that
+ * loads the library holds until the process exits. The call allocates
+ * nothing.
+ *   arguments    as for gs_cull, without workspace/workspace_bytes
+ *   N            at most GS_CULL_NOALLOC_MAX_N; larger N returns
+ *                GS_ERR_INVALID_ARGUMENT (use gs_cull with a workspace)
+ * The first call made with a given device current looks up the array's device
+ * address (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture on the device. Every call shares the one array: each
+ * clears what must start at zero, but calls that overlap on the GPU (other
+ * streams or host threads) race on it. Asynchronous otherwise. */
+#define GS_CULL_NOALLOC_MAX_N 16777216
+GS_API int gs_cull_noalloc(const float* means, const float* importance, int64_t N, const gs_camera* cam,
+                           float lod_dist, float importance_q, uint8_t* mask, int32_t* active_idx,
+                           int32_t* n_active, void* stream);
+
 /* Projection of every active Gaussian into records (EWA splatting):
  *   t = R mu + t, culled unless t.z > near_z; s = exp(log_s); q normalised;
  *   Sigma = Rq S S^T Rq^T; J = d(pinhole)/dt at t;

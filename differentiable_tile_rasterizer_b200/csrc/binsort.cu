@@ -58,6 +58,7 @@ struct SortWs {
   uint32_t* dkey[2];   // [n] depth keys
   uint32_t* dval[2];   // [n] record indices
   int32_t* doff;       // [n] instance offsets in depth order
+  int32_t* dtiles;     // [n] tiles_touched in depth order
   uint32_t* tkey[2];   // [capacity] tile ids
   uint32_t* tval[2];   // [capacity] record indices
 };
@@ -89,6 +90,8 @@ SortWs carve(void* ws, const BinSortPlan& p) {
     c += align256((size_t)p.n * sizeof(uint32_t));
   }
   w.doff = reinterpret_cast<int32_t*>(c);
+  c += align256((size_t)p.n * sizeof(int32_t));
+  w.dtiles = reinterpret_cast<int32_t*>(c);
   c += align256((size_t)p.n * sizeof(int32_t));
   for (int k = 0; k < 2; ++k) {
     w.tkey[k] = reinterpret_cast<uint32_t*>(c);
@@ -163,22 +166,59 @@ __global__ void __launch_bounds__(256) depth_keys_kernel(const float4* xyzo, con
   val[i] = (uint32_t)i;
 }
 
-// Instances of the r-th Gaussian in depth order, tiles row-major in its rect.
+// Instances of the Gaussians in depth order, tiles row-major in each rect.
+// A warp writes the instances of its 32 consecutive Gaussians as one
+// contiguous run (their offsets are consecutive), each lane finding the
+// Gaussian of its instance by a binary search over the warp's prefix sums,
+// so the stores coalesce however many tiles each Gaussian touches.
 __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const int32_t* doff,
-                                                   const ushort4* rect, const int32_t* tiles, int64_t n,
+                                                   const int32_t* dtiles, const ushort4* rect, int64_t n,
                                                    int TW, uint32_t* tkey, uint32_t* tval) {
   const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= n) return;
-  const uint32_t i = order[r];
-  if (tiles[i] <= 0) return;
-  int64_t off = doff[r];
-  const ushort4 b = rect[i];
-  for (int ty = b.y; ty < b.w; ++ty)
-    for (int tx = b.x; tx < b.z; ++tx) {
-      tkey[off] = (uint32_t)(ty * TW + tx);
-      tval[off] = i;
-      ++off;
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = r - lane;
+  if (r0 >= n) return;  // warp-uniform
+  int t = 0, x0 = 0, y0 = 0, bw = 1;
+  uint32_t i = 0;
+  if (r < n) {
+    t = dtiles[r];
+    if (t > 0) {
+      i = order[r];
+      const ushort4 b = rect[i];
+      x0 = b.x;
+      y0 = b.y;
+      bw = (int)b.z - (int)b.x;
     }
+  }
+  const int64_t base = doff[r0];
+  int inc = t;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  const int ex = inc - t;
+  const int total = __shfl_sync(0xffffffffu, inc, 31);
+  for (int p0 = 0; p0 < total; p0 += 32) {
+    const int q = p0 + lane;
+    int L = 0;
+#pragma unroll
+    for (int st = 16; st > 0; st >>= 1) {
+      const int c = L + st;
+      if (__shfl_sync(0xffffffffu, ex, c) <= q) L = c;
+    }
+    const int exL = __shfl_sync(0xffffffffu, ex, L);
+    const uint32_t iL = __shfl_sync(0xffffffffu, i, L);
+    const int x0L = __shfl_sync(0xffffffffu, x0, L);
+    const int y0L = __shfl_sync(0xffffffffu, y0, L);
+    const int bwL = __shfl_sync(0xffffffffu, bw, L);
+    if (q < total) {
+      const int li = q - exL;
+      const int row = li / bwL;
+      tkey[base + q] = (uint32_t)((y0L + row) * TW + x0L + (li - row * bwL));
+      tval[base + q] = iL;
+    }
+  }
 }
 
 // Digit histograms of `passes` passes (digit p = bits [8p, 8p + 8)).
@@ -213,6 +253,8 @@ struct PassArgs {
   uint32_t* vout;
   uint64_t* kout64;           // final pass: (tile << 32) | depth bits of the record
   const float4* xyzo;         // records, for the depth bits of the final keys
+  const int32_t* tiles_in;    // optional: also write tiles_out[out] = tiles_in[value]
+  int32_t* tiles_out;
   int64_t n;
   int shift;
   const uint32_t* digit_off;  // [256] exclusive global digit offsets
@@ -324,6 +366,7 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
       a.kout[out] = k;
     }
     a.vout[out] = v;
+    if (a.tiles_out) a.tiles_out[out] = a.tiles_in[v];
   }
 }
 
@@ -354,8 +397,8 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, int64
 // ping-ponging between (k0, v0) and (k1, v1); the last pass writes to
 // (last_k or last_k64, last_v). Returns the kernels launched, -1 on error.
 int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint32_t* v1, int64_t n, int passes,
-                uint32_t* last_k, uint64_t* last_k64, uint32_t* last_v, const float4* xyzo, int64_t stall,
-                cudaStream_t s) {
+                uint32_t* last_k, uint64_t* last_k64, uint32_t* last_v, const float4* xyzo,
+                const int32_t* tiles_in, int32_t* tiles_out, int64_t stall, cudaStream_t s) {
   if (cudaMemsetAsync(w.hist, 0, kMaxPasses * kRadix * sizeof(uint32_t), s) != cudaSuccess) return -1;
   const int64_t nt = sort_tiles(n);
   if (cudaMemsetAsync(w.counters, 0, (64 + (size_t)passes * nt * kRadix) * sizeof(uint32_t), s) != cudaSuccess)
@@ -374,6 +417,8 @@ int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint3
     a.kout64 = last ? last_k64 : nullptr;
     a.vout = last ? last_v : vb[(p + 1) & 1];
     a.xyzo = xyzo;
+    a.tiles_in = tiles_in;
+    a.tiles_out = last ? tiles_out : nullptr;
     a.n = n;
     a.shift = 8 * p;
     a.digit_off = w.hist + p * kRadix;
@@ -400,7 +445,7 @@ BinSortPlan binsort_plan(int64_t n, int64_t capacity, int64_t tiles) {
   p.passes = (tb + 7) / 8;  // tile-digit passes over the instances
   p.bytes = align256((size_t)(scan_blocks(n) + 1) * sizeof(int64_t)) + 256 + 256 +
             align256(kMaxPasses * kRadix * sizeof(uint32_t)) + align256(lookback_words(p) * sizeof(uint32_t)) +
-            4 * align256((size_t)n * sizeof(uint32_t)) + align256((size_t)n * sizeof(int32_t)) +
+            4 * align256((size_t)n * sizeof(uint32_t)) + 2 * align256((size_t)n * sizeof(int32_t)) +
             4 * align256((size_t)capacity * sizeof(uint32_t));
   return p;
 }
@@ -421,22 +466,21 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
     scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, nullptr, n, w.partials, offsets);
     launched += 3;
   }
-  const uint32_t* order = nullptr;
   if (n > 0) {
     depth_keys_kernel<<<grid_for(n, 256), 256, 0, s>>>(rec.xyzo, rec.tiles, n, w.dkey[0], w.dval[0]);
     // 4 passes: dkey[0] -> [1] -> [0] -> [1] -> [0]
+    // the last pass also writes tiles_touched in depth order (dtiles)
     const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, kDepthPasses, w.dkey[0],
-                              nullptr, w.dval[0], rec.xyzo, stall_tile, s);
+                              nullptr, w.dval[0], rec.xyzo, rec.tiles, w.dtiles, stall_tile, s);
     if (k < 0) return cudaErrorLaunchFailure;
     launched += 1 + k;
-    order = w.dval[0];
-    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, order, n, w.partials);
+    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials);
     launched += 1;
   }
   scan_partials_kernel<<<1, 1024, 0, s>>>(w.partials, nb, w.total);
   launched += 1;
   if (nb > 0) {
-    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, order, n, w.partials, w.doff);
+    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials, w.doff);
     launched += 1;
   }
   count_launches(launched);
@@ -450,7 +494,7 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
   const int64_t TT = (int64_t)cam.TW * cam.TH;
   cudaError_t e = cudaMemsetAsync(ranges, 0, (size_t)TT * 2 * sizeof(uint32_t), s);
   if (e != cudaSuccess || n_inst == 0) return e;
-  emit_kernel<<<grid_for(n, 256), 256, 0, s>>>(w.dval[0], w.doff, rec.rect, rec.tiles, n, cam.TW, w.tkey[0],
+  emit_kernel<<<grid_for(n, 256), 256, 0, s>>>(w.dval[0], w.doff, w.dtiles, rec.rect, n, cam.TW, w.tkey[0],
                                                w.tval[0]);
   int launched = 1;
   if (plan.passes == 0) {
@@ -458,7 +502,7 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
     ++launched;
   } else {
     const int k = sort_passes(w, w.tkey[0], w.tval[0], w.tkey[1], w.tval[1], n_inst, plan.passes, nullptr, keys,
-                              vals, rec.xyzo, stall_tile, s);
+                              vals, rec.xyzo, nullptr, nullptr, stall_tile, s);
     if (k < 0) return cudaErrorLaunchFailure;
     launched += k;
   }

@@ -169,6 +169,8 @@ __device__ __forceinline__ void project(const Params& p, const DevCam& cam, int6
     const float v = __fadd_rn(acc, 0.5f);
     o.rgb[ch] = v > 0.0f ? v : 0.0f;
   }
+  // an infinite colour (from infinite SH coefficients) culls, like a non-finite parameter
+  if (!(finitef(o.rgb[0]) && finitef(o.rgb[1]) && finitef(o.rgb[2]))) return;
   o.visible = true;
   o.px = px; o.py = py; o.depth = tz; o.opacity = op;
   o.A = cA; o.B = cB; o.C = cC; o.rf = rf;

@@ -21,6 +21,16 @@ namespace {
 
 constexpr int kTile = 16;
 constexpr int kBlock = kTile * kTile;
+#ifndef GS_RASTER_BATCH_FWD
+#define GS_RASTER_BATCH_FWD 256
+#endif
+#ifndef GS_RASTER_BATCH_BWD
+#define GS_RASTER_BATCH_BWD 256
+#endif
+// List entries staged in shared memory per CTA-wide step.
+constexpr int kBatchF = GS_RASTER_BATCH_FWD;
+constexpr int kBatchB = GS_RASTER_BATCH_BWD;
+static_assert(kBatchF % 32 == 0 && kBatchB % 32 == 0 && kBatchF >= kBlock && kBatchB >= kBlock, "batch: warp multiple, at least one block");
 
 // Pixel of thread `tid` in the tile: warp w covers the 8x4 block at
 // ((w & 1) * 8, (w >> 1) * 4).
@@ -41,25 +51,48 @@ __device__ __forceinline__ void tile_pixel(int tid, int& du, int& dv) {
 // up to ~2 ulp, i.e. p2 >= -log2(255 o) - 1e-3. Hence every blending pixel
 // lies in the ellipse d^T (M - sl I) d <= log2(255 o) + 1e-3, whose bounding
 // box is returned, widened by 2% plus 0.05 px to cover the rounding of this
-// computation. Returns an empty box if the Gaussian can never blend and an
-// unbounded one if (M - sl I) is not safely positive definite.
-__device__ __forceinline__ float4 blend_box(float px, float py, float a2, float b2, float c2, float o) {
+// computation. The same ellipse also lies in the disk of radius
+// sqrt(rho2 / lambda_min) around the centre; that disk is used too when the
+// ellipse is not elongated (lambda_min > lambda_max / 100, so lambda_min is
+// accurate in fp32), widened the same way. The region is returned as
+// (px, py, half-width, half-height) and the squared disk radius; an empty
+// region (negative half-widths) if the Gaussian can never blend, an unbounded
+// one if (M - sl I) is not safely positive definite.
+struct BlendRegion {
+  float4 box;  // px, py, hx, hy
+  float rc2;   // squared disk radius
+};
+
+__device__ __forceinline__ BlendRegion blend_region(float px, float py, float a2, float b2, float c2, float o) {
   const float kInf = __int_as_float(0x7f800000);
   const float rho2 = __log2f(255.0f * o) + 1e-3f;
-  if (!(rho2 > 0.0f)) return make_float4(kInf, -kInf, kInf, -kInf);
+  if (!(rho2 > 0.0f)) return BlendRegion{make_float4(px, py, -kInf, -kInf), -kInf};
   const float K = fmaxf(fabsf(a2), fabsf(c2)) + 0.5f * fabsf(b2);
   const float sl = 1e-6f * K;
   const float m00 = -a2 - sl, m11 = -c2 - sl, m01 = -0.5f * b2;
   const float det = m00 * m11 - m01 * m01;
   if (!(m00 > 0.0f) || !(m11 > 0.0f) || !(det > 1e-3f * (m00 * m11)))
-    return make_float4(-kInf, kInf, -kInf, kInf);
-  const float hx = sqrtf(rho2 * m11 / det) * 1.02f + 0.05f + 1e-6f * fabsf(px);
-  const float hy = sqrtf(rho2 * m00 / det) * 1.02f + 0.05f + 1e-6f * fabsf(py);
-  return make_float4(px - hx, px + hx, py - hy, py + hy);
+    return BlendRegion{make_float4(px, py, kInf, kInf), kInf};
+  const float pad = 0.05f + 1e-6f * (fabsf(px) + fabsf(py));
+  const float hx = sqrtf(rho2 * m11 / det) * 1.02f + pad;
+  const float hy = sqrtf(rho2 * m00 / det) * 1.02f + pad;
+  const float half_tr = 0.5f * (m00 + m11);
+  const float disc = sqrtf(0.25f * (m00 - m11) * (m00 - m11) + m01 * m01);
+  const float lmin = half_tr - disc;
+  float rc2 = kInf;
+  if (lmin > 0.01f * (half_tr + disc)) {
+    const float rc = sqrtf(rho2 / lmin) * 1.02f + pad;
+    rc2 = rc * rc;
+  }
+  return BlendRegion{make_float4(px, py, hx, hy), rc2};
 }
 
-__device__ __forceinline__ bool box_hits(const float4 b, float x0, float x1, float y0, float y1) {
-  return b.x <= x1 && b.y >= x0 && b.z <= y1 && b.w >= y0;
+// Can the Gaussian of region (b, rc2) blend at a pixel centre of the warp
+// block with centre (wcx, wcy) and half extents (3.5, 1.5)?
+__device__ __forceinline__ bool region_hits(const float4 b, float rc2, float wcx, float wcy) {
+  const float ex = fabsf(b.x - wcx) - 3.5f, ey = fabsf(b.y - wcy) - 1.5f;
+  const float qx = fmaxf(ex, 0.0f), qy = fmaxf(ey, 0.0f);
+  return ex <= b.z && ey <= b.w && qx * qx + qy * qy <= rc2;
 }
 
 struct FwdArgs {
@@ -77,10 +110,11 @@ struct FwdArgs {
 };
 
 __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
-  __shared__ float4 s_geo[kBlock];  // px, py, a2, b2
-  __shared__ float2 s_co[kBlock];   // c2, opacity
-  __shared__ float4 s_rgb[kBlock];
-  __shared__ float4 s_box[kBlock];
+  __shared__ float4 s_geo[kBatchF];  // px, py, a2, b2
+  __shared__ float2 s_co[kBatchF];   // c2, opacity
+  __shared__ float4 s_rgb[kBatchF];
+  __shared__ float4 s_box[kBatchF];  // px, py, hx, hy of the blend region
+  __shared__ float s_rc2[kBatchF];
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int du, dv;
@@ -89,40 +123,45 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
   const int u = tx0 + du, v = ty0 + dv;
   const bool inside = u < a.W && v < a.H;
   const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
-  // pixel-centre extent of this warp's 8x4 block
-  const float wx0 = (float)(tx0 + (warp & 1) * 8) + 0.5f, wx1 = wx0 + 7.0f;
-  const float wy0 = (float)(ty0 + (warp >> 1) * 4) + 0.5f, wy1 = wy0 + 3.0f;
+  // centre of this warp's 8x4 block of pixel centres
+  const float wcx = (float)(tx0 + (warp & 1) * 8) + 4.0f;
+  const float wcy = (float)(ty0 + (warp >> 1) * 4) + 2.0f;
   const uint2 range = a.ranges[tile];
   const int n = (int)(range.y - range.x);
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int cnt = 0, lst = 0;
   bool done = !inside;
-  for (int base = 0; base < n; base += kBlock) {
+  for (int base = 0; base < n; base += kBatchF) {
     if (__syncthreads_count(done) == kBlock) break;
-    if (base + tid < n) {
-      const uint32_t i = a.vals[range.x + base + tid];
+    for (int e = tid; e < kBatchF && base + e < n; e += kBlock) {
+      const uint32_t i = a.vals[range.x + base + e];
       const float4 g = a.xyzo[i];
       const float4 q = a.conic[i];
       const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
                   c2 = __fmul_rn(q.z, kHalfNegLog2e);
-      s_geo[tid] = make_float4(g.x, g.y, a2, b2);
-      s_co[tid] = make_float2(c2, g.w);
-      s_rgb[tid] = a.rgb[i];
-      s_box[tid] = blend_box(g.x, g.y, a2, b2, c2, g.w);
+      s_geo[e] = make_float4(g.x, g.y, a2, b2);
+      s_co[e] = make_float2(c2, g.w);
+      s_rgb[e] = a.rgb[i];
+      const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
+      s_box[e] = r.box;
+      s_rc2[e] = r.rc2;
     }
     __syncthreads();
-    const int m = min(kBlock, n - base);
+    const int m = min(kBatchF, n - base);
     for (int c0 = 0; c0 < m; c0 += 32) {
       if (__all_sync(0xffffffffu, done)) break;
       const int j = c0 + lane;
-      const bool rel = j < m && box_hits(s_box[j], wx0, wx1, wy0, wy1);
+      const bool rel = j < m && region_hits(s_box[j], s_rc2[j], wcx, wcy);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
+      // Branch-free body: a lane that skips the pair (alpha < 1/255) or has
+      // already stopped blends with alpha 0, which leaves C, T and the counts
+      // exactly as they were (colours are finite), so the warp never diverges.
       while (msk) {
         const int k = c0 + __ffs(msk) - 1;
         msk &= msk - 1;
-        if (done) continue;
         const float4 g = s_geo[k];
         const float2 co = s_co[k];
+        const float4 c = s_rgb[k];
         const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
         float qv = __fmul_rn(g.z, dx);
         qv = __fmaf_rn(g.w, dy, qv);
@@ -131,16 +170,16 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
         p2 = __fmaf_rn(wv, dy, p2);
         const float e = exp2_raster(p2);
         const float alpha = fminf(__fmul_rn(co.y, e), kAlphaMax);
-        if (alpha < kAlphaMin) continue;
-        const float4 c = s_rgb[k];
-        const float wgt = __fmul_rn(alpha, T);
+        const bool blend = !done && alpha >= kAlphaMin;
+        const float ab = blend ? alpha : 0.0f;
+        const float wgt = __fmul_rn(ab, T);
         C0 = __fmaf_rn(wgt, c.x, C0);
         C1 = __fmaf_rn(wgt, c.y, C1);
         C2 = __fmaf_rn(wgt, c.z, C2);
-        T = __fmul_rn(T, __fsub_rn(1.0f, alpha));
-        ++cnt;
-        lst = base + k + 1;
-        if (T < kTMin) done = true;
+        T = __fmul_rn(T, __fsub_rn(1.0f, ab));
+        cnt += blend ? 1 : 0;
+        lst = blend ? base + k + 1 : lst;
+        done = done || T < kTMin;
       }
     }
   }
@@ -222,12 +261,13 @@ __device__ __forceinline__ float warp_reduce9(const float v[9], int lane) {
 }
 
 __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
-  __shared__ float4 s_geo[kBlock];  // px, py, a2, b2
-  __shared__ float4 s_co[kBlock];   // c2, opacity, A, B
-  __shared__ float4 s_rgb[kBlock];  // r, g, b, C
-  __shared__ float4 s_box[kBlock];
-  __shared__ float s_acc[kBlock][9];  // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
-  __shared__ uint32_t s_idx[kBlock];
+  __shared__ float4 s_geo[kBatchB];  // px, py, a2, b2
+  __shared__ float4 s_co[kBatchB];   // c2, opacity, A, B
+  __shared__ float4 s_rgb[kBatchB];  // r, g, b, C
+  __shared__ float4 s_box[kBatchB];  // px, py, hx, hy of the blend region
+  __shared__ float s_rc2[kBatchB];
+  __shared__ float s_acc[kBatchB][9];  // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
+  __shared__ uint32_t s_idx[kBatchB];
   __shared__ int s_maxlast;
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -237,8 +277,8 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
   const int u = tx0 + du, v = ty0 + dv;
   const bool inside = u < a.W && v < a.H;
   const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
-  const float wx0 = (float)(tx0 + (warp & 1) * 8) + 0.5f, wx1 = wx0 + 7.0f;
-  const float wy0 = (float)(ty0 + (warp >> 1) * 4) + 0.5f, wy1 = wy0 + 3.0f;
+  const float wcx = (float)(tx0 + (warp & 1) * 8) + 4.0f;
+  const float wcy = (float)(ty0 + (warp >> 1) * 4) + 2.0f;
   const uint2 range = a.ranges[tile];
   const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
   float T = 1.0f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
@@ -258,74 +298,77 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
   if (lane == 0 && warp_last > 0) atomicMax(&s_maxlast, warp_last);
   __syncthreads();
   const int n = s_maxlast;  // list offsets [0, n) can hold a blend
-  for (int done = 0; done < n; done += kBlock) {
+  for (int done = 0; done < n; done += kBatchB) {
     // slot k of this batch holds list offset n - 1 - done - k (back to front)
     __syncthreads();
-    const int off = n - 1 - done - tid;
-    if (off >= 0) {
-      const uint32_t i = a.vals[range.x + off];
-      const float4 g = a.xyzo[i];
-      const float4 q = a.conic[i];
-      const float4 c = a.rgb[i];
-      const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
-                  c2 = __fmul_rn(q.z, kHalfNegLog2e);
-      s_geo[tid] = make_float4(g.x, g.y, a2, b2);
-      s_co[tid] = make_float4(c2, g.w, q.x, q.y);
-      s_rgb[tid] = make_float4(c.x, c.y, c.z, q.z);
-      s_box[tid] = blend_box(g.x, g.y, a2, b2, c2, g.w);
-      s_idx[tid] = i;
-    }
+    for (int e = tid; e < kBatchB; e += kBlock) {
+      const int off = n - 1 - done - e;
+      if (off >= 0) {
+        const uint32_t i = a.vals[range.x + off];
+        const float4 g = a.xyzo[i];
+        const float4 q = a.conic[i];
+        const float4 c = a.rgb[i];
+        const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
+                    c2 = __fmul_rn(q.z, kHalfNegLog2e);
+        s_geo[e] = make_float4(g.x, g.y, a2, b2);
+        s_co[e] = make_float4(c2, g.w, q.x, q.y);
+        s_rgb[e] = make_float4(c.x, c.y, c.z, q.z);
+        const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
+        s_box[e] = r.box;
+        s_rc2[e] = r.rc2;
+        s_idx[e] = i;
+      }
 #pragma unroll
-    for (int j = 0; j < 9; ++j) s_acc[tid][j] = 0.0f;
+      for (int j = 0; j < 9; ++j) s_acc[e][j] = 0.0f;
+    }
     __syncthreads();
-    const int m = min(kBlock, n - done);
+    const int m = min(kBatchB, n - done);
     for (int c0 = 0; c0 < m; c0 += 32) {
       const int j = c0 + lane;
-      const bool rel = j < m && (n - 1 - done - j) < warp_last && box_hits(s_box[j], wx0, wx1, wy0, wy1);
+      const bool rel = j < m && (n - 1 - done - j) < warp_last && region_hits(s_box[j], s_rc2[j], wcx, wcy);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
       while (msk) {
         const int k = c0 + __ffs(msk) - 1;
         msk &= msk - 1;
         const int offk = n - 1 - done - k;
-        float gv[9] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        bool contrib = false;
-        if (offk < my_last) {
-          const float4 g = s_geo[k];
-          const float4 co = s_co[k];
-          const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
-          float qv = __fmul_rn(g.z, dx);
-          qv = __fmaf_rn(g.w, dy, qv);
-          float p2 = __fmul_rn(dx, qv);
-          const float wv = __fmul_rn(co.x, dy);
-          p2 = __fmaf_rn(wv, dy, p2);
-          const float e = exp2_raster(p2);
-          const float vv = __fmul_rn(co.y, e);
-          const float alpha = fminf(vv, kAlphaMax);
-          contrib = alpha >= kAlphaMin;
-          if (contrib) {
-            const float4 c = s_rgb[k];
-            const float oma = 1.0f - alpha;
-            T = T / oma;  // transmittance in front of this Gaussian
-            const float wgt = alpha * T;
-            gv[6] = g0 * wgt;
-            gv[7] = g1 * wgt;
-            gv[8] = g2 * wgt;
-            const float Gk = T * (g0 * (c.x - R0) + g1 * (c.y - R1) + g2 * (c.z - R2));
-            if (vv < kAlphaMax) {
-              gv[2] = Gk * e;
-              const float dp = Gk * alpha;
-              const float A = co.z, B = co.w, Cc = c.w;
-              gv[0] = -dp * fmaf(A, dx, B * dy);
-              gv[1] = -dp * fmaf(B, dx, Cc * dy);
-              gv[3] = -0.5f * dp * dx * dx;
-              gv[4] = -dp * dx * dy;
-              gv[5] = -0.5f * dp * dy * dy;
-            }
-            R0 = fmaf(c.x, alpha, oma * R0);
-            R1 = fmaf(c.y, alpha, oma * R1);
-            R2 = fmaf(c.z, alpha, oma * R2);
-          }
-        }
+        // Branch-free body: a lane whose pair is not a blend of the forward
+        // (past its last blend, or alpha < 1/255) runs with alpha 0, which
+        // leaves T and R unchanged, and its terms are masked to zero.
+        const float4 g = s_geo[k];
+        const float4 co = s_co[k];
+        const float4 c = s_rgb[k];
+        const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
+        float qv = __fmul_rn(g.z, dx);
+        qv = __fmaf_rn(g.w, dy, qv);
+        float p2 = __fmul_rn(dx, qv);
+        const float wv = __fmul_rn(co.x, dy);
+        p2 = __fmaf_rn(wv, dy, p2);
+        const float e = exp2_raster(p2);
+        const float vv = __fmul_rn(co.y, e);
+        const float alpha = fminf(vv, kAlphaMax);
+        const bool contrib = offk < my_last && alpha >= kAlphaMin;
+        const float ab = contrib ? alpha : 0.0f;
+        const float oma = 1.0f - ab;
+        // transmittance in front of this Gaussian (gradient values only)
+        T = contrib ? __fdividef(T, oma) : T;
+        const float wgt = ab * T;
+        float gv[9];
+        gv[6] = g0 * wgt;
+        gv[7] = g1 * wgt;
+        gv[8] = g2 * wgt;
+        const float Gk = T * (g0 * (c.x - R0) + g1 * (c.y - R1) + g2 * (c.z - R2));
+        const float Gm = (contrib && vv < kAlphaMax) ? Gk : 0.0f;  // no gradient through a clamped alpha
+        gv[2] = Gm * e;
+        const float dp = Gm * ab;
+        const float A = co.z, B = co.w, Cc = c.w;
+        gv[0] = -dp * fmaf(A, dx, B * dy);
+        gv[1] = -dp * fmaf(B, dx, Cc * dy);
+        gv[3] = -0.5f * dp * dx * dx;
+        gv[4] = -dp * dx * dy;
+        gv[5] = -0.5f * dp * dy * dy;
+        R0 = fmaf(c.x, ab, oma * R0);
+        R1 = fmaf(c.y, ab, oma * R1);
+        R2 = fmaf(c.z, ab, oma * R2);
         if (__any_sync(0xffffffffu, contrib)) {
           const float tot = warp_reduce9(gv, lane);
           if (slot.owner) atomicAdd(&s_acc[k][slot.idx], tot);
@@ -333,16 +376,16 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
       }
     }
     __syncthreads();
-    if (tid < m) {
+    for (int e = tid; e < m; e += kBlock) {
       float r[9];
       bool any = false;
 #pragma unroll
       for (int j = 0; j < 9; ++j) {
-        r[j] = s_acc[tid][j];
+        r[j] = s_acc[e][j];
         any |= r[j] != 0.0f;
       }
       if (any) {
-        float4* dst = a.grad2d + 3 * (size_t)s_idx[tid];
+        float4* dst = a.grad2d + 3 * (size_t)s_idx[e];
         atomicAdd(dst, make_float4(r[0], r[1], r[2], 0.f));
         atomicAdd(dst + 1, make_float4(r[3], r[4], r[5], 0.f));
         atomicAdd(dst + 2, make_float4(r[6], r[7], r[8], 0.f));

@@ -411,6 +411,8 @@ void project_one(const Cam& cam, const R mu[3], const R ls[3], const R q[4], R l
     if (clamp_fixed) pass = !clamp_fixed[ch];
     o.rgb[ch] = pass ? v : R(0);
   }
+  // an infinite colour (from infinite SH coefficients) culls, like a non-finite parameter
+  if (!finite3(o.rgb[0], o.rgb[1], o.rgb[2])) return;
   o.visible = true;
   o.px = px; o.py = py; o.depth = t[2]; o.opacity = op;
   o.A = cA; o.B = cB; o.C = cC;

@@ -106,9 +106,12 @@ def test_preprocess_edge_cases():
     q[:, 3] = 0.0
     lg = np.zeros(N, np.float32)
     lg[6] = np.inf
-    sc = make_scene(means, ls, q, lg, np.ones((3, N)), 0, [cam])
+    sh = np.ones((3, N))
+    sh[1, 1] = np.inf  # infinite colour culls
+    sh[0, 2] = np.nan  # NaN colour clamps to 0
+    sc = make_scene(means, ls, q, lg, sh, 0, [cam])
     R, ref = _full_compare(sc)
-    assert list(ref["rec"]["tiles"] > 0) == [False, True, True, False, False, False, False, False, True]
+    assert list(ref["rec"]["tiles"] > 0) == [False, False, True, False, False, False, False, False, True]
     assert ref["rec"]["tiles"][8] == 16
 
 

@@ -162,12 +162,16 @@ def test_culling_cases(orc):
     q[:, 3] = 0.0  # degenerate quaternion
     lg = np.zeros(N, np.float32)
     lg[6] = np.inf  # non-finite logit
-    sc = make_scene(means, ls, q, lg, np.ones((3, N)), 0, [cam])
+    sh = np.ones((3, N))
+    sh[1, 1] = np.inf  # infinite colour
+    sh[0, 2] = np.nan  # NaN colour clamps to 0 and stays visible
+    sc = make_scene(means, ls, q, lg, sh, 0, [cam])
     rec = orc.preprocess(sc, cam)
     vis = rec["tiles"] > 0
-    # 0: on the near plane; 1: just beyond; 2: fine; 3: zero quaternion;
-    # 4: behind; 5: far off-screen; 6: infinite logit; 7: NaN mean
-    assert list(vis) == [False, True, True, False, False, False, False, False]
+    # 0: on the near plane; 1: just beyond but infinite colour; 2: fine (NaN colour -> 0);
+    # 3: zero quaternion; 4: behind; 5: far off-screen; 6: infinite logit; 7: NaN mean
+    assert list(vis) == [False, False, True, False, False, False, False, False]
+    assert rec["rgb"][2, 0] == 0.0
     for g in np.nonzero(~vis)[0]:
         assert not rec["xyzo"][g].any() and not rec["conic"][g].any() and rec["radius"][g] == 0
 

@@ -51,48 +51,62 @@ __device__ __forceinline__ void tile_pixel(int tid, int& du, int& dv) {
 // up to ~2 ulp, i.e. p2 >= -log2(255 o) - 1e-3. Hence every blending pixel
 // lies in the ellipse d^T (M - sl I) d <= log2(255 o) + 1e-3, whose bounding
 // box is returned, widened by 2% plus 0.05 px to cover the rounding of this
-// computation. The same ellipse also lies in the disk of radius
-// sqrt(rho2 / lambda_min) around the centre; that disk is used too when the
-// ellipse is not elongated (lambda_min > lambda_max / 100, so lambda_min is
-// accurate in fp32), widened the same way. The region is returned as
-// (px, py, half-width, half-height) and the squared disk radius; an empty
-// region (negative half-widths) if the Gaussian can never blend, an unbounded
-// one if (M - sl I) is not safely positive definite.
+// computation. For an ellipse that is not elongated (lambda_min >
+// lambda_max / 100, where the quadratic form is accurate in fp32 to ~1e-4
+// relative) the test is exact instead: the minimum of d^T (M - sl I) d over
+// the warp's rectangle of pixel centres (widened by the same pad) against
+// rho2 * 1.01. Returned: box = (px, py, hx, hy); q1 = (m00, m01, m11,
+// threshold), threshold +inf when only the box applies; q2 = (m01 / m00,
+// m01 / m11, pad, 0). An empty box (negative half-widths) if the Gaussian
+// can never blend, an unbounded one if (M - sl I) is not safely positive
+// definite.
 struct BlendRegion {
-  float4 box;  // px, py, hx, hy
-  float rc2;   // squared disk radius
+  float4 box;
+  float4 q1;
+  float4 q2;
 };
 
 __device__ __forceinline__ BlendRegion blend_region(float px, float py, float a2, float b2, float c2, float o) {
   const float kInf = __int_as_float(0x7f800000);
   const float rho2 = __log2f(255.0f * o) + 1e-3f;
-  if (!(rho2 > 0.0f)) return BlendRegion{make_float4(px, py, -kInf, -kInf), -kInf};
+  const float4 none = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!(rho2 > 0.0f)) return BlendRegion{make_float4(px, py, -kInf, -kInf), make_float4(1.f, 0.f, 1.f, kInf), none};
   const float K = fmaxf(fabsf(a2), fabsf(c2)) + 0.5f * fabsf(b2);
   const float sl = 1e-6f * K;
   const float m00 = -a2 - sl, m11 = -c2 - sl, m01 = -0.5f * b2;
   const float det = m00 * m11 - m01 * m01;
   if (!(m00 > 0.0f) || !(m11 > 0.0f) || !(det > 1e-3f * (m00 * m11)))
-    return BlendRegion{make_float4(px, py, kInf, kInf), kInf};
+    return BlendRegion{make_float4(px, py, kInf, kInf), make_float4(1.f, 0.f, 1.f, kInf), none};
   const float pad = 0.05f + 1e-6f * (fabsf(px) + fabsf(py));
   const float hx = sqrtf(rho2 * m11 / det) * 1.02f + pad;
   const float hy = sqrtf(rho2 * m00 / det) * 1.02f + pad;
   const float half_tr = 0.5f * (m00 + m11);
   const float disc = sqrtf(0.25f * (m00 - m11) * (m00 - m11) + m01 * m01);
   const float lmin = half_tr - disc;
-  float rc2 = kInf;
-  if (lmin > 0.01f * (half_tr + disc)) {
-    const float rc = sqrtf(rho2 / lmin) * 1.02f + pad;
-    rc2 = rc * rc;
-  }
-  return BlendRegion{make_float4(px, py, hx, hy), rc2};
+  const float thr = lmin > 0.01f * (half_tr + disc) ? rho2 * 1.01f : kInf;
+  return BlendRegion{make_float4(px, py, hx, hy), make_float4(m00, m01, m11, thr),
+                     make_float4(m01 / m00, m01 / m11, pad, 0.f)};
 }
 
-// Can the Gaussian of region (b, rc2) blend at a pixel centre of the warp
-// block with centre (wcx, wcy) and half extents (3.5, 1.5)?
-__device__ __forceinline__ bool region_hits(const float4 b, float rc2, float wcx, float wcy) {
-  const float ex = fabsf(b.x - wcx) - 3.5f, ey = fabsf(b.y - wcy) - 1.5f;
-  const float qx = fmaxf(ex, 0.0f), qy = fmaxf(ey, 0.0f);
-  return ex <= b.z && ey <= b.w && qx * qx + qy * qy <= rc2;
+// Can the Gaussian blend at a pixel centre of the warp block with centre
+// (wcx, wcy) and half extents (3.5, 1.5)? Box test, then (when enabled) the
+// minimum of the quadratic form over the rectangle of offsets d = (px, py) -
+// pixel centre: 0 if the rectangle holds the centre, else the least of the
+// four edges' one-dimensional minima.
+__device__ __forceinline__ bool region_hits(const float4 b, const float4 q1, const float4 q2, float wcx,
+                                            float wcy) {
+  const float ux = b.x - wcx, uy = b.y - wcy;
+  if (!(fabsf(ux) - 3.5f <= b.z && fabsf(uy) - 1.5f <= b.w)) return false;
+  if (!(q1.w < __int_as_float(0x7f800000))) return true;
+  const float dx0 = ux - 3.5f - q2.z, dx1 = ux + 3.5f + q2.z;
+  const float dy0 = uy - 1.5f - q2.z, dy1 = uy + 1.5f + q2.z;
+  if (dx0 <= 0.0f && dx1 >= 0.0f && dy0 <= 0.0f && dy1 >= 0.0f) return true;
+  const float m00 = q1.x, m01 = q1.y, m11 = q1.z;
+  auto qf = [&](float dx, float dy) { return fmaf(m00 * dx, dx, fmaf(2.0f * m01 * dx, dy, m11 * dy * dy)); };
+  const float xa = fminf(fmaxf(-q2.x * dy0, dx0), dx1), xb = fminf(fmaxf(-q2.x * dy1, dx0), dx1);
+  const float ya = fminf(fmaxf(-q2.y * dx0, dy0), dy1), yb = fminf(fmaxf(-q2.y * dx1, dy0), dy1);
+  const float best = fminf(fminf(qf(xa, dy0), qf(xb, dy1)), fminf(qf(dx0, ya), qf(dx1, yb)));
+  return best <= q1.w;
 }
 
 struct FwdArgs {
@@ -113,8 +127,9 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
   __shared__ float4 s_geo[kBatchF];  // px, py, a2, b2
   __shared__ float2 s_co[kBatchF];   // c2, opacity
   __shared__ float4 s_rgb[kBatchF];
-  __shared__ float4 s_box[kBatchF];  // px, py, hx, hy of the blend region
-  __shared__ float s_rc2[kBatchF];
+  __shared__ float4 s_box[kBatchF];  // blend region of each staged entry
+  __shared__ float4 s_q1[kBatchF];
+  __shared__ float4 s_q2[kBatchF];
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int du, dv;
@@ -144,14 +159,15 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
       s_rgb[e] = a.rgb[i];
       const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
       s_box[e] = r.box;
-      s_rc2[e] = r.rc2;
+      s_q1[e] = r.q1;
+      s_q2[e] = r.q2;
     }
     __syncthreads();
     const int m = min(kBatchF, n - base);
     for (int c0 = 0; c0 < m; c0 += 32) {
       if (__all_sync(0xffffffffu, done)) break;
       const int j = c0 + lane;
-      const bool rel = j < m && region_hits(s_box[j], s_rc2[j], wcx, wcy);
+      const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
       // Branch-free body: a lane that skips the pair (alpha < 1/255) or has
       // already stopped blends with alpha 0, which leaves C, T and the counts
@@ -264,8 +280,9 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
   __shared__ float4 s_geo[kBatchB];  // px, py, a2, b2
   __shared__ float4 s_co[kBatchB];   // c2, opacity, A, B
   __shared__ float4 s_rgb[kBatchB];  // r, g, b, C
-  __shared__ float4 s_box[kBatchB];  // px, py, hx, hy of the blend region
-  __shared__ float s_rc2[kBatchB];
+  __shared__ float4 s_box[kBatchB];  // blend region of each staged entry
+  __shared__ float4 s_q1[kBatchB];
+  __shared__ float4 s_q2[kBatchB];
   __shared__ float s_acc[kBatchB][9];  // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
   __shared__ uint32_t s_idx[kBatchB];
   __shared__ int s_maxlast;
@@ -315,7 +332,8 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
         s_rgb[e] = make_float4(c.x, c.y, c.z, q.z);
         const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
         s_box[e] = r.box;
-        s_rc2[e] = r.rc2;
+        s_q1[e] = r.q1;
+        s_q2[e] = r.q2;
         s_idx[e] = i;
       }
 #pragma unroll
@@ -325,7 +343,7 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
     const int m = min(kBatchB, n - done);
     for (int c0 = 0; c0 < m; c0 += 32) {
       const int j = c0 + lane;
-      const bool rel = j < m && (n - 1 - done - j) < warp_last && region_hits(s_box[j], s_rc2[j], wcx, wcy);
+      const bool rel = j < m && (n - 1 - done - j) < warp_last && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
       while (msk) {
         const int k = c0 + __ffs(msk) - 1;

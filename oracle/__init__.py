@@ -75,7 +75,7 @@ def _declare(L):
                                      P, P, P, P, P, P, P, P, P]
     L.or_loss_frozen_f64.restype = ctypes.c_double
     L.or_backward_f64.argtypes = [P, P, P, P, P, I32, I64, P, I64, P, I32, I32,
-                                  P, P, P, P, P, P, P, P, P, P] + [P] * 10 + [P, I64]
+                                  P, P, P, P, P, P, P, P, P, P] + [P] * 10 + [P, I64, I32]
     L.or_num_threads.restype = ctypes.c_int
     L.or_preprocess_bwd_f64.argtypes = [P, P, P, P, P, I32, I64, P, I64, P, I32, I32,
                                         P, P, P] + [P] * 10
@@ -243,8 +243,12 @@ def num_threads() -> int:
     return int(lib().or_num_threads())
 
 
-def backward(scene, cam, rec, bins, dL_dimage, params3d=True, tile_subset=None):
-    """Reference gradients (fp64, fp32 decisions) with magnitude bounds."""
+def backward(scene, cam, rec, bins, dL_dimage, params3d=True, tile_subset=None, records2d="fp32"):
+    """Reference gradients (fp64, fp32 decisions) with magnitude bounds.
+
+    records2d: "fp32" differentiates the compositing at the fp32 records (the
+    raster stage's inputs); "fp64" at an fp64 re-projection of the parameters,
+    the point the frozen-decision loss (finite differences) evaluates."""
     N, K = scene.N, scene.K
     na = rec["n_active"]
     act = rec.get("active_idx")
@@ -264,7 +268,7 @@ def backward(scene, cam, rec, bins, dL_dimage, params3d=True, tile_subset=None):
         _p(_c(scene.bg, np.float32)), _p(_c(dL_dimage, np.float32)), _p(g2), _p(s2),
         *[_p(a) for a in d], *[_p(a) for a in m],
         _p(None if tile_subset is None else _c(tile_subset, np.int32)),
-        0 if tile_subset is None else len(tile_subset))
+        0 if tile_subset is None else len(tile_subset), 1 if records2d == "fp32" else 0)
     if params3d:
         names = ["means", "log_scales", "quats", "opacity_logits", "sh"]
         out.update({"d_" + k: v for k, v in zip(names, d)})

@@ -435,7 +435,8 @@ void gather(const Src* means, const Src* ls, const Src* quats, const Src* logits
 
 // ------------------------------------------------------------- pixel walk
 // Front-to-back walk of one pixel over its tile's list in fp32 spec mode.
-// Calls blend(j, i, alpha, clamped) for every blended entry, in order.
+// Calls blend(j, i, alpha, clamped, e) for every blended entry, in order
+// (e = exp2 of the pair's exponent, alpha = min(0.99, o e), both fp32).
 struct Rec32 {
   const float* xyzo;
   const float* conic;
@@ -465,7 +466,7 @@ void walk_pixel(const Rec32& r, const uint32_t* vals, uint32_t start, uint32_t e
     const bool clamped = !(v < KC.alpha_max);
     const float alpha = clamped ? KC.alpha_max : v;
     if (alpha < KC.alpha_min) continue;
-    blend(j, i, alpha, clamped);
+    blend(j, i, alpha, clamped, e);
     T = T * (1.0f - alpha);
     n += 1;
     last = (int)(j - start + 1);
@@ -663,7 +664,7 @@ OR_API int or_raster_fwd(const float* xyzo, const float* conic, const float* rgb
         int n, lst;
         const float xc = (float)u + 0.5f, yc = (float)v + 0.5f;
         walk_pixel(r, vals, start, end, xc, yc, T, n, lst,
-                   [&](uint32_t, uint32_t i, float alpha, bool) {
+                   [&](uint32_t, uint32_t i, float alpha, bool, float) {
                      // T here is the transmittance before this blend.
                      const float wgt = alpha * T;
                      for (int ch = 0; ch < 3; ++ch) C[ch] = std::fmaf(wgt, rgb[4 * (size_t)i + ch], C[ch]);
@@ -706,7 +707,7 @@ OR_API int or_raster_fwd_bruteforce(const float* xyzo, const float* conic, const
       float C[3] = {0.0f, 0.0f, 0.0f}, T;
       int nc, lst;
       walk_pixel(r, idx.data(), 0, (uint32_t)idx.size(), (float)u + 0.5f, (float)v + 0.5f, T, nc, lst,
-                 [&](uint32_t, uint32_t i, float alpha, bool) {
+                 [&](uint32_t, uint32_t i, float alpha, bool, float) {
                    const float wgt = alpha * T;
                    for (int ch = 0; ch < 3; ++ch) C[ch] = std::fmaf(wgt, rgb[4 * (size_t)i + ch], C[ch]);
                  });
@@ -755,6 +756,7 @@ void project_all_f64(const double* means, const double* ls, const double* quats,
 struct Blend {
   uint32_t i;
   bool clamped;
+  float alpha, e;  // fp32 values of the forward
 };
 
 // Gradient-flow number types for the preprocess backward: plain values, or
@@ -947,7 +949,7 @@ OR_API double or_loss_frozen_f64(const double* means, const double* log_scales, 
         float T32;
         int n, lst;
         walk_pixel(r, vals, start, end, (float)xc, (float)yc, T32, n, lst,
-                   [&](uint32_t, uint32_t i, float, bool clamped) {
+                   [&](uint32_t, uint32_t i, float, bool clamped, float) {
                      const P64& g = P[i];
                      const double dx = g.px - xc, dy = g.py - yc;
                      const double p = -0.5 * (g.A * dx * dx + g.C * dy * dy) - g.B * dx * dy;
@@ -980,7 +982,7 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
                            double* d_means, double* d_log_scales, double* d_quats, double* d_logits,
                            double* d_sh, double* m_means, double* m_log_scales, double* m_quats,
                            double* m_logits, double* m_sh, const int32_t* tile_subset,
-                           int64_t n_subset) {
+                           int64_t n_subset, int records2d) {
   const int K = (sh_degree + 1) * (sh_degree + 1);
   const Cam cam = make_cam(camv, width, height);
   // fp64 copies of the parameters
@@ -994,6 +996,17 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
   std::vector<P64> P;
   project_all_f64(mu64.data(), ls64.data(), q64.data(), lg64.data(), sh64.data(), K, N, active_idx,
                   n_active, cam, rgb32, tiles32, P);
+  if (records2d) {
+    // The raster stage's backward takes the records as its inputs: differentiate
+    // the compositing at the fp32 record values the forward used.
+    for (int64_t i = 0; i < n_active; ++i) {
+      P64& o = P[(size_t)i];
+      if (!o.visible) continue;
+      o.px = xyzo32[4 * i]; o.py = xyzo32[4 * i + 1]; o.o = xyzo32[4 * i + 3];
+      o.A = conic32[4 * i]; o.B = conic32[4 * i + 1]; o.C = conic32[4 * i + 2];
+      for (int ch = 0; ch < 3; ++ch) o.rgb[ch] = rgb32[4 * i + ch];
+    }
+  }
   std::vector<double> G2((size_t)n_active * 9, 0.0), S2((size_t)n_active * 9, 0.0);
   const Rec32 r{xyzo32, conic32, rgb32};
   const int TW = cam.TW;
@@ -1013,7 +1026,9 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
         float T32;
         int n, lst;
         walk_pixel(r, vals, start, end, (float)xc, (float)yc, T32, n, lst,
-                   [&](uint32_t, uint32_t i, float, bool clamped) { bl.push_back(Blend{i, clamped}); });
+                   [&](uint32_t, uint32_t i, float alpha, bool clamped, float e) {
+                     bl.push_back(Blend{i, clamped, alpha, e});
+                   });
         const size_t pix = (size_t)v * width + u;
         const double gp[3] = {dL_dimage[pix], dL_dimage[NP + pix], dL_dimage[2 * NP + pix]};
         const size_t nb = bl.size();
@@ -1022,9 +1037,16 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
         for (size_t k = 0; k < nb; ++k) {
           const P64& g = P[bl[k].i];
           const double dx = g.px - xc, dy = g.py - yc;
-          const double p = -0.5 * (g.A * dx * dx + g.C * dy * dy) - g.B * dx * dy;
-          ex[k] = std::exp(p);
-          al[k] = bl[k].clamped ? 0.99 : g.o * ex[k];
+          if (records2d) {
+            // the forward's own alpha and exp values: the derivative of the
+            // computation that produced the image
+            ex[k] = bl[k].e;
+            al[k] = bl[k].alpha;
+          } else {
+            const double p = -0.5 * (g.A * dx * dx + g.C * dy * dy) - g.B * dx * dy;
+            ex[k] = std::exp(p);
+            al[k] = bl[k].clamped ? 0.99 : g.o * ex[k];
+          }
           Tk[k] = T;
           T *= (1.0 - al[k]);
         }
@@ -1032,28 +1054,40 @@ OR_API int or_backward_f64(const float* means, const float* log_scales, const fl
         for (size_t kk = nb; kk-- > 0;) {
           const uint32_t i = bl[kk].i;
           const P64& g = P[i];
-          double t9[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
-          double Gk = 0.0;
+          // t9: the pair's terms; a9: the same terms with every operand replaced
+          // by its magnitude (c - R becomes |c| + |R|), the scale of their
+          // rounding error in a single-precision evaluation.
+          double t9[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0}, a9[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+          double Gk = 0.0, Ga = 0.0;
           for (int ch = 0; ch < 3; ++ch) {
             t9[6 + ch] = gp[ch] * al[kk] * Tk[kk];
+            a9[6 + ch] = std::fabs(t9[6 + ch]);
             Gk += gp[ch] * (g.rgb[ch] - Rb[ch]);
+            Ga += std::fabs(gp[ch]) * (std::fabs(g.rgb[ch]) + std::fabs(Rb[ch]));
           }
           Gk *= Tk[kk];
+          Ga *= Tk[kk];
           if (!bl[kk].clamped) {
             const double dx = g.px - xc, dy = g.py - yc;
-            const double dp = Gk * al[kk];
+            const double dp = Gk * al[kk], dpa = Ga * al[kk];
             t9[5] = Gk * ex[kk];
             t9[0] = dp * (-(g.A * dx + g.B * dy));
             t9[1] = dp * (-(g.B * dx + g.C * dy));
             t9[2] = dp * (-0.5 * dx * dx);
             t9[3] = dp * (-dx * dy);
             t9[4] = dp * (-0.5 * dy * dy);
+            a9[5] = Ga * ex[kk];
+            a9[0] = dpa * (std::fabs(g.A * dx) + std::fabs(g.B * dy));
+            a9[1] = dpa * (std::fabs(g.B * dx) + std::fabs(g.C * dy));
+            a9[2] = dpa * 0.5 * dx * dx;
+            a9[3] = dpa * std::fabs(dx * dy);
+            a9[4] = dpa * 0.5 * dy * dy;
           }
           for (int m = 0; m < 9; ++m) {
 #pragma omp atomic
             G2[9 * (size_t)i + m] += t9[m];
 #pragma omp atomic
-            S2[9 * (size_t)i + m] += std::fabs(t9[m]);
+            S2[9 * (size_t)i + m] += a9[m];
           }
           for (int ch = 0; ch < 3; ++ch) Rb[ch] = g.rgb[ch] * al[kk] + (1.0 - al[kk]) * Rb[ch];
         }

@@ -22,7 +22,7 @@ def _fd_check(orc, sc, n_params=None, seed=0):
     r = orc.render(sc)
     rec, bins = r["rec"], r["bins"]
     g = sc.grad_image(0)
-    an = orc.backward(sc, cam, rec, bins, g)
+    an = orc.backward(sc, cam, rec, bins, g, records2d="fp64")
     base = params64(sc)
     idx = [(a, k) for a in range(5) for k in range(base[a].size)]
     if n_params is not None:
@@ -78,7 +78,7 @@ def test_single_gaussian_single_pixel_by_hand(orc):
     r = orc.render(sc)
     assert r["fwd"]["n_contrib"][0, 0] == 1
     g = np.array([0.3, -1.1, 0.6], np.float32)
-    an = orc.backward(sc, cam, r["rec"], r["bins"], g.reshape(3, 1, 1))
+    an = orc.backward(sc, cam, r["rec"], r["bins"], g.reshape(3, 1, 1), records2d="fp64")
     out, vis, _ = orc.project_f64(params64(sc), 0, 1, cam)
     px, py, _, o, A, B, C, cr, cg, cb = out[0]
     dx, dy = px - 0.5, py - 0.5
@@ -111,3 +111,15 @@ def test_magnitudes_bound_gradients_and_inactive_are_zero(orc):
     assert invisible[:20].all()
     for n in NAMES:
         assert not an["d_" + n][..., invisible].any()
+
+
+def test_record_point_and_fp64_point_agree_when_well_conditioned(orc):
+    # the two evaluation points differ only by fp32 rounding of the records
+    sc = S.random_scene(200, 64, 48, sh_degree=2, seed=25)
+    cam = sc.cameras[0]
+    r = orc.render(sc)
+    g = sc.grad_image(0)
+    a = orc.backward(sc, cam, r["rec"], r["bins"], g, records2d="fp32")
+    b = orc.backward(sc, cam, r["rec"], r["bins"], g, records2d="fp64")
+    assert np.all(np.abs(a["g2d"] - b["g2d"]) <= 1e-3 * np.abs(b["g2d"]) + 1e-4 * b["s2d"])
+    assert np.all(a["s2d"] >= np.abs(a["g2d"]) * (1 - 1e-12))

@@ -2,10 +2,12 @@
 //
 // One CTA per 16x16 tile, one thread per pixel; each warp owns an 8x4 pixel
 // block so that its lanes sit close together in the image. The tile's sorted
-// list is walked in batches of 256 records that the CTA stages cooperatively
-// in shared memory (one gathered 16-byte load per record field per batch),
-// after which every thread reads them as shared-memory broadcasts. The CTA
-// leaves the walk as soon as all its pixels have stopped.
+// list is walked in batches of 256 records, one per thread, that the CTA
+// stages in shared memory, after which every thread reads them as
+// shared-memory broadcasts. In the backward the gathers are
+// software-pipelined: a batch's records arrive by cp.async while the
+// previous batch is processed. The forward CTA leaves the walk as soon as
+// all its pixels have stopped.
 //
 // The per-pair arithmetic is the fixed fp32 specification: the conic is
 // scaled by -log2(e)/2 (and -log2(e) for the cross term) when it is staged,
@@ -21,16 +23,18 @@ namespace {
 
 constexpr int kTile = 16;
 constexpr int kBlock = kTile * kTile;
-#ifndef GS_RASTER_BATCH_FWD
-#define GS_RASTER_BATCH_FWD 256
-#endif
-#ifndef GS_RASTER_BATCH_BWD
-#define GS_RASTER_BATCH_BWD 256
-#endif
-// List entries staged in shared memory per CTA-wide step.
-constexpr int kBatchF = GS_RASTER_BATCH_FWD;
-constexpr int kBatchB = GS_RASTER_BATCH_BWD;
-static_assert(kBatchF % 32 == 0 && kBatchB % 32 == 0 && kBatchF >= kBlock && kBatchB >= kBlock, "batch: warp multiple, at least one block");
+// List entries staged in shared memory per CTA-wide step: one per thread.
+constexpr int kBatchF = kBlock;
+constexpr int kBatchB = kBlock;
+
+// 16-byte asynchronous global -> shared copy (L2 only), its commit and the
+// wait for all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 // Pixel of thread `tid` in the tile: warp w covers the 8x4 block at
 // ((w & 1) * 8, (w >> 1) * 4).
@@ -109,6 +113,21 @@ __device__ __forceinline__ bool region_hits(const float4 b, const float4 q1, con
   return best <= q1.w;
 }
 
+// Centre of the 8x4 block of pixel centres of warp w in the tile at (tx0, ty0).
+__device__ __forceinline__ float block_cx(int tx0, int w) { return (float)(tx0 + (w & 1) * 8) + 4.0f; }
+__device__ __forceinline__ float block_cy(int ty0, int w) { return (float)(ty0 + (w >> 1) * 4) + 2.0f; }
+
+// Bit w set: the region can reach a pixel centre of warp w's block (the
+// test each warp would make, made once by the thread that stages the entry,
+// so the CTA keeps one byte per entry instead of the region itself).
+__device__ __forceinline__ uint32_t region_mask(const BlendRegion& r, int tx0, int ty0) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int w = 0; w < kBlock / 32; ++w)
+    if (region_hits(r.box, r.q1, r.q2, block_cx(tx0, w), block_cy(ty0, w))) m |= 1u << w;
+  return m;
+}
+
 struct FwdArgs {
   const float4* xyzo;
   const float4* conic;
@@ -123,7 +142,7 @@ struct FwdArgs {
   int32_t* last;
 };
 
-__global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
+__global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   __shared__ float4 s_geo[kBatchF];  // px, py, a2, b2
   __shared__ float2 s_co[kBatchF];   // c2, opacity
   __shared__ float4 s_rgb[kBatchF];
@@ -139,16 +158,18 @@ __global__ void __launch_bounds__(kBlock) raster_fwd_kernel(FwdArgs a) {
   const bool inside = u < a.W && v < a.H;
   const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
   // centre of this warp's 8x4 block of pixel centres
-  const float wcx = (float)(tx0 + (warp & 1) * 8) + 4.0f;
-  const float wcy = (float)(ty0 + (warp >> 1) * 4) + 2.0f;
+  const float wcx = block_cx(tx0, warp), wcy = block_cy(ty0, warp);
   const uint2 range = a.ranges[tile];
   const int n = (int)(range.y - range.x);
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int cnt = 0, lst = 0;
   bool done = !inside;
+  // (The forward stages with plain gathers: with five CTAs per SM the
+  // others cover a staging CTA's latency.)
   for (int base = 0; base < n; base += kBatchF) {
     if (__syncthreads_count(done) == kBlock) break;
-    for (int e = tid; e < kBatchF && base + e < n; e += kBlock) {
+    if (base + tid < n) {
+      const int e = tid;
       const uint32_t i = a.vals[range.x + base + e];
       const float4 g = a.xyzo[i];
       const float4 q = a.conic[i];
@@ -276,15 +297,13 @@ __device__ __forceinline__ float warp_reduce9(const float v[9], int lane) {
   return w4 + __shfl_xor_sync(0xffffffffu, w4, 1);
 }
 
-__global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(kBlock, 5) raster_bwd_kernel(BwdArgs a) {
+  __shared__ float4 s_raw[3][kBatchB];  // xyzo, conic, rgb of the next batch, in flight
   __shared__ float4 s_geo[kBatchB];  // px, py, a2, b2
   __shared__ float4 s_co[kBatchB];   // c2, opacity, A, B
   __shared__ float4 s_rgb[kBatchB];  // r, g, b, C
-  __shared__ float4 s_box[kBatchB];  // blend region of each staged entry
-  __shared__ float4 s_q1[kBatchB];
-  __shared__ float4 s_q2[kBatchB];
+  __shared__ uint8_t s_hit[kBatchB];   // region_mask of each staged entry
   __shared__ float s_acc[kBatchB][9];  // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
-  __shared__ uint32_t s_idx[kBatchB];
   __shared__ int s_maxlast;
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -294,8 +313,6 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
   const int u = tx0 + du, v = ty0 + dv;
   const bool inside = u < a.W && v < a.H;
   const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
-  const float wcx = (float)(tx0 + (warp & 1) * 8) + 4.0f;
-  const float wcy = (float)(ty0 + (warp >> 1) * 4) + 2.0f;
   const uint2 range = a.ranges[tile];
   const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
   float T = 1.0f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
@@ -315,35 +332,49 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
   if (lane == 0 && warp_last > 0) atomicMax(&s_maxlast, warp_last);
   __syncthreads();
   const int n = s_maxlast;  // list offsets [0, n) can hold a blend
-  for (int done = 0; done < n; done += kBatchB) {
-    // slot k of this batch holds list offset n - 1 - done - k (back to front)
-    __syncthreads();
-    for (int e = tid; e < kBatchB; e += kBlock) {
-      const int off = n - 1 - done - e;
-      if (off >= 0) {
-        const uint32_t i = a.vals[range.x + off];
-        const float4 g = a.xyzo[i];
-        const float4 q = a.conic[i];
-        const float4 c = a.rgb[i];
-        const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
-                    c2 = __fmul_rn(q.z, kHalfNegLog2e);
-        s_geo[e] = make_float4(g.x, g.y, a2, b2);
-        s_co[e] = make_float4(c2, g.w, q.x, q.y);
-        s_rgb[e] = make_float4(c.x, c.y, c.z, q.z);
-        const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
-        s_box[e] = r.box;
-        s_q1[e] = r.q1;
-        s_q2[e] = r.q2;
-        s_idx[e] = i;
-      }
-#pragma unroll
-      for (int j = 0; j < 9; ++j) s_acc[e][j] = 0.0f;
+  // Slot k of the batch that starts at `done` holds list offset
+  // n - 1 - done - k (back to front); thread tid owns slot tid. The records
+  // of the next batch are copied into s_raw while this one is processed and
+  // the indices of the batch after it are loaded into a register.
+  const uint32_t* lv = a.vals + range.x;
+  auto index_of = [&](int d) { return n - 1 - d - tid >= 0 ? lv[n - 1 - d - tid] : 0u; };
+  auto fetch = [&](int d, uint32_t i) {
+    if (n - 1 - d - tid >= 0) {
+      cp_async16(&s_raw[0][tid], a.xyzo + i);
+      cp_async16(&s_raw[1][tid], a.conic + i);
+      cp_async16(&s_raw[2][tid], a.rgb + i);
     }
+    cp_async_commit();
+  };
+  uint32_t icur = index_of(0);
+  fetch(0, icur);
+  uint32_t inext = index_of(kBatchB);
+  for (int done = 0; done < n; done += kBatchB) {
+    cp_async_wait_all();
+    const bool have = n - 1 - done - tid >= 0;
+    if (have) {
+      const int e = tid;
+      const float4 g = s_raw[0][e];
+      const float4 q = s_raw[1][e];
+      const float4 c = s_raw[2][e];
+      const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
+                  c2 = __fmul_rn(q.z, kHalfNegLog2e);
+      s_geo[e] = make_float4(g.x, g.y, a2, b2);
+      s_co[e] = make_float4(c2, g.w, q.x, q.y);
+      s_rgb[e] = make_float4(c.x, c.y, c.z, q.z);
+      s_hit[e] = (uint8_t)region_mask(blend_region(g.x, g.y, a2, b2, c2, g.w), tx0, ty0);
+    }
+#pragma unroll
+    for (int j = 0; j < 9; ++j) s_acc[tid][j] = 0.0f;
+    const uint32_t ithis = icur;
+    icur = inext;
+    fetch(done + kBatchB, icur);
+    inext = index_of(done + 2 * kBatchB);
     __syncthreads();
     const int m = min(kBatchB, n - done);
     for (int c0 = 0; c0 < m; c0 += 32) {
       const int j = c0 + lane;
-      const bool rel = j < m && (n - 1 - done - j) < warp_last && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy);
+      const bool rel = j < m && (n - 1 - done - j) < warp_last && ((s_hit[j] >> warp) & 1u);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
       while (msk) {
         const int k = c0 + __ffs(msk) - 1;
@@ -394,22 +425,33 @@ __global__ void __launch_bounds__(kBlock) raster_bwd_kernel(BwdArgs a) {
       }
     }
     __syncthreads();
-    for (int e = tid; e < m; e += kBlock) {
+    // flush this thread's slot (only this thread touches it until the next
+    // batch's barrier)
+    if (have) {
       float r[9];
       bool any = false;
 #pragma unroll
       for (int j = 0; j < 9; ++j) {
-        r[j] = s_acc[e][j];
+        r[j] = s_acc[tid][j];
         any |= r[j] != 0.0f;
       }
       if (any) {
-        float4* dst = a.grad2d + 3 * (size_t)s_idx[e];
+        float4* dst = a.grad2d + 3 * (size_t)ithis;
         atomicAdd(dst, make_float4(r[0], r[1], r[2], 0.f));
         atomicAdd(dst + 1, make_float4(r[3], r[4], r[5], 0.f));
         atomicAdd(dst + 2, make_float4(r[6], r[7], r[8], 0.f));
       }
     }
   }
+  cp_async_wait_all();  // no copy outlives the CTA
+}
+
+// Five CTAs of up to ~34 KB each share an SM: ask for the largest shared-memory
+// carveout (a preference; the launch is valid without it).
+template <typename K>
+bool prefer_shared(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
 }
 
 }  // namespace
@@ -423,6 +465,8 @@ cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const ui
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.image = image; a.final_T = final_T; a.n_contrib = n_contrib; a.last = last;
+  static const bool carve = prefer_shared(raster_fwd_kernel);
+  (void)carve;
   raster_fwd_kernel<<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
@@ -440,6 +484,8 @@ cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const ui
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d;
+  static const bool carve = prefer_shared(raster_bwd_kernel);
+  (void)carve;
   raster_bwd_kernel<<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();

@@ -23,9 +23,11 @@ namespace {
 
 constexpr int kTile = 16;
 constexpr int kBlock = kTile * kTile;
+// Backward CTA: 4 warps, two pixels per thread.
+constexpr int kBlockB = kBlock / 2;
 // List entries staged in shared memory per CTA-wide step: one per thread.
 constexpr int kBatchF = kBlock;
-constexpr int kBatchB = kBlock;
+constexpr int kBatchB = kBlockB;
 
 // 16-byte asynchronous global -> shared copy (L2 only), its commit and the
 // wait for all of this thread's outstanding copies.
@@ -93,17 +95,17 @@ __device__ __forceinline__ BlendRegion blend_region(float px, float py, float a2
 }
 
 // Can the Gaussian blend at a pixel centre of the warp block with centre
-// (wcx, wcy) and half extents (3.5, 1.5)? Box test, then (when enabled) the
+// (wcx, wcy) and half extents (hwx, hwy)? Box test, then (when enabled) the
 // minimum of the quadratic form over the rectangle of offsets d = (px, py) -
 // pixel centre: 0 if the rectangle holds the centre, else the least of the
 // four edges' one-dimensional minima.
 __device__ __forceinline__ bool region_hits(const float4 b, const float4 q1, const float4 q2, float wcx,
-                                            float wcy) {
+                                            float wcy, float hwx, float hwy) {
   const float ux = b.x - wcx, uy = b.y - wcy;
-  if (!(fabsf(ux) - 3.5f <= b.z && fabsf(uy) - 1.5f <= b.w)) return false;
+  if (!(fabsf(ux) - hwx <= b.z && fabsf(uy) - hwy <= b.w)) return false;
   if (!(q1.w < __int_as_float(0x7f800000))) return true;
-  const float dx0 = ux - 3.5f - q2.z, dx1 = ux + 3.5f + q2.z;
-  const float dy0 = uy - 1.5f - q2.z, dy1 = uy + 1.5f + q2.z;
+  const float dx0 = ux - hwx - q2.z, dx1 = ux + hwx + q2.z;
+  const float dy0 = uy - hwy - q2.z, dy1 = uy + hwy + q2.z;
   if (dx0 <= 0.0f && dx1 >= 0.0f && dy0 <= 0.0f && dy1 >= 0.0f) return true;
   const float m00 = q1.x, m01 = q1.y, m11 = q1.z;
   auto qf = [&](float dx, float dy) { return fmaf(m00 * dx, dx, fmaf(2.0f * m01 * dx, dy, m11 * dy * dy)); };
@@ -113,20 +115,10 @@ __device__ __forceinline__ bool region_hits(const float4 b, const float4 q1, con
   return best <= q1.w;
 }
 
-// Centre of the 8x4 block of pixel centres of warp w in the tile at (tx0, ty0).
+// Centre of the 8x4 block of pixel centres of forward warp w in the tile at
+// (tx0, ty0).
 __device__ __forceinline__ float block_cx(int tx0, int w) { return (float)(tx0 + (w & 1) * 8) + 4.0f; }
 __device__ __forceinline__ float block_cy(int ty0, int w) { return (float)(ty0 + (w >> 1) * 4) + 2.0f; }
-
-// Bit w set: the region can reach a pixel centre of warp w's block (the
-// test each warp would make, made once by the thread that stages the entry,
-// so the CTA keeps one byte per entry instead of the region itself).
-__device__ __forceinline__ uint32_t region_mask(const BlendRegion& r, int tx0, int ty0) {
-  uint32_t m = 0;
-#pragma unroll
-  for (int w = 0; w < kBlock / 32; ++w)
-    if (region_hits(r.box, r.q1, r.q2, block_cx(tx0, w), block_cy(ty0, w))) m |= 1u << w;
-  return m;
-}
 
 struct FwdArgs {
   const float4* xyzo;
@@ -188,7 +180,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
     for (int c0 = 0; c0 < m; c0 += 32) {
       if (__all_sync(0xffffffffu, done)) break;
       const int j = c0 + lane;
-      const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy);
+      const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy, 3.5f, 1.5f);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
       // Branch-free body: a lane that skips the pair (alpha < 1/255) or has
       // already stopped blends with alpha 0, which leaves C, T and the counts
@@ -297,36 +289,115 @@ __device__ __forceinline__ float warp_reduce9(const float v[9], int lane) {
   return w4 + __shfl_xor_sync(0xffffffffu, w4, 1);
 }
 
-__global__ void __launch_bounds__(kBlock, 5) raster_bwd_kernel(BwdArgs a) {
+// State of one pixel in the backward walk.
+struct BwdPixel {
+  float xc, yc;     // pixel centre
+  float T;          // transmittance in front of the current entry
+  float R0, R1, R2; // colour accumulated behind it (background included)
+  float g0, g1, g2; // dL/dimage
+  int last;         // 1 + list offset of its last blend (0: none)
+};
+
+__device__ __forceinline__ BwdPixel load_bwd_pixel(const BwdArgs& a, int u, int v, size_t P) {
+  BwdPixel p;
+  p.xc = __fadd_rn((float)u, 0.5f);
+  p.yc = __fadd_rn((float)v, 0.5f);
+  p.R0 = a.bg0;
+  p.R1 = a.bg1;
+  p.R2 = a.bg2;
+  p.T = 1.0f;
+  p.g0 = p.g1 = p.g2 = 0.0f;
+  p.last = 0;
+  if (u < a.W && v < a.H) {
+    const size_t pix = (size_t)v * a.W + u;
+    p.T = a.final_T[pix];
+    p.last = a.last[pix];
+    p.g0 = a.dL_dimage[pix];
+    p.g1 = a.dL_dimage[P + pix];
+    p.g2 = a.dL_dimage[2 * P + pix];
+  }
+  return p;
+}
+
+// One (pixel, entry) step of the backward walk: recompute alpha exactly as
+// the forward did, step T and R back over the entry and add the pixel's nine
+// gradient terms (mean2D x, y, opacity, conic A, B, C, colour r, g, b) to
+// gv (kFirst: gv is overwritten). A pair that was not a blend of the forward
+// (past the pixel's last blend, or alpha < 1/255) runs with alpha 0, which
+// leaves T and R unchanged, and adds zeros. Returns whether it was a blend.
+template <bool kFirst>
+__device__ __forceinline__ bool bwd_step(BwdPixel& p, const float4 g, const float4 co, const float4 c, int offk,
+                                         float gv[9]) {
+  const float dx = __fsub_rn(g.x, p.xc), dy = __fsub_rn(g.y, p.yc);
+  float qv = __fmul_rn(g.z, dx);
+  qv = __fmaf_rn(g.w, dy, qv);
+  float p2 = __fmul_rn(dx, qv);
+  const float wv = __fmul_rn(co.x, dy);
+  p2 = __fmaf_rn(wv, dy, p2);
+  const float e = exp2_raster(p2);
+  const float vv = __fmul_rn(co.y, e);
+  const float alpha = fminf(vv, kAlphaMax);
+  const bool contrib = offk < p.last && alpha >= kAlphaMin;
+  const float ab = contrib ? alpha : 0.0f;
+  const float oma = 1.0f - ab;
+  // transmittance in front of this entry (gradient values only)
+  p.T = contrib ? __fdividef(p.T, oma) : p.T;
+  const float wgt = ab * p.T;
+  const float Gk = p.T * (p.g0 * (c.x - p.R0) + p.g1 * (c.y - p.R1) + p.g2 * (c.z - p.R2));
+  const float Gm = (contrib && vv < kAlphaMax) ? Gk : 0.0f;  // no gradient through a clamped alpha
+  const float dp = Gm * ab;
+  const float A = co.z, B = co.w, Cc = c.w;
+  const float t0 = fmaf(A, dx, B * dy), t1 = fmaf(B, dx, Cc * dy);
+  const float ndp = -dp, hdx = -0.5f * dp * dx, ndx = ndp * dx, hdy = -0.5f * dp * dy;
+  if (kFirst) {
+    gv[0] = ndp * t0;
+    gv[1] = ndp * t1;
+    gv[2] = Gm * e;
+    gv[3] = hdx * dx;
+    gv[4] = ndx * dy;
+    gv[5] = hdy * dy;
+    gv[6] = p.g0 * wgt;
+    gv[7] = p.g1 * wgt;
+    gv[8] = p.g2 * wgt;
+  } else {
+    gv[0] = fmaf(ndp, t0, gv[0]);
+    gv[1] = fmaf(ndp, t1, gv[1]);
+    gv[2] = fmaf(Gm, e, gv[2]);
+    gv[3] = fmaf(hdx, dx, gv[3]);
+    gv[4] = fmaf(ndx, dy, gv[4]);
+    gv[5] = fmaf(hdy, dy, gv[5]);
+    gv[6] = fmaf(p.g0, wgt, gv[6]);
+    gv[7] = fmaf(p.g1, wgt, gv[7]);
+    gv[8] = fmaf(p.g2, wgt, gv[8]);
+  }
+  p.R0 = fmaf(c.x, ab, oma * p.R0);
+  p.R1 = fmaf(c.y, ab, oma * p.R1);
+  p.R2 = fmaf(c.z, ab, oma * p.R2);
+  return contrib;
+}
+
+// Backward CTA: 4 warps per tile, warp w owns the 8x8 block at
+// ((w & 1) * 8, (w >> 1) * 8) and lane l its pixels (l & 7, l >> 3) and
+// (l & 7, (l >> 3) + 4). One warp step handles one entry for 64 pixels, so
+// the warp sum of the gradient terms is paid once per 64 pixels.
+__global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
   __shared__ float4 s_raw[3][kBatchB];  // xyzo, conic, rgb of the next batch, in flight
-  __shared__ float4 s_geo[kBatchB];  // px, py, a2, b2
-  __shared__ float4 s_co[kBatchB];   // c2, opacity, A, B
-  __shared__ float4 s_rgb[kBatchB];  // r, g, b, C
-  __shared__ uint8_t s_hit[kBatchB];   // region_mask of each staged entry
-  __shared__ float s_acc[kBatchB][9];  // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
+  __shared__ float4 s_geo[kBatchB];     // px, py, a2, b2
+  __shared__ float4 s_co[kBatchB];      // c2, opacity, A, B
+  __shared__ float4 s_rgb[kBatchB];     // r, g, b, C
+  __shared__ uint8_t s_hit[kBatchB];    // bit w: the entry can blend in warp w's block
+  __shared__ float s_acc[kBatchB][9];   // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
   __shared__ int s_maxlast;
   const int tile = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int du, dv;
-  tile_pixel(tid, du, dv);
   const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
-  const int u = tx0 + du, v = ty0 + dv;
-  const bool inside = u < a.W && v < a.H;
-  const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
+  const int u = tx0 + (warp & 1) * 8 + (lane & 7), v = ty0 + (warp >> 1) * 8 + (lane >> 3);
   const uint2 range = a.ranges[tile];
-  const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
-  float T = 1.0f, g0 = 0.f, g1 = 0.f, g2 = 0.f;
-  int my_last = 0;
-  if (inside) {
-    T = a.final_T[pix];
-    my_last = a.last[pix];
-    g0 = a.dL_dimage[pix];
-    g1 = a.dL_dimage[P + pix];
-    g2 = a.dL_dimage[2 * P + pix];
-  }
-  const int warp_last = __reduce_max_sync(0xffffffffu, my_last);
+  const size_t P = (size_t)a.W * a.H;
+  BwdPixel p0 = load_bwd_pixel(a, u, v, P);
+  BwdPixel p1 = load_bwd_pixel(a, u, v + 4, P);
+  const int warp_last = __reduce_max_sync(0xffffffffu, max(p0.last, p1.last));
   const Reduce9Slot slot = reduce9_slot(lane);
-  float R0 = a.bg0, R1 = a.bg1, R2 = a.bg2;
   if (tid == 0) s_maxlast = 0;
   __syncthreads();
   if (lane == 0 && warp_last > 0) atomicMax(&s_maxlast, warp_last);
@@ -362,7 +433,14 @@ __global__ void __launch_bounds__(kBlock, 5) raster_bwd_kernel(BwdArgs a) {
       s_geo[e] = make_float4(g.x, g.y, a2, b2);
       s_co[e] = make_float4(c2, g.w, q.x, q.y);
       s_rgb[e] = make_float4(c.x, c.y, c.z, q.z);
-      s_hit[e] = (uint8_t)region_mask(blend_region(g.x, g.y, a2, b2, c2, g.w), tx0, ty0);
+      const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
+      uint32_t hit = 0;
+#pragma unroll
+      for (int w = 0; w < kBlockB / 32; ++w) {
+        const float bcx = (float)(tx0 + (w & 1) * 8) + 4.0f, bcy = (float)(ty0 + (w >> 1) * 8) + 4.0f;
+        if (region_hits(r.box, r.q1, r.q2, bcx, bcy, 3.5f, 3.5f)) hit |= 1u << w;
+      }
+      s_hit[e] = (uint8_t)hit;
     }
 #pragma unroll
     for (int j = 0; j < 9; ++j) s_acc[tid][j] = 0.0f;
@@ -380,45 +458,13 @@ __global__ void __launch_bounds__(kBlock, 5) raster_bwd_kernel(BwdArgs a) {
         const int k = c0 + __ffs(msk) - 1;
         msk &= msk - 1;
         const int offk = n - 1 - done - k;
-        // Branch-free body: a lane whose pair is not a blend of the forward
-        // (past its last blend, or alpha < 1/255) runs with alpha 0, which
-        // leaves T and R unchanged, and its terms are masked to zero.
         const float4 g = s_geo[k];
         const float4 co = s_co[k];
         const float4 c = s_rgb[k];
-        const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
-        float qv = __fmul_rn(g.z, dx);
-        qv = __fmaf_rn(g.w, dy, qv);
-        float p2 = __fmul_rn(dx, qv);
-        const float wv = __fmul_rn(co.x, dy);
-        p2 = __fmaf_rn(wv, dy, p2);
-        const float e = exp2_raster(p2);
-        const float vv = __fmul_rn(co.y, e);
-        const float alpha = fminf(vv, kAlphaMax);
-        const bool contrib = offk < my_last && alpha >= kAlphaMin;
-        const float ab = contrib ? alpha : 0.0f;
-        const float oma = 1.0f - ab;
-        // transmittance in front of this Gaussian (gradient values only)
-        T = contrib ? __fdividef(T, oma) : T;
-        const float wgt = ab * T;
         float gv[9];
-        gv[6] = g0 * wgt;
-        gv[7] = g1 * wgt;
-        gv[8] = g2 * wgt;
-        const float Gk = T * (g0 * (c.x - R0) + g1 * (c.y - R1) + g2 * (c.z - R2));
-        const float Gm = (contrib && vv < kAlphaMax) ? Gk : 0.0f;  // no gradient through a clamped alpha
-        gv[2] = Gm * e;
-        const float dp = Gm * ab;
-        const float A = co.z, B = co.w, Cc = c.w;
-        gv[0] = -dp * fmaf(A, dx, B * dy);
-        gv[1] = -dp * fmaf(B, dx, Cc * dy);
-        gv[3] = -0.5f * dp * dx * dx;
-        gv[4] = -dp * dx * dy;
-        gv[5] = -0.5f * dp * dy * dy;
-        R0 = fmaf(c.x, ab, oma * R0);
-        R1 = fmaf(c.y, ab, oma * R1);
-        R2 = fmaf(c.z, ab, oma * R2);
-        if (__any_sync(0xffffffffu, contrib)) {
+        const bool b0 = bwd_step<true>(p0, g, co, c, offk, gv);
+        const bool b1 = bwd_step<false>(p1, g, co, c, offk, gv);
+        if (__any_sync(0xffffffffu, b0 || b1)) {
           const float tot = warp_reduce9(gv, lane);
           if (slot.owner) atomicAdd(&s_acc[k][slot.idx], tot);
         }
@@ -446,14 +492,6 @@ __global__ void __launch_bounds__(kBlock, 5) raster_bwd_kernel(BwdArgs a) {
   cp_async_wait_all();  // no copy outlives the CTA
 }
 
-// Five CTAs of up to ~34 KB each share an SM: ask for the largest shared-memory
-// carveout (a preference; the launch is valid without it).
-template <typename K>
-bool prefer_shared(K kernel) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              (int)cudaSharedmemCarveoutMaxShared) == cudaSuccess;
-}
-
 }  // namespace
 
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
@@ -465,8 +503,6 @@ cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const ui
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.image = image; a.final_T = final_T; a.n_contrib = n_contrib; a.last = last;
-  static const bool carve = prefer_shared(raster_fwd_kernel);
-  (void)carve;
   raster_fwd_kernel<<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
@@ -484,9 +520,7 @@ cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const ui
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d;
-  static const bool carve = prefer_shared(raster_bwd_kernel);
-  (void)carve;
-  raster_bwd_kernel<<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
+  raster_bwd_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -319,32 +319,43 @@ __device__ __forceinline__ BwdPixel load_bwd_pixel(const BwdArgs& a, int u, int 
   return p;
 }
 
-// One (pixel, entry) step of the backward walk: recompute alpha exactly as
-// the forward did, step T and R back over the entry and add the pixel's nine
-// gradient terms (mean2D x, y, opacity, conic A, B, C, colour r, g, b) to
-// gv (kFirst: gv is overwritten). A pair that was not a blend of the forward
-// (past the pixel's last blend, or alpha < 1/255) runs with alpha 0, which
-// leaves T and R unchanged, and adds zeros. Returns whether it was a blend.
+// Alpha of one (pixel, entry) pair of the backward walk, recomputed exactly
+// as the forward computed it. A pair that was not a blend of the forward
+// (past the pixel's last blend, or alpha < 1/255) gets ab = 0.
+struct BwdEval {
+  float dx, dy, e, vv, ab;
+  bool contrib;
+};
+__device__ __forceinline__ BwdEval bwd_eval(const BwdPixel& p, const float4 g, const float4 co, int offk) {
+  BwdEval r;
+  r.dx = __fsub_rn(g.x, p.xc);
+  r.dy = __fsub_rn(g.y, p.yc);
+  float qv = __fmul_rn(g.z, r.dx);
+  qv = __fmaf_rn(g.w, r.dy, qv);
+  float p2 = __fmul_rn(r.dx, qv);
+  const float wv = __fmul_rn(co.x, r.dy);
+  p2 = __fmaf_rn(wv, r.dy, p2);
+  r.e = exp2_raster(p2);
+  r.vv = __fmul_rn(co.y, r.e);
+  const float alpha = fminf(r.vv, kAlphaMax);
+  r.contrib = offk < p.last && alpha >= kAlphaMin;
+  r.ab = r.contrib ? alpha : 0.0f;
+  return r;
+}
+
+// Step T and R of the pixel back over the entry and add its nine gradient
+// terms (mean2D x, y, opacity, conic A, B, C, colour r, g, b) to gv (kFirst:
+// gv is overwritten). With ab = 0 it leaves T and R unchanged and adds zeros.
 template <bool kFirst>
-__device__ __forceinline__ bool bwd_step(BwdPixel& p, const float4 g, const float4 co, const float4 c, int offk,
+__device__ __forceinline__ void bwd_grad(BwdPixel& p, const BwdEval& r, const float4 co, const float4 c,
                                          float gv[9]) {
-  const float dx = __fsub_rn(g.x, p.xc), dy = __fsub_rn(g.y, p.yc);
-  float qv = __fmul_rn(g.z, dx);
-  qv = __fmaf_rn(g.w, dy, qv);
-  float p2 = __fmul_rn(dx, qv);
-  const float wv = __fmul_rn(co.x, dy);
-  p2 = __fmaf_rn(wv, dy, p2);
-  const float e = exp2_raster(p2);
-  const float vv = __fmul_rn(co.y, e);
-  const float alpha = fminf(vv, kAlphaMax);
-  const bool contrib = offk < p.last && alpha >= kAlphaMin;
-  const float ab = contrib ? alpha : 0.0f;
+  const float dx = r.dx, dy = r.dy, ab = r.ab;
   const float oma = 1.0f - ab;
   // transmittance in front of this entry (gradient values only)
-  p.T = contrib ? __fdividef(p.T, oma) : p.T;
+  p.T = r.contrib ? __fdividef(p.T, oma) : p.T;
   const float wgt = ab * p.T;
   const float Gk = p.T * (p.g0 * (c.x - p.R0) + p.g1 * (c.y - p.R1) + p.g2 * (c.z - p.R2));
-  const float Gm = (contrib && vv < kAlphaMax) ? Gk : 0.0f;  // no gradient through a clamped alpha
+  const float Gm = (r.contrib && r.vv < kAlphaMax) ? Gk : 0.0f;  // no gradient through a clamped alpha
   const float dp = Gm * ab;
   const float A = co.z, B = co.w, Cc = c.w;
   const float t0 = fmaf(A, dx, B * dy), t1 = fmaf(B, dx, Cc * dy);
@@ -352,7 +363,7 @@ __device__ __forceinline__ bool bwd_step(BwdPixel& p, const float4 g, const floa
   if (kFirst) {
     gv[0] = ndp * t0;
     gv[1] = ndp * t1;
-    gv[2] = Gm * e;
+    gv[2] = Gm * r.e;
     gv[3] = hdx * dx;
     gv[4] = ndx * dy;
     gv[5] = hdy * dy;
@@ -362,7 +373,7 @@ __device__ __forceinline__ bool bwd_step(BwdPixel& p, const float4 g, const floa
   } else {
     gv[0] = fmaf(ndp, t0, gv[0]);
     gv[1] = fmaf(ndp, t1, gv[1]);
-    gv[2] = fmaf(Gm, e, gv[2]);
+    gv[2] = fmaf(Gm, r.e, gv[2]);
     gv[3] = fmaf(hdx, dx, gv[3]);
     gv[4] = fmaf(ndx, dy, gv[4]);
     gv[5] = fmaf(hdy, dy, gv[5]);
@@ -373,7 +384,6 @@ __device__ __forceinline__ bool bwd_step(BwdPixel& p, const float4 g, const floa
   p.R0 = fmaf(c.x, ab, oma * p.R0);
   p.R1 = fmaf(c.y, ab, oma * p.R1);
   p.R2 = fmaf(c.z, ab, oma * p.R2);
-  return contrib;
 }
 
 // Backward CTA: 4 warps per tile, warp w owns the 8x8 block at
@@ -460,14 +470,15 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
         const int offk = n - 1 - done - k;
         const float4 g = s_geo[k];
         const float4 co = s_co[k];
+        const BwdEval e0 = bwd_eval(p0, g, co, offk), e1 = bwd_eval(p1, g, co, offk);
+        // no pixel of the warp blended this entry: T and R stay, no terms
+        if (!__any_sync(0xffffffffu, e0.contrib || e1.contrib)) continue;
         const float4 c = s_rgb[k];
         float gv[9];
-        const bool b0 = bwd_step<true>(p0, g, co, c, offk, gv);
-        const bool b1 = bwd_step<false>(p1, g, co, c, offk, gv);
-        if (__any_sync(0xffffffffu, b0 || b1)) {
-          const float tot = warp_reduce9(gv, lane);
-          if (slot.owner) atomicAdd(&s_acc[k][slot.idx], tot);
-        }
+        bwd_grad<true>(p0, e0, co, c, gv);
+        bwd_grad<false>(p1, e1, co, c, gv);
+        const float tot = warp_reduce9(gv, lane);
+        if (slot.owner) atomicAdd(&s_acc[k][slot.idx], tot);
       }
     }
     __syncthreads();

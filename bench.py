@@ -233,7 +233,10 @@ def run_ours(args):
         counts.append(R.work_counts())
     torch.cuda.synchronize()
 
-    # ---- timed region: whole steps, device-resident inputs
+    # ---- timed region: whole steps, device-resident inputs. The bin/sort
+    # results (instance counts, statuses) stay on the device and are checked
+    # once after the region (Rasterizer.check raises on any failure).
+    R.deferred = True
     R.stage_events = {}
     launches0 = gs.gs_debug_kernel_launches()
     _barrier(world)
@@ -247,6 +250,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     _barrier(world)
     launches = gs.gs_debug_kernel_launches() - launches0
+    R.check()
     elapsed_ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
     stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in R.stage_events.items()}
     stage_n = {k: len(v) for k, v in R.stage_events.items()}
@@ -345,6 +349,7 @@ def e2e(args, scene, R, gimg, cams, bg, world):
     for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize()
+    R.check()
     _barrier(world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
@@ -352,6 +357,7 @@ def e2e(args, scene, R, gimg, cams, bg, world):
         step()
     ev1.record()
     torch.cuda.synchronize()
+    R.check()
     ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
     return {"value": 1000.0 * args.steps * len(cams) * world / ms, "unit": "frames/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms / args.steps}
@@ -360,14 +366,14 @@ def e2e(args, scene, R, gimg, cams, bg, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--ref-tile-stride", type=int, default=32,
                     help="reference arm: sample every n-th tile per step")
-    ap.add_argument("--cpu-tile-stride", type=int, default=8,
+    ap.add_argument("--cpu-tile-stride", type=int, default=1,
                     help="cpu_baseline: sample every n-th tile")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -103,9 +103,15 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
   return cuda_status(launch_preprocess(p, make_devcam(*cam), to_records(out), static_cast<cudaStream_t>(stream)));
 }
 
-GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
-                       uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
-                       int64_t* n_instances, void* workspace, size_t* workspace_bytes, void* stream) {
+namespace {
+// Shared by gs_bin_sort and gs_bin_sort_async: checks the arguments and
+// enqueues the whole bin/sort on the stream (no host round trip). Returns
+// GS_OK with *plan_out set, GS_OK with only *workspace_bytes set on a size
+// query (*enqueued = false), or an argument/launch error.
+int bin_sort_enqueue(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets, uint64_t* keys,
+                     uint32_t* vals, int64_t capacity, uint32_t* tile_ranges, void* workspace,
+                     size_t* workspace_bytes, void* stream, BinSortPlan* plan_out, bool* enqueued) {
+  *enqueued = false;
   if (!workspace_bytes || !camera_ok(cam) || n < 0 || n >= (int64_t(1) << 31) || capacity < 0 ||
       capacity >= (int64_t(1) << 30))
     return GS_ERR_INVALID_ARGUMENT;
@@ -117,31 +123,49 @@ GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, 
   }
   if (*workspace_bytes < plan.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return GS_ERR_INVALID_ARGUMENT;
-  if (!records_ok(in) || !n_instances || !tile_ranges || (capacity > 0 && (!keys || !vals)))
-    return GS_ERR_INVALID_ARGUMENT;
+  if (!records_ok(in) || !tile_ranges || (capacity > 0 && (!keys || !vals))) return GS_ERR_INVALID_ARGUMENT;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Records rec = to_records(in);
   cudaError_t e = launch_depth_order(rec, n, offsets, workspace, plan, g_stall_tile, s);
+  if (e == cudaSuccess) e = launch_emit_sort_ranges(rec, n, dc, keys, vals, tile_ranges, workspace, plan, g_stall_tile, s);
   if (e != cudaSuccess) return GS_ERR_CUDA;
+  *plan_out = plan;
+  *enqueued = true;
+  return GS_OK;
+}
+}  // namespace
+
+GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
+                       uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
+                       int64_t* n_instances, void* workspace, size_t* workspace_bytes, void* stream) {
+  if (workspace && !n_instances) return GS_ERR_INVALID_ARGUMENT;
+  BinSortPlan plan;
+  bool enqueued;
+  const int st = bin_sort_enqueue(in, n, cam, offsets, keys, vals, capacity, tile_ranges, workspace,
+                                  workspace_bytes, stream, &plan, &enqueued);
+  if (st != GS_OK || !enqueued) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int64_t total = 0;
-  e = cudaMemcpyAsync(&total, binsort_total_ptr(workspace, plan), sizeof(int64_t), cudaMemcpyDeviceToHost, s);
+  int32_t status = 0;
+  cudaError_t e = cudaMemcpyAsync(&total, binsort_total_ptr(workspace, plan), sizeof(int64_t),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(&status, binsort_status_ptr(workspace, plan), sizeof(int32_t), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return GS_ERR_CUDA;
   *n_instances = total;
-  if (total > capacity) return GS_ERR_CAPACITY;
-  e = launch_emit_sort_ranges(rec, n, dc, total, keys, vals, tile_ranges, workspace, plan, g_stall_tile, s);
-  if (e != cudaSuccess) return GS_ERR_CUDA;
-  int32_t status = 0;
-  e = cudaMemcpyAsync(&status, binsort_status_ptr(workspace, plan), sizeof(int32_t), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return GS_ERR_CUDA;
-  if (status != 0) {
-    // Leave every tile empty so that a raster call on these buffers reads nothing.
-    cudaMemsetAsync(tile_ranges, 0, (size_t)dc.TW * dc.TH * 2 * sizeof(uint32_t), s);
-    cudaStreamSynchronize(s);
-    return GS_ERR_DEVICE_TIMEOUT;
-  }
-  return GS_OK;
+  return status;  // GS_OK, GS_ERR_CAPACITY or GS_ERR_DEVICE_TIMEOUT
+}
+
+GS_API int gs_bin_sort_async(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
+                             uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
+                             int64_t* result, void* workspace, size_t* workspace_bytes, void* stream) {
+  BinSortPlan plan;
+  bool enqueued;
+  const int st = bin_sort_enqueue(in, n, cam, offsets, keys, vals, capacity, tile_ranges, workspace,
+                                  workspace_bytes, stream, &plan, &enqueued);
+  if (st != GS_OK || !enqueued || !result) return st;
+  return cuda_status(launch_publish(workspace, plan, result, static_cast<cudaStream_t>(stream)));
 }
 
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,

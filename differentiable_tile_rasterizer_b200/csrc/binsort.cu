@@ -12,7 +12,7 @@
 //
 // Each sort pass is one "onesweep" kernel: a CTA takes the next 4096-key tile
 // (atomic ticket, so all earlier tiles are already resident), ranks its keys
-// per digit with warp match-any, publishes its per-digit counts and finds its
+// per digit with warp ballots, publishes its per-digit counts and finds its
 // global offsets by decoupled look-back over its predecessors' counts, then
 // scatters through shared memory so that writes of equal digits are
 // contiguous. Every look-back wait is bounded: past the limit the CTA records
@@ -111,6 +111,14 @@ __device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// Instances to emit and sort, read on the device so that no host round trip
+// sits between the count and the sort: the scan's total, or none when it
+// exceeds the capacity (the emit kernel then records GS_ERR_CAPACITY).
+__device__ __forceinline__ int64_t live_instances(const int64_t* total, int64_t capacity) {
+  const int64_t t = *total;
+  return t <= capacity ? t : 0;
+}
+
 // ---------------------------------------------------------------- scans
 // Exclusive scan of tiles[order[r]] (order == nullptr: identity).
 __global__ void __launch_bounds__(kScanBlock) scan_reduce_kernel(const int32_t* tiles, const uint32_t* order,
@@ -173,7 +181,13 @@ __global__ void __launch_bounds__(256) depth_keys_kernel(const float4* xyzo, con
 // so the stores coalesce however many tiles each Gaussian touches.
 __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const int32_t* doff,
                                                    const int32_t* dtiles, const ushort4* rect, int64_t n,
-                                                   int TW, uint32_t* tkey, uint32_t* tval) {
+                                                   int TW, const int64_t* total, int64_t capacity,
+                                                   int32_t* status, uint32_t* tkey, uint32_t* tval) {
+  if (*status != 0) return;  // the depth order is not valid
+  if (*total > capacity) {    // nothing is emitted or sorted
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = GS_ERR_CAPACITY;
+    return;
+  }
   const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
   const int64_t r0 = r - lane;
@@ -182,8 +196,8 @@ __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const 
   uint32_t i = 0;
   if (r < n) {
     t = dtiles[r];
-    if (t > 0) {
-      i = order[r];
+    i = order[r];
+    if (t > 0 && i < n) {
       const ushort4 b = rect[i];
       x0 = b.x;
       y0 = b.y;
@@ -198,8 +212,8 @@ __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const 
     if (lane >= o) inc += v;
   }
   const int ex = inc - t;
-  const int total = __shfl_sync(0xffffffffu, inc, 31);
-  for (int p0 = 0; p0 < total; p0 += 32) {
+  const int wtotal = __shfl_sync(0xffffffffu, inc, 31);  // instances of the warp
+  for (int p0 = 0; p0 < wtotal; p0 += 32) {
     const int q = p0 + lane;
     int L = 0;
 #pragma unroll
@@ -212,7 +226,7 @@ __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const 
     const int x0L = __shfl_sync(0xffffffffu, x0, L);
     const int y0L = __shfl_sync(0xffffffffu, y0, L);
     const int bwL = __shfl_sync(0xffffffffu, bw, L);
-    if (q < total) {
+    if (q < wtotal) {
       const int li = q - exL;
       const int row = li / bwL;
       tkey[base + q] = (uint32_t)((y0L + row) * TW + x0L + (li - row * bwL));
@@ -222,9 +236,10 @@ __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const 
 }
 
 // Digit histograms of `passes` passes (digit p = bits [8p, 8p + 8)).
-__global__ void __launch_bounds__(256) digit_hist_kernel(const uint32_t* keys, int64_t n, int passes,
-                                                         uint32_t* hist) {
+__global__ void __launch_bounds__(256) digit_hist_kernel(const uint32_t* keys, int64_t n, const int64_t* n_dev,
+                                                         int64_t cap, int passes, uint32_t* hist) {
   __shared__ uint32_t sh[kMaxPasses * kRadix];
+  if (n_dev) n = live_instances(n_dev, cap);
   for (int b = threadIdx.x; b < kMaxPasses * kRadix; b += blockDim.x) sh[b] = 0;
   __syncthreads();
   for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
@@ -253,9 +268,12 @@ struct PassArgs {
   uint32_t* vout;
   uint64_t* kout64;           // final pass: (tile << 32) | depth bits of the record
   const float4* xyzo;         // records, for the depth bits of the final keys
+  int64_t n_records;          // values index records [0, n_records)
   const int32_t* tiles_in;    // optional: also write tiles_out[out] = tiles_in[value]
   int32_t* tiles_out;
-  int64_t n;
+  int64_t n;                  // keys, or (n_dev set) an upper bound on them
+  const int64_t* n_dev;       // optional: the key count on the device ...
+  int64_t cap;                // ... used only if it is <= cap (else none)
   int shift;
   const uint32_t* digit_off;  // [256] exclusive global digit offsets
   uint32_t* lookback;         // [n_tiles][256]
@@ -279,22 +297,35 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
   __syncthreads();
   const int64_t tile = s_tile;
   const int64_t base = tile * kSortTile;
+  const int64_t n = a.n_dev ? live_instances(a.n_dev, a.cap) : a.n;
+  // CTAs past the keys leave (tickets are taken in order, so none that
+  // stays waits on them)
+  if (base >= n) return;
 
   uint32_t key[kSortItems], val[kSortItems], dig[kSortItems], rank[kSortItems];
 #pragma unroll
   for (int j = 0; j < kSortItems; ++j) {
     const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
-    const bool ok = idx < a.n;
+    const bool ok = idx < n;
     key[j] = ok ? a.kin[idx] : 0u;
     val[j] = ok ? a.vin[idx] : 0u;
     dig[j] = ok ? ((key[j] >> a.shift) & 255u) : (uint32_t)kRadix;
   }
-  // Rank within the warp, in (j, lane) order = original order.
+  // Rank within the warp, in (j, lane) order = original order. The lanes
+  // holding the same digit are found with one ballot per digit bit (plus
+  // one for the out-of-range lanes): a fixed cost, where a match-any grows
+  // with the number of distinct digits in the warp.
   const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
   for (int j = 0; j < kSortItems; ++j) {
     const uint32_t d = dig[j];
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    const uint32_t vm = __ballot_sync(0xffffffffu, d < kRadix);
+    uint32_t peers = d < kRadix ? vm : ~vm;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const uint32_t bb = __ballot_sync(0xffffffffu, (d >> b) & 1u);
+      peers &= ((d >> b) & 1u) ? bb : ~bb;
+    }
     const uint32_t pre = d < kRadix ? s_whist[warp][d] : 0u;
     __syncwarp();
     if (d < kRadix && lane == 31 - __clz(peers)) s_whist[warp][d] = pre + __popc(peers);
@@ -353,26 +384,31 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
     }
   }
   __syncthreads();
-  const int64_t rem = a.n - base;
+  const int64_t rem = n - base;
   const int items = rem < kSortTile ? (int)rem : kSortTile;
   for (int s = tid; s < items; s += kSortBlock) {
     const uint32_t k = s_keys[s];
     const uint32_t dd = (k >> a.shift) & 255u;
     const uint32_t out = s_gbase[dd] + ((uint32_t)s - s_dstart[dd]);
     const uint32_t v = s_vals[s];
+    // (values are record indices; the bound only matters after a look-back
+    // timeout, when a slot can hold a stale value)
+    const bool vok = v < a.n_records;
     if (a.kout64) {
-      a.kout64[out] = ((uint64_t)k << 32) | __float_as_uint(a.xyzo[v].z);
+      a.kout64[out] = ((uint64_t)k << 32) | (vok ? __float_as_uint(a.xyzo[v].z) : kInvisibleKey);
     } else {
       a.kout[out] = k;
     }
     a.vout[out] = v;
-    if (a.tiles_out) a.tiles_out[out] = a.tiles_in[v];
+    if (a.tiles_out) a.tiles_out[out] = vok ? a.tiles_in[v] : 0;
   }
 }
 
 // Final keys when no tile pass runs (a single tile): (0 << 32) | depth bits.
-__global__ void __launch_bounds__(256) finalize_kernel(const uint32_t* tkey, const uint32_t* tval, int64_t n,
-                                                       const float4* xyzo, uint64_t* keys, uint32_t* vals) {
+__global__ void __launch_bounds__(256) finalize_kernel(const uint32_t* tkey, const uint32_t* tval,
+                                                       const int64_t* n_dev, int64_t cap, const float4* xyzo,
+                                                       uint64_t* keys, uint32_t* vals) {
+  const int64_t n = live_instances(n_dev, cap);
   const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= n) return;
   const uint32_t v = tval[k];
@@ -380,9 +416,20 @@ __global__ void __launch_bounds__(256) finalize_kernel(const uint32_t* tkey, con
   vals[k] = v;
 }
 
+// ---------------------------------------------------------------- results
+// Copies the instance count and the status word to the caller's result[2].
+__global__ void publish_kernel(const int64_t* total, const int32_t* status, int64_t* result) {
+  result[0] = *total;
+  result[1] = *status;
+}
+
 // ---------------------------------------------------------------- ranges
-__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, int64_t n, int64_t TT,
-                                                     uint2* ranges) {
+// Tiles stay empty when the sort failed (status set), so a raster call on
+// these buffers reads nothing.
+__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, const int64_t* n_dev, int64_t cap,
+                                                     const int32_t* status, int64_t TT, uint2* ranges) {
+  if (*status != 0) return;
+  const int64_t n = live_instances(n_dev, cap);
   const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= n) return;
   const uint64_t tile = keys[k] >> 32;
@@ -395,16 +442,19 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, int64
 
 // One LSD sort over `passes` 8-bit digits starting at bit 0, keys/values
 // ping-ponging between (k0, v0) and (k1, v1); the last pass writes to
-// (last_k or last_k64, last_v). Returns the kernels launched, -1 on error.
-int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint32_t* v1, int64_t n, int passes,
-                uint32_t* last_k, uint64_t* last_k64, uint32_t* last_v, const float4* xyzo,
-                const int32_t* tiles_in, int32_t* tiles_out, int64_t stall, cudaStream_t s) {
+// (last_k or last_k64, last_v). n keys, or with n_dev at most n keys, their
+// number read on the device (live_instances(n_dev, n)). Returns the kernels
+// launched, -1 on error.
+int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint32_t* v1, int64_t n,
+                const int64_t* n_dev, int passes, uint32_t* last_k, uint64_t* last_k64, uint32_t* last_v,
+                const float4* xyzo, int64_t n_records, const int32_t* tiles_in, int32_t* tiles_out, int64_t stall,
+                cudaStream_t s) {
   if (cudaMemsetAsync(w.hist, 0, kMaxPasses * kRadix * sizeof(uint32_t), s) != cudaSuccess) return -1;
   const int64_t nt = sort_tiles(n);
   if (cudaMemsetAsync(w.counters, 0, (64 + (size_t)passes * nt * kRadix) * sizeof(uint32_t), s) != cudaSuccess)
     return -1;
   const unsigned hgrid = (unsigned)std::min<int64_t>(grid_for(n, 256), 148 * 4);
-  digit_hist_kernel<<<hgrid, 256, 0, s>>>(k0, n, passes, w.hist);
+  digit_hist_kernel<<<hgrid, 256, 0, s>>>(k0, n, n_dev, n, passes, w.hist);
   digit_offsets_kernel<<<passes, kRadix, 0, s>>>(w.hist);
   uint32_t* kb[2] = {k0, k1};
   uint32_t* vb[2] = {v0, v1};
@@ -417,9 +467,12 @@ int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint3
     a.kout64 = last ? last_k64 : nullptr;
     a.vout = last ? last_v : vb[(p + 1) & 1];
     a.xyzo = xyzo;
+    a.n_records = n_records;
     a.tiles_in = tiles_in;
     a.tiles_out = last ? tiles_out : nullptr;
     a.n = n;
+    a.n_dev = n_dev;
+    a.cap = n;
     a.shift = 8 * p;
     a.digit_off = w.hist + p * kRadix;
     a.lookback = w.lookback + (size_t)p * nt * kRadix;
@@ -451,6 +504,13 @@ BinSortPlan binsort_plan(int64_t n, int64_t capacity, int64_t tiles) {
 }
 
 const int64_t* binsort_total_ptr(void* ws, const BinSortPlan& plan) { return carve(ws, plan).total; }
+
+cudaError_t launch_publish(void* ws, const BinSortPlan& plan, int64_t* result, cudaStream_t s) {
+  const SortWs w = carve(ws, plan);
+  publish_kernel<<<1, 1, 0, s>>>(w.total, w.status, result);
+  count_launches(1);
+  return cudaGetLastError();
+}
 const int32_t* binsort_status_ptr(void* ws, const BinSortPlan& plan) { return carve(ws, plan).status; }
 
 cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, void* ws,
@@ -470,8 +530,8 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
     depth_keys_kernel<<<grid_for(n, 256), 256, 0, s>>>(rec.xyzo, rec.tiles, n, w.dkey[0], w.dval[0]);
     // 4 passes: dkey[0] -> [1] -> [0] -> [1] -> [0]
     // the last pass also writes tiles_touched in depth order (dtiles)
-    const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, kDepthPasses, w.dkey[0],
-                              nullptr, w.dval[0], rec.xyzo, rec.tiles, w.dtiles, stall_tile, s);
+    const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, nullptr, kDepthPasses, w.dkey[0],
+                              nullptr, w.dval[0], rec.xyzo, n, rec.tiles, w.dtiles, stall_tile, s);
     if (k < 0) return cudaErrorLaunchFailure;
     launched += 1 + k;
     scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials);
@@ -487,27 +547,36 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam& cam, int64_t n_inst,
-                                    uint64_t* keys, uint32_t* vals, uint32_t* ranges, void* ws,
-                                    const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s) {
+cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam& cam, uint64_t* keys,
+                                    uint32_t* vals, uint32_t* ranges, void* ws, const BinSortPlan& plan,
+                                    int64_t stall_tile, cudaStream_t s) {
   SortWs w = carve(ws, plan);
   const int64_t TT = (int64_t)cam.TW * cam.TH;
+  const int64_t cap = plan.capacity;
   cudaError_t e = cudaMemsetAsync(ranges, 0, (size_t)TT * 2 * sizeof(uint32_t), s);
-  if (e != cudaSuccess || n_inst == 0) return e;
-  emit_kernel<<<grid_for(n, 256), 256, 0, s>>>(w.dval[0], w.doff, w.dtiles, rec.rect, n, cam.TW, w.tkey[0],
-                                               w.tval[0]);
-  int launched = 1;
-  if (plan.passes == 0) {
-    finalize_kernel<<<grid_for(n_inst, 256), 256, 0, s>>>(w.tkey[0], w.tval[0], n_inst, rec.xyzo, keys, vals);
+  if (e != cudaSuccess) return e;
+  int launched = 0;
+  if (n > 0) {
+    emit_kernel<<<grid_for(n, 256), 256, 0, s>>>(w.dval[0], w.doff, w.dtiles, rec.rect, n, cam.TW, w.total, cap,
+                                                 w.status, w.tkey[0], w.tval[0]);
     ++launched;
-  } else {
-    const int k = sort_passes(w, w.tkey[0], w.tval[0], w.tkey[1], w.tval[1], n_inst, plan.passes, nullptr, keys,
-                              vals, rec.xyzo, nullptr, nullptr, stall_tile, s);
-    if (k < 0) return cudaErrorLaunchFailure;
-    launched += k;
   }
-  ranges_kernel<<<grid_for(n_inst, 256), 256, 0, s>>>(keys, n_inst, TT, reinterpret_cast<uint2*>(ranges));
-  count_launches(launched + 1);
+  if (cap > 0) {
+    if (plan.passes == 0) {
+      finalize_kernel<<<grid_for(cap, 256), 256, 0, s>>>(w.tkey[0], w.tval[0], w.total, cap, rec.xyzo, keys,
+                                                         vals);
+      ++launched;
+    } else {
+      const int k = sort_passes(w, w.tkey[0], w.tval[0], w.tkey[1], w.tval[1], cap, w.total, plan.passes,
+                                nullptr, keys, vals, rec.xyzo, n, nullptr, nullptr, stall_tile, s);
+      if (k < 0) return cudaErrorLaunchFailure;
+      launched += k;
+    }
+    ranges_kernel<<<grid_for(cap, 256), 256, 0, s>>>(keys, w.total, cap, w.status, TT,
+                                                      reinterpret_cast<uint2*>(ranges));
+    ++launched;
+  }
+  count_launches(launched);
   return cudaGetLastError();
 }
 

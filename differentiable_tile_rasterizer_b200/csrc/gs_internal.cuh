@@ -90,9 +90,14 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
                                const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s);
 const int64_t* binsort_total_ptr(void* ws, const BinSortPlan& plan);
 const int32_t* binsort_status_ptr(void* ws, const BinSortPlan& plan);
-cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam& cam, int64_t n_inst,
-                                    uint64_t* keys, uint32_t* vals, uint32_t* ranges, void* ws,
-                                    const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s);
+// Emits the instances in depth order, sorts them by tile and writes the tile
+// ranges; the instance count is read on the device (none are emitted when it
+// exceeds plan.capacity: status GS_ERR_CAPACITY). Enqueue only.
+cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam& cam, uint64_t* keys,
+                                    uint32_t* vals, uint32_t* ranges, void* ws, const BinSortPlan& plan,
+                                    int64_t stall_tile, cudaStream_t s);
+// result[0] = instance count, result[1] = status, on the device.
+cudaError_t launch_publish(void* ws, const BinSortPlan& plan, int64_t* result, cudaStream_t s);
 
 // raster.cu
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,

@@ -23,7 +23,7 @@ GS_ERR_CUDA = 3
 GS_ERR_DEVICE_TIMEOUT = 4
 GS_ERR_UNSUPPORTED = 5
 
-EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_bin_sort",
+EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_bin_sort", "gs_bin_sort_async",
             "gs_rasterize_fwd", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
             "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
@@ -76,6 +76,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_cull.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P, PSZ, P]
         L.gs_preprocess.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, PCAM, PPROJ, P]
         L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
+        L.gs_bin_sort_async.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, P, P, PSZ, P]
         L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P]
         L.gs_rasterize_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P, P, P,
                                        P, P, P, P, P, P, P, P, P, P]
@@ -88,7 +89,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_debug_kernel_launches.argtypes = []
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
         L.gs_debug_set_stalled_sort_tile.restype = None
-        for name in ["gs_cull", "gs_preprocess", "gs_bin_sort", "gs_rasterize_fwd",
+        for name in ["gs_cull", "gs_preprocess", "gs_bin_sort", "gs_bin_sort_async", "gs_rasterize_fwd",
                      "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
             getattr(L, name).restype = ctypes.c_int
         _LIB = L
@@ -190,6 +191,16 @@ def gs_bin_sort(rec: GsProjected, n, cam: GsCamera, offsets, keys, vals, capacit
         return st, ni.value
     _check("gs_bin_sort", st)
     return st, ni.value
+
+
+def gs_bin_sort_async(rec: GsProjected, n, cam: GsCamera, offsets, keys, vals, capacity, tile_ranges,
+                      result, workspace, stream=None):
+    """Enqueues the bin/sort only; result [device] int64[2] receives (I, status).
+    Raises on argument errors."""
+    nbytes = ctypes.c_size_t(workspace.numel() * workspace.element_size())
+    _check("gs_bin_sort_async", load().gs_bin_sort_async(
+        ctypes.byref(rec), int(n), ctypes.byref(cam), _p(offsets), _p(keys), _p(vals), int(capacity),
+        _p(tile_ranges), _p(result), _p(workspace), ctypes.byref(nbytes), _stream(stream)))
 
 
 def gs_rasterize_fwd(rec: GsProjected, vals, tile_ranges, cam: GsCamera, bg, image, final_T,

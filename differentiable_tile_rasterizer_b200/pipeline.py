@@ -129,6 +129,12 @@ class Rasterizer:
         self.stage_events = None
         # Also produce the record-order scan of tiles_touched (gs_bin_sort offsets).
         self.want_offsets = False
+        # Deferred checking: forward() enqueues the bin/sort without a host
+        # round trip (gs_bin_sort_async); each view's (instances, status) stays
+        # in a device slot until check() reads them all at once.
+        self.deferred = False
+        self._results = torch.zeros((4096, 2), dtype=torch.int64, device=d)
+        self._n_pending = 0
 
     def _timed(self, stage):
         ev = self.stage_events
@@ -165,8 +171,15 @@ class Rasterizer:
         with self._timed("bin_sort"):
             return self._bin_sort(cam)
 
-    def _bin_sort(self, cam: gs.GsCamera) -> int:
+    def _bin_sort(self, cam: gs.GsCamera):
         offs = self.offsets if self.want_offsets else None
+        if self.deferred:
+            if self._n_pending == self._results.shape[0]:
+                self.check()
+            gs.gs_bin_sort_async(self._proj, self.N, cam, offs, self.keys, self.vals, self.capacity,
+                                 self.ranges, self._results[self._n_pending], self.sort_ws)
+            self._n_pending += 1
+            return None
         st, ni = gs.gs_bin_sort(self._proj, self.N, cam, offs, self.keys, self.vals, self.capacity,
                                 self.ranges, self.sort_ws, raise_on_capacity=False)
         if st == gs.GS_ERR_CAPACITY:
@@ -175,6 +188,25 @@ class Rasterizer:
                                     self.capacity, self.ranges, self.sort_ws)
         self.n_instances = ni
         return ni
+
+    def check(self) -> list:
+        """Instance counts of the views binned in deferred mode since the last
+        check (one host read). Raises GsError if one of them failed; after a
+        capacity failure the buffers have been grown, so repeating those views
+        succeeds."""
+        k = self._n_pending
+        self._n_pending = 0
+        if k == 0:
+            return []
+        res = self._results[:k].cpu().tolist()
+        counts = [int(ni) for ni, _ in res]
+        self.n_instances = counts[-1]
+        for ni, st in res:
+            if st == gs.GS_ERR_CAPACITY:
+                self._ensure_capacity(int(max(counts) * 1.25) + 1024)
+            if st != gs.GS_OK:
+                gs._check("gs_bin_sort_async", int(st))
+        return counts
 
     def raster_fwd(self, cam: gs.GsCamera, bg):
         with self._timed("raster_fwd"):

@@ -171,14 +171,34 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
  *   capacity     size of keys/vals, < 2^30
  *   tile_ranges  [device] [TW*TH][2] u32 out
  *   n_instances  [host] out: number of instances I
- * Synchronous: waits on `stream` once to read I and once at the end to read
- * the device status. Returns GS_ERR_CAPACITY (with *n_instances set, nothing
- * sorted) when I > capacity, GS_ERR_DEVICE_TIMEOUT if a look-back wait hit its
- * iteration limit (tile_ranges are then all empty). */
+ * The instance count is read on the device between the scan and the sort,
+ * so the whole call is enqueued at once; it then waits on `stream` once to
+ * read I and the device status. Returns GS_ERR_CAPACITY (with *n_instances
+ * set, nothing sorted, tile_ranges all empty) when I > capacity,
+ * GS_ERR_DEVICE_TIMEOUT if a look-back wait hit its iteration limit
+ * (tile_ranges are then all empty). */
 GS_API int gs_bin_sort(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
                        uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
                        int64_t* n_instances, void* workspace, size_t* workspace_bytes,
                        void* stream);
+
+/* gs_bin_sort without the wait: the same work and outputs, enqueued on
+ * `stream` only, so a caller can queue several views (and their raster
+ * calls) without a host round trip. The workspace is the same as
+ * gs_bin_sort's. The pages have no counterpart of this split; it exists
+ * because the instance count is data-dependent and reading it on the host
+ * stalls the device between views.
+ *   result       [device] i64[2] out, or NULL: result[0] = I, result[1] =
+ *                status (GS_OK, GS_ERR_CAPACITY: I > capacity, nothing sorted;
+ *                GS_ERR_DEVICE_TIMEOUT: a look-back wait hit its limit); in
+ *                both error cases tile_ranges are all empty, so a raster call
+ *                on them reads nothing.
+ * Grids of the instance kernels are sized for `capacity` (CTAs past I exit),
+ * so a capacity far above I costs idle CTAs. Argument errors are returned
+ * directly; device outcomes only through `result`. Asynchronous. */
+GS_API int gs_bin_sort_async(const gs_projected* in, int64_t n, const gs_camera* cam, int32_t* offsets,
+                             uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
+                             int64_t* result, void* workspace, size_t* workspace_bytes, void* stream);
 
 /* Forward compositing (tiled rasterization with alpha blending). For each
  * pixel, over its tile's sorted list: alpha = min(0.99, o exp(p)) with

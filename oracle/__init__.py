@@ -71,6 +71,8 @@ def _declare(L):
     L.or_raster_fwd.argtypes = [P, P, P, P, P, I32, I32, P, P, P, P, P, P, I64]
     L.or_raster_fwd.restype = ctypes.c_int
     L.or_raster_fwd_bruteforce.argtypes = [P, P, P, P, P, I64, I32, I32, P, P, P, P, P]
+    L.or_importance.argtypes = [P, P, P, P, P, I32, I32, P, P]
+    L.or_importance.restype = ctypes.c_int
     L.or_loss_frozen_f64.argtypes = [P, P, P, P, P, I32, I64, P, I64, P, I32, I32,
                                      P, P, P, P, P, P, P, P, P]
     L.or_loss_frozen_f64.restype = ctypes.c_double
@@ -201,6 +203,23 @@ def raster_fwd(rec, bins, cam, bg, tile_subset=None):
                         _p(image), _p(T), _p(nc), _p(last), _p(sub),
                         0 if sub is None else sub.size)
     return {"image": image, "final_T": T, "n_contrib": nc, "last": last}
+
+
+def importance(rec, bins, cam, n_gaussians, out=None):
+    """Cross-view visibility weights (BlitzGS write-up, section 2.2): adds this
+    view's sum over pixels of alpha*T per Gaussian (fp32 spec values of the
+    forward walk, summed in float64) to `out` (float64 [n_gaussians], zeros if
+    not given) and returns it. Record i belongs to Gaussian rec["active_idx"][i]
+    when the records come from a culled view, else to Gaussian i."""
+    if out is None:
+        out = np.zeros(n_gaussians, np.float64)
+    assert out.dtype == np.float64 and out.shape == (n_gaussians,)
+    act = rec.get("active_idx")
+    act = None if act is None else _c(act, np.int32)
+    vals = bins["vals"] if bins["vals"].size else np.zeros(1, np.uint32)
+    lib().or_importance(_p(rec["xyzo"]), _p(rec["conic"]), _p(rec["rgb"]), _p(vals),
+                        _p(_c(bins["ranges"], np.uint32)), cam.width, cam.height, _p(act), _p(out))
+    return out
 
 
 def raster_fwd_bruteforce(rec, cam, bg):

@@ -679,6 +679,39 @@ OR_API int or_raster_fwd(const float* xyzo, const float* conic, const float* rgb
   return 0;
 }
 
+// ---- importance weights (BlitzGS write-up, section 2.2 "模型层级重要性评分传递":
+// a cross-view visibility weight per Gaussian, its total contribution to the
+// rendered views). Read as the sum over the view's pixels of the blend weight
+// alpha T of each of its blends, with the fp32 spec values of the forward walk;
+// accumulated (+=) in double into importance[gaussian], where the Gaussian of
+// record i is active_idx[i] (or i when active_idx is null). Calling it once per
+// view sums over views.
+OR_API int or_importance(const float* xyzo, const float* conic, const float* rgb, const uint32_t* vals,
+                         const uint32_t* ranges, int width, int height, const int32_t* active_idx,
+                         double* importance) {
+  const int TW = (width + 15) / 16;
+  const int64_t TT = tile_count(width, height);
+  const Rec32 r{xyzo, conic, rgb};
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t tile = 0; tile < TT; ++tile) {
+    const int tx = (int)(tile % TW), ty = (int)(tile / TW);
+    const uint32_t start = ranges[2 * tile], end = ranges[2 * tile + 1];
+    for (int v = ty * 16; v < std::min(height, ty * 16 + 16); ++v)
+      for (int u = tx * 16; u < std::min(width, tx * 16 + 16); ++u) {
+        float T;
+        int n, lst;
+        walk_pixel(r, vals, start, end, (float)u + 0.5f, (float)v + 0.5f, T, n, lst,
+                   [&](uint32_t, uint32_t i, float alpha, bool, float) {
+                     const float wgt = alpha * T;  // T before this blend
+                     const int64_t g = active_idx ? active_idx[i] : (int64_t)i;
+#pragma omp atomic
+                     importance[g] += (double)wgt;
+                   });
+      }
+  }
+  return 0;
+}
+
 // ---- brute force forward: no tile lists. Per pixel, every visible Gaussian
 // whose rect contains the pixel's tile, in ascending (depth, index) order.
 OR_API int or_raster_fwd_bruteforce(const float* xyzo, const float* conic, const float* rgb,

@@ -300,6 +300,12 @@ def run_ours(args):
             "stages_ms_per_step": {k: v / args.steps for k, v in stage_ms.items()},
             "roofline": roof, "gpu_launches": int(launches), "clocks": clocks}
 
+    # ---- the importance pass: the forward that also sums alpha*T per Gaussian
+    if not args.no_importance:
+        fwd_ms = stage_ms["raster_fwd"] / max(stage_n["raster_fwd"], 1)
+        line["importance_pass"] = importance_pass(R, params, cams, bg, per_kernel["raster_fwd"] / len(poses),
+                                                  peak_alu, fwd_ms)
+
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
         line["e2e"] = e2e(args, scene, R, gimg, cams, bg, world)
@@ -322,6 +328,32 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def importance_pass(R, params, cams, bg, ops_per_view, peak_alu, fwd_ms, reps=10):
+    """Times gs_rasterize_fwd_importance over all poses (one pass of the
+    cross-view importance weights), per view, against the plain forward."""
+    import torch
+    imp = torch.zeros(R.N, dtype=torch.float32, device=R.dev)
+    for c in cams:  # warm-up
+        R.forward_importance(params, c, imp, bg)
+    torch.cuda.synchronize()
+    R.check()
+    R.stage_events = {}
+    for _ in range(reps):
+        imp.zero_()
+        for c in cams:
+            R.forward_importance(params, c, imp, bg)
+    torch.cuda.synchronize()
+    R.check()
+    ev = R.stage_events["raster_fwd_importance"]
+    R.stage_events = None
+    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    achieved = ops_per_view / (ms * 1e-3) / 1e12
+    return {"raster_ms_per_view": ms, "forward_raster_ms_per_view": fwd_ms, "overhead_vs_forward": ms / fwd_ms - 1.0,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
+                         "frac": achieved / peak_alu, "ops": "the forward's spec operations (21 E + 8 B)"},
+            "views": len(cams), "reps": reps}
 
 
 def e2e(args, scene, R, gimg, cams, bg, world):
@@ -379,6 +411,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--ref-tile-stride", type=int, default=32,
                     help="reference arm: sample every n-th tile per step")
+    ap.add_argument("--no-importance", action="store_true", help="skip timing the importance pass")
     ap.add_argument("--cpu-tile-stride", type=int, default=1,
                     help="cpu_baseline: sample every n-th tile")
     args = ap.parse_args()

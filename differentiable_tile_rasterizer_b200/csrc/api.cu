@@ -175,7 +175,20 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals, const 
     return GS_ERR_INVALID_ARGUMENT;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
-                                       n_contrib, last, static_cast<cudaStream_t>(stream)));
+                                       n_contrib, last, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,
+                                       const gs_camera* cam, const float* bg, const int32_t* active_idx,
+                                       float* image, float* final_T, int32_t* n_contrib, int32_t* last,
+                                       float* importance, void* stream) {
+  if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last ||
+      !importance)
+    return GS_ERR_INVALID_ARGUMENT;
+  const float b[3] = {bg[0], bg[1], bg[2]};
+  return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
+                                       n_contrib, last, importance, active_idx,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,

@@ -100,9 +100,12 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
 cudaError_t launch_publish(void* ws, const BinSortPlan& plan, int64_t* result, cudaStream_t s);
 
 // raster.cu
+// importance == nullptr: the plain forward. Otherwise also adds each
+// Gaussian's sum over pixels of alpha * T to importance[active_idx[i] or i].
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], float* image, float* final_T,
-                              int32_t* n_contrib, int32_t* last, cudaStream_t s);
+                              int32_t* n_contrib, int32_t* last, float* importance, const int32_t* active_idx,
+                              cudaStream_t s);
 cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], const float* final_T,
                               const int32_t* last, const float* dL_dimage, float4* grad2d,

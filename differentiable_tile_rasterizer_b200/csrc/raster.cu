@@ -132,9 +132,16 @@ struct FwdArgs {
   float* final_T;
   int32_t* n_contrib;
   int32_t* last;
+  float* importance;           // kImp: [N] += sum over pixels of alpha * T
+  const int32_t* active_idx;   // record -> Gaussian, or null (identity)
 };
 
+// kImp also accumulates each Gaussian's importance weight (the sum over the
+// view's pixels of its blend weights alpha * T): a warp sum per step, a
+// shared-memory sum per staged entry, one atomic per (Gaussian, tile).
+template <bool kImp>
 __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
+  __shared__ float s_imp[kImp ? kBatchF : 1];
   __shared__ float4 s_geo[kBatchF];  // px, py, a2, b2
   __shared__ float2 s_co[kBatchF];   // c2, opacity
   __shared__ float4 s_rgb[kBatchF];
@@ -156,13 +163,30 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int cnt = 0, lst = 0;
   bool done = !inside;
+  // importance: the entry this thread staged last, and its flush
+  uint32_t istaged = 0;
+  bool have_staged = false;
+  if (kImp) s_imp[tid] = 0.0f;
+  auto flush = [&]() {
+    if (kImp && have_staged) {
+      const float w = s_imp[tid];
+      if (w != 0.0f) atomicAdd(a.importance + (a.active_idx ? a.active_idx[istaged] : (int32_t)istaged), w);
+      s_imp[tid] = 0.0f;
+      have_staged = false;
+    }
+  };
   // (The forward stages with plain gathers: with five CTAs per SM the
   // others cover a staging CTA's latency.)
   for (int base = 0; base < n; base += kBatchF) {
     if (__syncthreads_count(done) == kBlock) break;
+    flush();  // the previous batch's sums are complete (barrier above)
     if (base + tid < n) {
       const int e = tid;
       const uint32_t i = a.vals[range.x + base + e];
+      if (kImp) {
+        istaged = i;
+        have_staged = true;
+      }
       const float4 g = a.xyzo[i];
       const float4 q = a.conic[i];
       const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
@@ -209,8 +233,18 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
         cnt += blend ? 1 : 0;
         lst = blend ? base + k + 1 : lst;
         done = done || T < kTMin;
+        if (kImp && __any_sync(0xffffffffu, blend)) {
+          float ws = wgt;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+          if (lane == 0 && ws != 0.0f) atomicAdd(&s_imp[k], ws);
+        }
       }
     }
+  }
+  if (kImp) {
+    __syncthreads();
+    flush();
   }
   if (inside) {
     const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
@@ -507,14 +541,19 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
 
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], float* image, float* final_T,
-                              int32_t* n_contrib, int32_t* last, cudaStream_t s) {
+                              int32_t* n_contrib, int32_t* last, float* importance, const int32_t* active_idx,
+                              cudaStream_t s) {
   FwdArgs a;
   a.xyzo = rec.xyzo; a.conic = rec.conic; a.rgb = rec.rgb;
   a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges);
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.image = image; a.final_T = final_T; a.n_contrib = n_contrib; a.last = last;
-  raster_fwd_kernel<<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
+  a.importance = importance; a.active_idx = active_idx;
+  if (importance)
+    raster_fwd_kernel<true><<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
+  else
+    raster_fwd_kernel<false><<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
 }

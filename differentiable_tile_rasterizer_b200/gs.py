@@ -24,7 +24,7 @@ GS_ERR_DEVICE_TIMEOUT = 4
 GS_ERR_UNSUPPORTED = 5
 
 EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_bin_sort", "gs_bin_sort_async",
-            "gs_rasterize_fwd", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
+            "gs_rasterize_fwd", "gs_rasterize_fwd_importance", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
             "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
 
@@ -78,6 +78,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
         L.gs_bin_sort_async.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, P, P, PSZ, P]
         L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P]
+        L.gs_rasterize_fwd_importance.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P, P, P]
         L.gs_rasterize_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P, P, P,
                                        P, P, P, P, P, P, P, P, P, P]
         L.gs_preprocess_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P,
@@ -90,6 +91,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
         L.gs_debug_set_stalled_sort_tile.restype = None
         for name in ["gs_cull", "gs_preprocess", "gs_bin_sort", "gs_bin_sort_async", "gs_rasterize_fwd",
+                     "gs_rasterize_fwd_importance",
                      "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
             getattr(L, name).restype = ctypes.c_int
         _LIB = L
@@ -209,6 +211,14 @@ def gs_rasterize_fwd(rec: GsProjected, vals, tile_ranges, cam: GsCamera, bg, ima
     _check("gs_rasterize_fwd", load().gs_rasterize_fwd(
         ctypes.byref(rec), _p(vals), _p(tile_ranges), ctypes.byref(cam), ctypes.cast(bgv, P),
         _p(image), _p(final_T), _p(n_contrib), _p(last), _stream(stream)))
+
+
+def gs_rasterize_fwd_importance(rec: GsProjected, vals, tile_ranges, cam: GsCamera, bg, active_idx, image,
+                                final_T, n_contrib, last, importance, stream=None):
+    bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
+    _check("gs_rasterize_fwd_importance", load().gs_rasterize_fwd_importance(
+        ctypes.byref(rec), _p(vals), _p(tile_ranges), ctypes.byref(cam), ctypes.cast(bgv, P), _p(active_idx),
+        _p(image), _p(final_T), _p(n_contrib), _p(last), _p(importance), _stream(stream)))
 
 
 def gs_rasterize_bwd(means, log_scales, quats, opacity_logits, sh, sh_degree, N, active_idx, n_active,

@@ -189,6 +189,25 @@ class Rasterizer:
         self.n_instances = ni
         return ni
 
+    def forward_importance(self, params: GaussianParams, cam, importance: torch.Tensor, bg=(0.0, 0.0, 0.0),
+                           lod_dist=0.0, importance_q=0.0) -> torch.Tensor:
+        """The forward of one view that also adds each Gaussian's importance
+        weight (sum over the view's pixels of alpha * T) to `importance`
+        (float32 [N] on the device; zero it once, call once per view)."""
+        c = cam if isinstance(cam, gs.GsCamera) else gs.camera(cam)
+        if (c.width, c.height) != (self.W, self.H):
+            raise ValueError("camera size differs from the rasterizer's")
+        if importance.dtype != torch.float32 or importance.numel() != self.N or not importance.is_cuda:
+            raise ValueError("importance must be a float32 CUDA tensor of N elements")
+        self.params, self.cam, self.bg = params, c, tuple(float(b) for b in bg)
+        self.cull(params, c, lod_dist, importance_q)
+        self.preprocess(params, c)
+        self.bin_sort(c)
+        with self._timed("raster_fwd_importance"):
+            gs.gs_rasterize_fwd_importance(self._proj, self.vals, self.ranges, c, self.bg, self.active_idx,
+                                           self.image, self.final_T, self.n_contrib, self.last, importance)
+        return self.image
+
     def check(self) -> list:
         """Instance counts of the views binned in deferred mode since the last
         check (one host read). Raises GsError if one of them failed; after a

@@ -217,6 +217,25 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
                             float* image, float* final_T, int32_t* n_contrib, int32_t* last,
                             void* stream);
 
+/* Importance pass: gs_rasterize_fwd plus the cross-view visibility weight
+ * of every Gaussian (BlitzGS write-up, section 2.2 "模型层级重要性评分传递":
+ * a weight per Gaussian for its total contribution over the views, used to
+ * suppress the least important Gaussians and as the weights of the
+ * view-level importance cull of gs_cull). The page prints no formula. It is
+ * read as the sum over the view's pixels of the blend weight alpha * T of
+ * each of the Gaussian's blends, with the forward's own fp32 values. The
+ * image outputs equal gs_rasterize_fwd's bit for bit.
+ *   active_idx   [device] [n_records] i32 or NULL: Gaussian of record i
+ *                (from gs_cull; NULL: record i is Gaussian i)
+ *   importance   [device] [N] f32 in/out: this view's weights are ADDED, so
+ *                zero it once and call once per view to sum over views
+ * The sums are fp32 atomics in an unspecified order (a warp sum, a CTA sum,
+ * then one atomic per (Gaussian, tile)). Asynchronous. */
+GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* vals,
+                                       const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                                       const int32_t* active_idx, float* image, float* final_T,
+                                       int32_t* n_contrib, int32_t* last, float* importance, void* stream);
+
 /* Backward pass: exact derivatives of the forward with every discrete decision
  * held fixed (visibility, tile lists, skips, the 0.99 clamp -- zero gradient
  * through a clamped alpha -- colour clamps, stop points).

@@ -82,6 +82,25 @@ def test_1m_1080p_sh3_bench_workload_pose0():
         grad_tol_check(R.grads[n].cpu().numpy(), ob["d_" + n], ob["m_" + n], what=n)
 
 
+def test_1m_1080p_sh3_importance_pass_pose0():
+    # importance weights of the whole view, every Gaussian (tolerance as in
+    # test_gpu_importance: the fp32 summation tree of positive terms)
+    sc = S.make_config(2)
+    cam = sc.cameras[0]
+    R = Rasterizer(sc.N, sc.sh_degree, cam.width, cam.height, capacity=6 * sc.N)
+    imp = torch.zeros(sc.N, dtype=torch.float32, device="cuda")
+    R.forward_importance(GaussianParams.from_scene(sc), cam, imp, sc.bg)
+    torch.cuda.synchronize()
+    got = imp.cpu().numpy().astype(np.float64)
+    rec = oracle.preprocess(sc, cam)
+    bins = oracle.bin_sort(rec, cam)
+    ref = oracle.importance(rec, bins, cam, sc.N)
+    bound = (16.0 + rec["tiles"]) * 2.0 ** -23 * ref + 1e-30
+    bad = np.abs(got - ref) > bound
+    assert not bad.any(), (bad.sum(), got[bad][:3], ref[bad][:3])
+    assert ref.sum() > 1e5
+
+
 def test_1m_1080p_sh3_bench_workload_other_poses_forward():
     sc = S.make_config(2)
     for pose in (1, 3):

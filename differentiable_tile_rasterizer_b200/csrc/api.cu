@@ -103,6 +103,24 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
   return cuda_status(launch_preprocess(p, make_devcam(*cam), to_records(out), static_cast<cudaStream_t>(stream)));
 }
 
+GS_API int gs_preprocess_multiview(const float* means, const float* log_scales, const float* quats,
+                                   const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                                   const gs_camera* cams, int n_views, const gs_projected* outs, void* stream) {
+  if (sh_degree < 0 || n_views < 0 || n_views > GS_MAX_VIEWS || (n_views > 0 && (!cams || !outs)))
+    return GS_ERR_INVALID_ARGUMENT;
+  if (sh_degree > 3) return GS_ERR_UNSUPPORTED;
+  if (!params_ok(means, log_scales, quats, opacity_logits, sh, N)) return GS_ERR_INVALID_ARGUMENT;
+  MultiViewArgs mv;
+  mv.n_views = n_views;
+  for (int v = 0; v < n_views; ++v) {
+    if (!camera_ok(&cams[v]) || !records_ok(&outs[v])) return GS_ERR_INVALID_ARGUMENT;
+    mv.cam[v] = make_devcam(cams[v]);
+    mv.out[v] = to_records(&outs[v]);
+  }
+  Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, nullptr, nullptr};
+  return cuda_status(launch_preprocess_multiview(p, mv, static_cast<cudaStream_t>(stream)));
+}
+
 namespace {
 // Shared by gs_bin_sort and gs_bin_sort_async: checks the arguments and
 // enqueues the whole bin/sort on the stream (no host round trip). Returns

@@ -77,6 +77,15 @@ cudaError_t launch_cull(const float* means, const float* importance, int64_t N, 
                         float lod_dist, float q, uint8_t* mask, int32_t* active_idx,
                         int32_t* n_active, void* ws, cudaStream_t s);
 
+// Several views of one preprocess pass (all N Gaussians, no cull).
+constexpr int kMaxViews = 16;
+struct MultiViewArgs {
+  DevCam cam[kMaxViews];
+  Records out[kMaxViews];
+  int n_views;
+};
+cudaError_t launch_preprocess_multiview(const Params& p, const MultiViewArgs& mv, cudaStream_t s);
+
 // binsort.cu
 struct BinSortPlan {
   int64_t n, capacity, tiles;

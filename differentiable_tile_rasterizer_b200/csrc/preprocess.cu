@@ -26,14 +26,46 @@ __device__ __forceinline__ float clamp_grid(float v, float hi) {
   return v < 0.0f ? 0.0f : (v > hi ? hi : v);
 }
 
+// Where project() reads a Gaussian's parameters: straight from the SoA
+// planes (single view: the SH planes are read only for Gaussians that get
+// that far) or from registers loaded once (several views).
+struct PlaneSource {
+  const Params& p;
+  int64_t g;
+  __device__ __forceinline__ float mean(int r) const { return p.means[r * p.N + g]; }
+  __device__ __forceinline__ float log_scale(int r) const { return p.log_scales[r * p.N + g]; }
+  __device__ __forceinline__ float quat(int r) const { return p.quats[r * p.N + g]; }
+  __device__ __forceinline__ float logit() const { return p.logits[g]; }
+  __device__ __forceinline__ float sh(int plane) const { return p.sh[(int64_t)plane * p.N + g]; }
+};
 template <int K>
-__device__ __forceinline__ void project(const Params& p, const DevCam& cam, int64_t g, Proj& o) {
+struct RegisterSource {
+  float m[3], l[3], q[4], lg, c[3 * K];
+  __device__ __forceinline__ void load(const Params& p, int64_t g) {
+#pragma unroll
+    for (int r = 0; r < 3; ++r) m[r] = p.means[r * p.N + g];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) l[r] = p.log_scales[r * p.N + g];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) q[r] = p.quats[r * p.N + g];
+    lg = p.logits[g];
+#pragma unroll
+    for (int k = 0; k < 3 * K; ++k) c[k] = p.sh[(int64_t)k * p.N + g];
+  }
+  __device__ __forceinline__ float mean(int r) const { return m[r]; }
+  __device__ __forceinline__ float log_scale(int r) const { return l[r]; }
+  __device__ __forceinline__ float quat(int r) const { return q[r]; }
+  __device__ __forceinline__ float logit() const { return lg; }
+  __device__ __forceinline__ float sh(int plane) const { return c[plane]; }
+};
+
+template <int K, class Src>
+__device__ __forceinline__ void project(const Src& src, const DevCam& cam, Proj& o) {
   o.visible = false;
-  const int64_t N = p.N;
-  const float mx = p.means[g], my = p.means[N + g], mz = p.means[2 * N + g];
-  const float l0 = p.log_scales[g], l1 = p.log_scales[N + g], l2 = p.log_scales[2 * N + g];
-  const float qw = p.quats[g], qx = p.quats[N + g], qy = p.quats[2 * N + g], qz = p.quats[3 * N + g];
-  const float logit = p.logits[g];
+  const float mx = src.mean(0), my = src.mean(1), mz = src.mean(2);
+  const float l0 = src.log_scale(0), l1 = src.log_scale(1), l2 = src.log_scale(2);
+  const float qw = src.quat(0), qx = src.quat(1), qy = src.quat(2), qz = src.quat(3);
+  const float logit = src.logit();
   if (!(finitef(mx) && finitef(my) && finitef(mz) && finitef(l0) && finitef(l1) && finitef(l2) &&
         finitef(qw) && finitef(qx) && finitef(qy) && finitef(qz) && finitef(logit)))
     return;
@@ -163,9 +195,9 @@ __device__ __forceinline__ void project(const Params& p, const DevCam& cam, int6
   sh_basis<K>(__fdiv_rn(dx, nd), __fdiv_rn(dy, nd), __fdiv_rn(dz, nd), Y);
 #pragma unroll
   for (int ch = 0; ch < 3; ++ch) {
-    float acc = __fmul_rn(Y[0], p.sh[(int64_t)ch * N + g]);
+    float acc = __fmul_rn(Y[0], src.sh(ch));
 #pragma unroll
-    for (int k = 1; k < K; ++k) acc = __fmaf_rn(Y[k], p.sh[(int64_t)(3 * k + ch) * N + g], acc);
+    for (int k = 1; k < K; ++k) acc = __fmaf_rn(Y[k], src.sh(3 * k + ch), acc);
     const float v = __fadd_rn(acc, 0.5f);
     o.rgb[ch] = v > 0.0f ? v : 0.0f;
   }
@@ -177,14 +209,8 @@ __device__ __forceinline__ void project(const Params& p, const DevCam& cam, int6
   o.x0 = x0; o.y0 = y0; o.x1 = x1; o.y1 = y1;
 }
 
-template <int K>
-__global__ void __launch_bounds__(256) preprocess_kernel(Params p, DevCam cam, Records out) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= p.N) return;
-  const int64_t na = p.n_active ? (int64_t)*p.n_active : p.N;
-  Proj o;
-  o.visible = false;
-  if (i < na) project<K>(p, cam, p.active_idx ? (int64_t)p.active_idx[i] : i, o);
+// One record: the projection, or zeros for a Gaussian that is culled.
+__device__ __forceinline__ void write_record(const Proj& o, const Records& out, int64_t i) {
   if (o.visible) {
     out.xyzo[i] = make_float4(o.px, o.py, o.depth, o.opacity);
     out.conic[i] = make_float4(o.A, o.B, o.C, 0.0f);
@@ -203,6 +229,33 @@ __global__ void __launch_bounds__(256) preprocess_kernel(Params p, DevCam cam, R
     out.tiles[i] = 0;
   }
 }
+
+template <int K>
+__global__ void __launch_bounds__(256) preprocess_kernel(Params p, DevCam cam, Records out) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.N) return;
+  const int64_t na = p.n_active ? (int64_t)*p.n_active : p.N;
+  Proj o;
+  o.visible = false;
+  if (i < na) project<K>(PlaneSource{p, p.active_idx ? (int64_t)p.active_idx[i] : i}, cam, o);
+  write_record(o, out, i);
+}
+
+// Several views in one pass: each Gaussian's 11 + 3K parameters are read from
+// HBM once, into registers, and projected into every view.
+template <int K>
+__global__ void __launch_bounds__(256) preprocess_multiview_kernel(Params p, MultiViewArgs mv) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= p.N) return;
+  RegisterSource<K> src;
+  src.load(p, i);
+  for (int v = 0; v < mv.n_views; ++v) {
+    Proj o;
+    project<K>(src, mv.cam[v], o);
+    write_record(o, mv.out[v], i);
+  }
+}
+
 
 // ------------------------------------------------------------------ backward
 
@@ -426,6 +479,19 @@ cudaError_t launch_preprocess(const Params& p, const DevCam& cam, const Records&
     case 1: preprocess_kernel<4><<<grid, 256, 0, s>>>(p, cam, out); break;
     case 2: preprocess_kernel<9><<<grid, 256, 0, s>>>(p, cam, out); break;
     default: preprocess_kernel<16><<<grid, 256, 0, s>>>(p, cam, out); break;
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_preprocess_multiview(const Params& p, const MultiViewArgs& mv, cudaStream_t s) {
+  if (p.N == 0 || mv.n_views == 0) return cudaSuccess;
+  const unsigned grid = grid_for(p.N, 256);
+  switch (p.sh_degree) {
+    case 0: preprocess_multiview_kernel<1><<<grid, 256, 0, s>>>(p, mv); break;
+    case 1: preprocess_multiview_kernel<4><<<grid, 256, 0, s>>>(p, mv); break;
+    case 2: preprocess_multiview_kernel<9><<<grid, 256, 0, s>>>(p, mv); break;
+    default: preprocess_multiview_kernel<16><<<grid, 256, 0, s>>>(p, mv); break;
   }
   count_launches(1);
   return cudaGetLastError();

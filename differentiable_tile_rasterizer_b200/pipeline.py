@@ -296,3 +296,47 @@ class Rasterizer:
                 "vals": self.vals[:I].cpu().numpy().view(np.uint32),
                 "ranges": self.ranges.cpu().numpy().view(np.uint32),
                 "offsets": self.offsets.cpu().numpy(), "n_instances": I}
+
+
+class MultiViewRenderer:
+    """Forward rendering of several views of one model: one pass over the
+    parameters projects every Gaussian into all views
+    (gs_preprocess_multiview), then each view runs its bin/sort and raster
+    forward on its own buffers (a Rasterizer per view). No cull: every
+    Gaussian is projected into every view."""
+
+    def __init__(self, N: int, sh_degree: int, cams, device=None, capacity: Optional[int] = None):
+        self.cams = [c if isinstance(c, gs.GsCamera) else gs.camera(c) for c in cams]
+        if not 0 < len(self.cams) <= gs.GS_MAX_VIEWS:
+            raise ValueError(f"1 .. {gs.GS_MAX_VIEWS} views per pass")
+        self.N, self.sh_degree = int(N), int(sh_degree)
+        self.views = [Rasterizer(N, sh_degree, c.width, c.height, device=device, capacity=capacity)
+                      for c in self.cams]
+        self.stage_events = None
+
+    def _timed(self, stage):
+        ev = self.stage_events
+        if ev is None:
+            return _NoTimer()
+        return _StageTimer(ev.setdefault(stage, []))
+
+    def forward(self, params: GaussianParams, bg=(0.0, 0.0, 0.0)) -> list:
+        bg = tuple(float(b) for b in bg)
+        with self._timed("preprocess_multiview"):
+            gs.gs_preprocess_multiview(params.means, params.log_scales, params.quats, params.opacity_logits,
+                                       params.sh, params.sh_degree, self.N, self.cams,
+                                       [R._proj for R in self.views])
+        for R, c in zip(self.views, self.cams):
+            R.params, R.cam, R.bg, R.culled = params, c, bg, False
+            with self._timed("bin_sort"):
+                R._bin_sort(c)
+            with self._timed("raster_fwd"):
+                gs.gs_rasterize_fwd(R._proj, R.vals, R.ranges, c, bg, R.image, R.final_T, R.n_contrib, R.last)
+        return [R.image for R in self.views]
+
+    def set_deferred(self, on: bool):
+        for R in self.views:
+            R.deferred = on
+
+    def check(self) -> list:
+        return [R.check() for R in self.views]

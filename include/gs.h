@@ -155,6 +155,28 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
                          const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
                          const gs_projected* out, void* stream);
 
+/* Views per gs_preprocess_multiview call. */
+#define GS_MAX_VIEWS 16
+
+/* gs_preprocess for several views in one pass over the parameters: each
+ * Gaussian's 11 + 3K parameters are read once and projected into every view
+ * (the batched multi-view step for rendering many poses of one model, as
+ * in the 10M-Gaussian eight-view 4K workload). Record i of view v is
+ * Gaussian i; there is no cull (every Gaussian of every view is
+ * projected), and outs[v] receives exactly what gs_preprocess with
+ * cams[v], active_idx = NULL writes. The pages print no kernel for this;
+ * the parameter layout and per-view records follow the Gsplat page's split
+ * of per-Gaussian projection from the raster stages.
+ *   cams         [host] [n_views] cameras (all may differ in size)
+ *   n_views      0 .. GS_MAX_VIEWS
+ *   outs         [host] [n_views] record sets, each of capacity N
+ * HBM traffic: (11 + 3K) * 4 bytes read + n_views * 64 bytes written per
+ * Gaussian, against n_views times both for separate calls. Asynchronous. */
+GS_API int gs_preprocess_multiview(const float* means, const float* log_scales, const float* quats,
+                                   const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                                   const gs_camera* cams, int n_views, const gs_projected* outs,
+                                   void* stream);
+
 /* Tile binning: one (key, value) per (Gaussian, tile) instance with
  * key = (tile_id << 32) | bits(depth) and value = record index, tiles in
  * row-major order within the record's rect, sorted stably by key (equal keys

@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from differentiable_tile_rasterizer_b200 import synthetic as S
-from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, Rasterizer
+from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, MultiViewRenderer, Rasterizer
 from tests.gpu_helpers import assert_bits, grad_tol_check
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -147,3 +147,18 @@ def test_10m_4k_sh3_forward_two_poses():
         _check_forward(sc, pose, R, n_tiles=200, seed=10 + pose)
         del R
         torch.cuda.empty_cache()
+
+
+def test_10m_4k_sh3_multiview_all_eight_poses():
+    # one parameter pass for the 8 views; views 0 and 5 checked in full
+    # (records, sort) and on sampled tiles (image)
+    sc = S.make_config(4)
+    mv = MultiViewRenderer(sc.N, sc.sh_degree, sc.cameras, capacity=6 * sc.N)
+    for R in mv.views:
+        R.want_offsets = True
+    mv.forward(GaussianParams.from_scene(sc), sc.bg)
+    torch.cuda.synchronize()
+    for pose in (0, 5):
+        _check_forward(sc, pose, mv.views[pose], n_tiles=200, seed=20 + pose)
+    del mv
+    torch.cuda.empty_cache()

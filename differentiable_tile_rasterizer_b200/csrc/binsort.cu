@@ -42,7 +42,6 @@ constexpr uint32_t kFlagAgg = 1u << 30;
 constexpr uint32_t kFlagInc = 2u << 30;
 constexpr uint32_t kSpinLimit = 1u << 20;
 constexpr uint32_t kInvisibleKey = 0xffffffffu;
-constexpr int kScanCounter = 32;  // counters[kScanCounter]: ticket of the fused scan/emit
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -58,6 +57,7 @@ struct SortWs {
   uint32_t* lookback;  // [passes][sort tiles][kRadix]
   uint32_t* dkey[2];   // [n] depth keys
   uint32_t* dval[2];   // [n] record indices
+  int32_t* doff;       // [n] instance offsets in depth order
   int32_t* dtiles;     // [n] tiles_touched in depth order
   uint32_t* tkey[2];   // [capacity] tile ids
   uint32_t* tval[2];   // [capacity] record indices
@@ -89,6 +89,8 @@ SortWs carve(void* ws, const BinSortPlan& p) {
     w.dval[k] = reinterpret_cast<uint32_t*>(c);
     c += align256((size_t)p.n * sizeof(uint32_t));
   }
+  w.doff = reinterpret_cast<int32_t*>(c);
+  c += align256((size_t)p.n * sizeof(int32_t));
   w.dtiles = reinterpret_cast<int32_t*>(c);
   c += align256((size_t)p.n * sizeof(int32_t));
   for (int k = 0; k < 2; ++k) {
@@ -172,154 +174,65 @@ __global__ void __launch_bounds__(256) depth_keys_kernel(const float4* xyzo, con
   val[i] = (uint32_t)i;
 }
 
-// Scan of tiles_touched in depth order, fused with the emission of the
-// instances and the histograms of their tile digits. A CTA takes the next
-// 4096 Gaussians of the depth order (atomic ticket), sums their tile counts,
-// finds its exclusive prefix by a bounded decoupled look-back over its
-// predecessors' sums (int64 words: flag in the top two bits), and then each
-// warp writes the instances of its Gaussians, 32 at a time, as one contiguous
-// run, each lane finding the Gaussian of its instance by a binary search over
-// the warp's prefix sums, so the stores coalesce however many tiles each
-// Gaussian touches. Tiles are row-major within each rect. Writes at or past
-// `capacity` are dropped; the last CTA publishes the total and records
-// GS_ERR_CAPACITY if it exceeds the capacity (nothing is then sorted).
-constexpr int kEmitBlock = 1024;  // 32 warps, 4 groups of 32 Gaussians each
-constexpr int kEmitItems = 4;
-constexpr int kEmitTile = kEmitBlock * kEmitItems;  // 4096, the scan tile
-constexpr int kEmitWarps = kEmitBlock / 32;
-static_assert(kEmitTile == kScanTile, "the scan look-back words are the partials array");
-constexpr uint64_t kScanAgg = 1ull << 62;
-constexpr uint64_t kScanInc = 2ull << 62;
-constexpr uint64_t kScanValMask = (1ull << 62) - 1ull;
-
-__device__ __forceinline__ uint64_t ld_relaxed64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_relaxed64(unsigned long long* p, uint64_t v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"((unsigned long long)v) : "memory");
-}
-
-__global__ void __launch_bounds__(kEmitBlock) scan_emit_kernel(const uint32_t* order, const int32_t* dtiles,
-                                                               const ushort4* rect, int64_t n, int TW,
-                                                               int64_t capacity, int passes,
-                                                               unsigned long long* lookback, uint32_t* counter,
-                                                               int64_t* total, int32_t* status, uint32_t* hist,
-                                                               uint32_t* tkey, uint32_t* tval) {
-  __shared__ uint32_t s_hist[4 * kRadix];  // tile digits of the (at most four) tile passes
-  __shared__ int64_t s_warp[kEmitWarps];
-  __shared__ int64_t s_prefix;
-  __shared__ uint32_t s_tile;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) s_tile = atomicAdd(counter, 1u);
-  for (int b = tid; b < 4 * kRadix; b += kEmitBlock) s_hist[b] = 0;
-  __syncthreads();
-  const int64_t tile = s_tile;
-  const int64_t wbase = tile * kEmitTile + (int64_t)warp * (kEmitItems * 32);
-  // tile counts of this warp's 128 Gaussians (clamped at 0: after a look-back
-  // timeout of the depth sort a slot can hold a stale value); read again,
-  // from cache, when emitting
-  auto count_of = [&](int64_t r) { return r < n ? max(dtiles[r], 0) : 0; };
-  int64_t wsum = 0;
-#pragma unroll
-  for (int j = 0; j < kEmitItems; ++j) wsum += count_of(wbase + j * 32 + lane);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-  if (lane == 0) s_warp[warp] = wsum;
-  __syncthreads();
-  if (tid == 0) {
-    int64_t cta = 0;
-    for (int w = 0; w < kEmitWarps; ++w) {
-      const int64_t x = s_warp[w];
-      s_warp[w] = cta;
-      cta += x;
-    }
-    int64_t excl = 0;
-    if (tile == 0) {
-      st_relaxed64(lookback, kScanInc | (uint64_t)cta);
-    } else {
-      st_relaxed64(lookback + tile, kScanAgg | (uint64_t)cta);
-      int64_t k = tile - 1;
-      uint32_t spins = 0;
-      while (true) {
-        const uint64_t sv = ld_relaxed64(lookback + k);
-        const uint64_t flag = sv & ~kScanValMask;
-        if (flag == 0) {
-          if (++spins > kSpinLimit) {
-            atomicExch(status, (int32_t)GS_ERR_DEVICE_TIMEOUT);
-            break;
-          }
-          __nanosleep(64);
-          continue;
-        }
-        excl += (int64_t)(sv & kScanValMask);
-        if (flag == kScanInc || k == 0) break;
-        --k;
-      }
-      st_relaxed64(lookback + tile, kScanInc | (uint64_t)(excl + cta));
-    }
-    s_prefix = excl;
-    if (tile == (int64_t)gridDim.x - 1) {
-      *total = excl + cta;
-      if (excl + cta > capacity) atomicCAS(status, 0, (int32_t)GS_ERR_CAPACITY);
+// Instances of the Gaussians in depth order, tiles row-major in each rect.
+// A warp writes the instances of its 32 consecutive Gaussians as one
+// contiguous run (their offsets are consecutive), each lane finding the
+// Gaussian of its instance by a binary search over the warp's prefix sums,
+// so the stores coalesce however many tiles each Gaussian touches.
+__global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const int32_t* doff,
+                                                   const int32_t* dtiles, const ushort4* rect, int64_t n,
+                                                   int TW, const int64_t* total, int64_t capacity,
+                                                   int32_t* status, uint32_t* tkey, uint32_t* tval) {
+  if (*status != 0) return;  // the depth order is not valid
+  if (*total > capacity) {    // nothing is emitted or sorted
+    if (blockIdx.x == 0 && threadIdx.x == 0) *status = GS_ERR_CAPACITY;
+    return;
+  }
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int64_t r0 = r - lane;
+  if (r0 >= n) return;  // warp-uniform
+  int t = 0, x0 = 0, y0 = 0, bw = 1;
+  uint32_t i = 0;
+  if (r < n) {
+    t = dtiles[r];
+    i = order[r];
+    if (t > 0 && i < n) {
+      const ushort4 b = rect[i];
+      x0 = b.x;
+      y0 = b.y;
+      bw = (int)b.z - (int)b.x;
     }
   }
-  __syncthreads();
-  int64_t run = s_prefix + s_warp[warp];
-#pragma unroll 1
-  for (int j = 0; j < kEmitItems; ++j) {
-    const int64_t r = wbase + j * 32 + lane;
-    const int t = count_of(r);
-    int x0 = 0, y0 = 0, bw = 1;
-    uint32_t i = 0;
-    if (t > 0) {
-      i = order[r];
-      if (i < n) {
-        const ushort4 b = rect[i];
-        x0 = b.x;
-        y0 = b.y;
-        bw = max((int)b.z - (int)b.x, 1);
-      }
-    }
-    int inc = t;
+  const int64_t base = doff[r0];
+  int inc = t;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += v;
-    }
-    const int ex = inc - t;
-    const int gtotal = __shfl_sync(0xffffffffu, inc, 31);  // instances of these 32 Gaussians
-    for (int p0 = 0; p0 < gtotal; p0 += 32) {
-      const int q = p0 + lane;
-      int L = 0;
-#pragma unroll
-      for (int st = 16; st > 0; st >>= 1) {
-        const int c = L + st;
-        if (__shfl_sync(0xffffffffu, ex, c) <= q) L = c;
-      }
-      const int exL = __shfl_sync(0xffffffffu, ex, L);
-      const uint32_t iL = __shfl_sync(0xffffffffu, i, L);
-      const int x0L = __shfl_sync(0xffffffffu, x0, L);
-      const int y0L = __shfl_sync(0xffffffffu, y0, L);
-      const int bwL = __shfl_sync(0xffffffffu, bw, L);
-      if (q < gtotal) {
-        const int li = q - exL;
-        const int row = li / bwL;
-        const uint32_t tid_ = (uint32_t)((y0L + row) * TW + x0L + (li - row * bwL));
-        const int64_t pos = run + q;
-        if (pos < capacity) {
-          tkey[pos] = tid_;
-          tval[pos] = iL;
-        }
-        for (int pp = 0; pp < passes; ++pp) atomicAdd(&s_hist[pp * kRadix + ((tid_ >> (8 * pp)) & 255u)], 1u);
-      }
-    }
-    run += gtotal;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
   }
-  __syncthreads();
-  for (int b = tid; b < passes * kRadix; b += kEmitBlock)
-    if (s_hist[b]) atomicAdd(&hist[b], s_hist[b]);
+  const int ex = inc - t;
+  const int wtotal = __shfl_sync(0xffffffffu, inc, 31);  // instances of the warp
+  for (int p0 = 0; p0 < wtotal; p0 += 32) {
+    const int q = p0 + lane;
+    int L = 0;
+#pragma unroll
+    for (int st = 16; st > 0; st >>= 1) {
+      const int c = L + st;
+      if (__shfl_sync(0xffffffffu, ex, c) <= q) L = c;
+    }
+    const int exL = __shfl_sync(0xffffffffu, ex, L);
+    const uint32_t iL = __shfl_sync(0xffffffffu, i, L);
+    const int x0L = __shfl_sync(0xffffffffu, x0, L);
+    const int y0L = __shfl_sync(0xffffffffu, y0, L);
+    const int bwL = __shfl_sync(0xffffffffu, bw, L);
+    if (q < wtotal) {
+      const int li = q - exL;
+      const int row = li / bwL;
+      tkey[base + q] = (uint32_t)((y0L + row) * TW + x0L + (li - row * bwL));
+      tval[base + q] = iL;
+    }
+  }
 }
 
 // Digit histograms of `passes` passes (digit p = bits [8p, 8p + 8)).
@@ -535,14 +448,13 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, const
 int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint32_t* v1, int64_t n,
                 const int64_t* n_dev, int passes, uint32_t* last_k, uint64_t* last_k64, uint32_t* last_v,
                 const float4* xyzo, int64_t n_records, const int32_t* tiles_in, int32_t* tiles_out, int64_t stall,
-                bool hist_ready, cudaStream_t s) {
-  if (!hist_ready && cudaMemsetAsync(w.hist, 0, kMaxPasses * kRadix * sizeof(uint32_t), s) != cudaSuccess)
-    return -1;
+                cudaStream_t s) {
+  if (cudaMemsetAsync(w.hist, 0, kMaxPasses * kRadix * sizeof(uint32_t), s) != cudaSuccess) return -1;
   const int64_t nt = sort_tiles(n);
   if (cudaMemsetAsync(w.counters, 0, (64 + (size_t)passes * nt * kRadix) * sizeof(uint32_t), s) != cudaSuccess)
     return -1;
   const unsigned hgrid = (unsigned)std::min<int64_t>(grid_for(n, 256), 148 * 4);
-  if (!hist_ready) digit_hist_kernel<<<hgrid, 256, 0, s>>>(k0, n, n_dev, n, passes, w.hist);
+  digit_hist_kernel<<<hgrid, 256, 0, s>>>(k0, n, n_dev, n, passes, w.hist);
   digit_offsets_kernel<<<passes, kRadix, 0, s>>>(w.hist);
   uint32_t* kb[2] = {k0, k1};
   uint32_t* vb[2] = {v0, v1};
@@ -570,7 +482,7 @@ int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint3
     onesweep_kernel<<<(unsigned)nt, kSortBlock, 0, s>>>(a);
   }
   if (cudaGetLastError() != cudaSuccess) return -1;
-  return (hist_ready ? 1 : 2) + passes;
+  return 2 + passes;
 }
 
 }  // namespace
@@ -586,7 +498,7 @@ BinSortPlan binsort_plan(int64_t n, int64_t capacity, int64_t tiles) {
   p.passes = (tb + 7) / 8;  // tile-digit passes over the instances
   p.bytes = align256((size_t)(scan_blocks(n) + 1) * sizeof(int64_t)) + 256 + 256 +
             align256(kMaxPasses * kRadix * sizeof(uint32_t)) + align256(lookback_words(p) * sizeof(uint32_t)) +
-            4 * align256((size_t)n * sizeof(uint32_t)) + align256((size_t)n * sizeof(int32_t)) +
+            4 * align256((size_t)n * sizeof(uint32_t)) + 2 * align256((size_t)n * sizeof(int32_t)) +
             4 * align256((size_t)capacity * sizeof(uint32_t));
   return p;
 }
@@ -605,7 +517,6 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
                                const BinSortPlan& plan, int64_t stall_tile, cudaStream_t s) {
   SortWs w = carve(ws, plan);
   cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(w.total, 0, sizeof(int64_t), s);
   if (e != cudaSuccess) return e;
   const int64_t nb = scan_blocks(n);
   int launched = 0;
@@ -620,9 +531,17 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
     // 4 passes: dkey[0] -> [1] -> [0] -> [1] -> [0]
     // the last pass also writes tiles_touched in depth order (dtiles)
     const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, nullptr, kDepthPasses, w.dkey[0],
-                              nullptr, w.dval[0], rec.xyzo, n, rec.tiles, w.dtiles, stall_tile, false, s);
+                              nullptr, w.dval[0], rec.xyzo, n, rec.tiles, w.dtiles, stall_tile, s);
     if (k < 0) return cudaErrorLaunchFailure;
     launched += 1 + k;
+    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials);
+    launched += 1;
+  }
+  scan_partials_kernel<<<1, 1024, 0, s>>>(w.partials, nb, w.total);
+  launched += 1;
+  if (nb > 0) {
+    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials, w.doff);
+    launched += 1;
   }
   count_launches(launched);
   return cudaGetLastError();
@@ -637,18 +556,9 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
   cudaError_t e = cudaMemsetAsync(ranges, 0, (size_t)TT * 2 * sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   int launched = 0;
-  // the tile-digit histograms are counted while the instances are emitted
-  e = cudaMemsetAsync(w.hist, 0, kMaxPasses * kRadix * sizeof(uint32_t), s);
-  if (e != cudaSuccess) return e;
   if (n > 0) {
-    const int64_t nb = scan_blocks(n);
-    e = cudaMemsetAsync(w.partials, 0, (size_t)nb * sizeof(int64_t), s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(w.counters + kScanCounter, 0, sizeof(uint32_t), s);
-    if (e != cudaSuccess) return e;
-    scan_emit_kernel<<<(unsigned)nb, kEmitBlock, 0, s>>>(
-        w.dval[0], w.dtiles, rec.rect, n, cam.TW, cap, plan.passes,
-        reinterpret_cast<unsigned long long*>(w.partials), w.counters + kScanCounter, w.total, w.status, w.hist,
-        w.tkey[0], w.tval[0]);
+    emit_kernel<<<grid_for(n, 256), 256, 0, s>>>(w.dval[0], w.doff, w.dtiles, rec.rect, n, cam.TW, w.total, cap,
+                                                 w.status, w.tkey[0], w.tval[0]);
     ++launched;
   }
   if (cap > 0) {
@@ -658,7 +568,7 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
       ++launched;
     } else {
       const int k = sort_passes(w, w.tkey[0], w.tval[0], w.tkey[1], w.tval[1], cap, w.total, plan.passes,
-                                nullptr, keys, vals, rec.xyzo, n, nullptr, nullptr, stall_tile, true, s);
+                                nullptr, keys, vals, rec.xyzo, n, nullptr, nullptr, stall_tile, s);
       if (k < 0) return cudaErrorLaunchFailure;
       launched += k;
     }

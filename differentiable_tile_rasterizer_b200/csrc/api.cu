@@ -223,6 +223,17 @@ GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const 
                                        static_cast<cudaStream_t>(stream)));
 }
 
+GS_API int gs_accumulate_grad2d_norm(const float* grad2d, const int32_t* tiles_touched, const int32_t* active_idx,
+                                     const int32_t* n_active, int64_t n_records, float* norm_sum,
+                                     int32_t* view_count, void* stream) {
+  if (n_records < 0 || n_records >= (int64_t(1) << 31) ||
+      (n_records > 0 && (!grad2d || !tiles_touched || !norm_sum || !view_count)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_grad2d_norm(reinterpret_cast<const float4*>(grad2d), tiles_touched, active_idx,
+                                        n_active, n_records, norm_sum, view_count,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const float* quats,
                              const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                              const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,

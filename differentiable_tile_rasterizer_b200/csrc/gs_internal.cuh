@@ -86,6 +86,12 @@ struct MultiViewArgs {
 };
 cudaError_t launch_preprocess_multiview(const Params& p, const MultiViewArgs& mv, cudaStream_t s);
 
+// stats.cu: norm_sum[g] += |(dpx, dpy)|, view_count[g] += 1 for every
+// visible record of the view (Gaussian g = active_idx[i] or i).
+cudaError_t launch_grad2d_norm(const float4* grad2d, const int32_t* tiles, const int32_t* active_idx,
+                               const int32_t* n_active, int64_t n_records, float* norm_sum, int32_t* view_count,
+                               cudaStream_t s);
+
 // binsort.cu
 struct BinSortPlan {
   int64_t n, capacity, tiles;

@@ -24,7 +24,7 @@ GS_ERR_DEVICE_TIMEOUT = 4
 GS_ERR_UNSUPPORTED = 5
 
 EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_preprocess_multiview",
-            "gs_bin_sort", "gs_bin_sort_async",
+            "gs_bin_sort", "gs_bin_sort_async", "gs_accumulate_grad2d_norm",
             "gs_rasterize_fwd", "gs_rasterize_fwd_importance", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
             "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
@@ -78,6 +78,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_cull.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P, PSZ, P]
         L.gs_preprocess.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, PCAM, PPROJ, P]
         L.gs_preprocess_multiview.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, ctypes.c_int, P, P]
+        L.gs_accumulate_grad2d_norm.argtypes = [P, P, P, P, I64, P, P, P]
         L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
         L.gs_bin_sort_async.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, P, P, PSZ, P]
         L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P]
@@ -93,7 +94,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_debug_kernel_launches.argtypes = []
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
         L.gs_debug_set_stalled_sort_tile.restype = None
-        for name in ["gs_cull", "gs_preprocess", "gs_preprocess_multiview", "gs_bin_sort", "gs_bin_sort_async", "gs_rasterize_fwd",
+        for name in ["gs_cull", "gs_preprocess", "gs_preprocess_multiview", "gs_bin_sort", "gs_accumulate_grad2d_norm", "gs_bin_sort_async", "gs_rasterize_fwd",
                      "gs_rasterize_fwd_importance",
                      "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
             getattr(L, name).restype = ctypes.c_int
@@ -186,6 +187,13 @@ def gs_preprocess_multiview(means, log_scales, quats, opacity_logits, sh, sh_deg
     _check("gs_preprocess_multiview", load().gs_preprocess_multiview(
         _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
         ctypes.cast(cam_arr, P), V, ctypes.cast(out_arr, P), _stream(stream)))
+
+
+def gs_accumulate_grad2d_norm(grad2d, tiles_touched, active_idx, n_active, n_records, norm_sum, view_count,
+                              stream=None):
+    _check("gs_accumulate_grad2d_norm", load().gs_accumulate_grad2d_norm(
+        _p(grad2d), _p(tiles_touched), _p(active_idx), _p(n_active), int(n_records), _p(norm_sum),
+        _p(view_count), _stream(stream)))
 
 
 def gs_bin_sort_workspace(n, cam: GsCamera, capacity) -> int:

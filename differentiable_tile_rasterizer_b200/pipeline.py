@@ -208,6 +208,13 @@ class Rasterizer:
                                            self.image, self.final_T, self.n_contrib, self.last, importance)
         return self.image
 
+    def accumulate_grad_stats(self, norm_sum: torch.Tensor, view_count: torch.Tensor):
+        """After backward(): adds this view's |dL/d(mean2D)| of every visible
+        Gaussian to norm_sum (float32 [N]) and 1 to view_count (int32 [N])."""
+        act = self.active_idx if self.culled else None
+        na = self.n_active if self.culled else None
+        gs.gs_accumulate_grad2d_norm(self.grad2d, self.rec["tiles"], act, na, self.N, norm_sum, view_count)
+
     def check(self) -> list:
         """Instance counts of the views binned in deferred mode since the last
         check (one host read). Raises GsError if one of them failed; after a

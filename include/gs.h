@@ -155,6 +155,25 @@ GS_API int gs_preprocess(const float* means, const float* log_scales, const floa
                          const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
                          const gs_projected* out, void* stream);
 
+/* Densification statistic of a view, from the raster backward's 2-D
+ * gradients: for every record i that the view sees (tiles_touched > 0,
+ * i < n_active), norm_sum[g] += sqrt(dpx^2 + dpy^2) and view_count[g] += 1,
+ * with g = active_idx[i] (or i). Called once per view after
+ * gs_rasterize_bwd(_2d); the mean norm_sum / view_count is the usual
+ * densification criterion of Gaussian-splat training (positional gradient
+ * in screen space). The pages print no formula for it; it pairs with the
+ * importance weights (gs_rasterize_fwd_importance) as the two per-Gaussian
+ * statistics a training schedule reads.
+ *   grad2d        [device] [n_records][12] from gs_rasterize_bwd(_2d)
+ *   tiles_touched [device] [n_records] i32 of the view's records
+ *   active_idx, n_active [device] from gs_cull, or NULL
+ *   norm_sum      [device] [N] f32 in/out (added to)
+ *   view_count    [device] [N] i32 in/out (added to)
+ * fp32: the norm is sqrt(fma(dpx, dpx, dpy * dpy)). Asynchronous. */
+GS_API int gs_accumulate_grad2d_norm(const float* grad2d, const int32_t* tiles_touched,
+                                     const int32_t* active_idx, const int32_t* n_active, int64_t n_records,
+                                     float* norm_sum, int32_t* view_count, void* stream);
+
 /* Views per gs_preprocess_multiview call. */
 #define GS_MAX_VIEWS 16
 

@@ -222,6 +222,22 @@ def importance(rec, bins, cam, n_gaussians, out=None):
     return out
 
 
+def grad2d_norm(grad2d, tiles, active_idx, n_gaussians, norm_sum=None, view_count=None):
+    """Densification statistic of one view: for every visible record i
+    (tiles[i] > 0), adds |(dpx, dpy)| = hypot of grad2d[i][0:2] to
+    norm_sum[g] and 1 to view_count[g], g = active_idx[i] (or i). float64."""
+    if norm_sum is None:
+        norm_sum = np.zeros(n_gaussians, np.float64)
+    if view_count is None:
+        view_count = np.zeros(n_gaussians, np.int64)
+    g2 = np.asarray(grad2d, np.float64).reshape(-1, 12)
+    vis = np.flatnonzero(np.asarray(tiles) > 0)
+    gid = vis if active_idx is None else np.asarray(active_idx)[vis]
+    norm_sum[gid] += np.sqrt(g2[vis, 0] ** 2 + g2[vis, 1] ** 2)
+    view_count[gid] += 1
+    return norm_sum, view_count
+
+
 def raster_fwd_bruteforce(rec, cam, bg):
     W, H = cam.width, cam.height
     image = np.zeros((3, H, W), np.float32)

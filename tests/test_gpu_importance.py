@@ -105,3 +105,29 @@ def test_importance_feeds_the_cull():
     assert int(R.n_active.item()) == na
     assert_bits(R.active_idx[:na].cpu().numpy(), cl["active_idx"], "active_idx")
     assert 0 < na < sc.N
+
+
+def test_grad2d_norm_statistic_matches_oracle():
+    # on the GPU's own 2-D gradients (the same input for both), over 3 views
+    # with a cull; fp32 sqrt(fma(x, x, y*y)) against float64 hypot: within
+    # 2 ulp per view plus the fp32 sums over views
+    sc = S.random_scene(2500, 96, 80, sh_degree=1, seed=76, n_poses=3, with_importance=True, lod_dist=3.2,
+                        importance_q=0.2)
+    cam = sc.cameras[0]
+    R = Rasterizer(sc.N, sc.sh_degree, cam.width, cam.height, capacity=64 * sc.N)
+    params = GaussianParams.from_scene(sc)
+    nsum = torch.zeros(sc.N, dtype=torch.float32, device="cuda")
+    cnt = torch.zeros(sc.N, dtype=torch.int32, device="cuda")
+    ref_s, ref_c = np.zeros(sc.N), np.zeros(sc.N, np.int64)
+    for p in range(3):
+        R.forward(params, sc.cameras[p], sc.bg, sc.lod_dist, sc.importance_q)
+        R.backward(torch.from_numpy(sc.grad_image(p)).cuda())
+        R.accumulate_grad_stats(nsum, cnt)
+        torch.cuda.synchronize()
+        na = int(R.n_active.item())
+        oracle.grad2d_norm(R.grad2d.cpu().numpy()[:na], R.rec["tiles"].cpu().numpy()[:na],
+                           R.active_idx.cpu().numpy()[:na], sc.N, ref_s, ref_c)
+    got_s, got_c = nsum.cpu().numpy().astype(np.float64), cnt.cpu().numpy()
+    np.testing.assert_array_equal(got_c, ref_c)
+    assert ref_c.max() == 3 and (ref_c == 0).any()
+    np.testing.assert_allclose(got_s, ref_s, rtol=4 * 2.0 ** -23, atol=0)

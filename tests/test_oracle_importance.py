@@ -128,3 +128,26 @@ def test_views_add_up():
         parts.append(oracle.importance(r["rec"], r["bins"], sc.cameras[p], sc.N))
         oracle.importance(r["rec"], r["bins"], sc.cameras[p], sc.N, out=total)
     np.testing.assert_allclose(total, parts[0] + parts[1] + parts[2], rtol=1e-12, atol=0)
+
+
+def test_grad2d_norm_statistic_is_the_plain_definition():
+    # the densification statistic: per visible record, hypot(dpx, dpy) added
+    # to its Gaussian, one view counted; checked element by element with
+    # math.hypot over a permuted active list with invisible records
+    import math
+    rng = np.random.default_rng(65)
+    n, N = 50, 80
+    g2 = rng.normal(0, 1, (n, 12)).astype(np.float32)
+    tiles = rng.integers(-1, 3, n).astype(np.int32)
+    act = rng.permutation(N)[:n].astype(np.int32)
+    s, c = oracle.grad2d_norm(g2, tiles, act, N)
+    s2, c2 = oracle.grad2d_norm(g2, tiles, act, N, s.copy(), c.copy())
+    ref_s, ref_c = np.zeros(N), np.zeros(N, np.int64)
+    for i in range(n):
+        if tiles[i] > 0:
+            ref_s[act[i]] += math.hypot(float(g2[i, 0]), float(g2[i, 1]))
+            ref_c[act[i]] += 1
+    np.testing.assert_allclose(s, ref_s, rtol=1e-15, atol=0)
+    np.testing.assert_array_equal(c, ref_c)
+    np.testing.assert_allclose(s2, 2 * ref_s, rtol=1e-15, atol=0)
+    np.testing.assert_array_equal(c2, 2 * ref_c)

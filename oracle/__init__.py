@@ -72,6 +72,13 @@ def _declare(L):
     L.or_raster_fwd.restype = ctypes.c_int
     L.or_raster_fwd_bruteforce.argtypes = [P, P, P, P, P, I64, I32, I32, P, P, P, P, P]
     L.or_importance.argtypes = [P, P, P, P, P, I32, I32, P, P]
+    for f in ("or_log2_spec", "or_log1p_spec", "or_expm1_spec"):
+        getattr(L, f).argtypes = [ctypes.c_float]
+        getattr(L, f).restype = ctypes.c_float
+    L.or_quant_encode.argtypes = [P, I64, I64, I32, P, P]
+    L.or_quant_decode.argtypes = [P, P, I64, I64, I32, P]
+    D = ctypes.c_double
+    L.or_adam_sh_quant.argtypes = [P, I64, I64, P, P, P, P, P, P, D, D, D, D, D, I64]
     L.or_importance.restype = ctypes.c_int
     L.or_loss_frozen_f64.argtypes = [P, P, P, P, P, I32, I64, P, I64, P, I32, I32,
                                      P, P, P, P, P, P, P, P, P]
@@ -236,6 +243,55 @@ def grad2d_norm(grad2d, tiles, active_idx, n_gaussians, norm_sum=None, view_coun
     norm_sum[gid] += np.sqrt(g2[vis, 0] ** 2 + g2[vis, 1] ** 2)
     view_count[gid] += 1
     return norm_sum, view_count
+
+
+# ---- quantised SH Adam (Spirula Studio page: 16-bit SH value codes, 8-bit
+# log codes of the Adam moments, per-256-unit block bounds)
+def log2_spec(y):
+    return lib().or_log2_spec(float(y))
+
+
+def log1p_spec(z):
+    return lib().or_log1p_spec(float(z))
+
+
+def expm1_spec(y):
+    return lib().or_expm1_spec(float(y))
+
+
+def quant_encode(x, bits):
+    """Block codes of float32 planes x [U, N]: (codes uint32 [U, Npad], bounds
+    float32 [U, nblk, 2]); blocks of 256 consecutive units of a plane."""
+    x = _c(x, np.float32)
+    U, N = x.shape
+    nblk = (N + 255) // 256
+    codes = np.zeros((U, nblk * 256), np.uint32)
+    bounds = np.zeros((U, nblk, 2), np.float32)
+    lib().or_quant_encode(_p(x), U, N, int(bits), _p(codes), _p(bounds))
+    return codes, bounds
+
+
+def quant_decode(codes, bounds, N, bits):
+    U = codes.shape[0]
+    x = np.zeros((U, N), np.float32)
+    lib().or_quant_decode(_p(_c(codes, np.uint32)), _p(_c(bounds, np.float32)), U, N, int(bits), _p(x))
+    return x
+
+
+def adam_sh_quant(grad, state, lr, beta1, beta2, eps, scale, step):
+    """One Adam step in place on state = {"pc","pb","mc","mb","vc","vb"}
+    (value codes 16-bit, moment log codes 8-bit, as quant_encode lays them
+    out); grad float32 [U, N]."""
+    g = _c(grad, np.float32)
+    U, N = g.shape
+    for k in ("pc", "mc", "vc"):
+        assert state[k].dtype == np.uint32 and state[k].flags.c_contiguous
+    for k in ("pb", "mb", "vb"):
+        assert state[k].dtype == np.float32 and state[k].flags.c_contiguous
+    lib().or_adam_sh_quant(_p(g), U, N, _p(state["pc"]), _p(state["pb"]), _p(state["mc"]), _p(state["mb"]),
+                           _p(state["vc"]), _p(state["vb"]), float(lr), float(beta1), float(beta2), float(eps),
+                           float(scale), int(step))
+    return state
 
 
 def raster_fwd_bruteforce(rec, cam, bg):

@@ -1242,3 +1242,170 @@ OR_API int or_project_f64(const double* means, const double* log_scales, const d
   }
   return 0;
 }
+
+// ===================================================== quantised SH Adam
+// The fused optimizer step over block-quantised SH coefficients and Adam
+// moments (Spirula Studio page, sections "先算一笔账", "一个开关" and
+// "为什么 8-bit 量化 Adam 状态居然不掉精度"): the view-dependent SH units are
+// stored as 16-bit linear block codes, each moment as an 8-bit linear block
+// code of its logarithm, every 256 consecutive units of a plane sharing one
+// (min, max) pair; gradients stay fp32. Readings fixed here (the page prints
+// no formula beyond the log transform and the decode):
+//   block      256 consecutive Gaussians of one unit plane (the transposed
+//              layout); codes have row stride Npad = N rounded up to 256,
+//              bounds are [U][N/256 rounded up][2] = (lo, hi)
+//   code       q = rint(((x - lo) / (hi - lo)) * Q) clamped to [0, Q],
+//              Q = 2^bits - 1; decode lo + (hi - lo) * (q / Q); a block with
+//              hi == lo codes everything 0; fp32, no fused multiply-add
+//   moments    first moment m: y = sign(m) log1p(|m| / e); second moment v:
+//              y = log1p(sqrt(v) / e); e is the code scale (an input);
+//              decode through expm1
+//   log1p      ln 2 * log2(1 + z), log2 by the atanh series below; expm1 as
+//              exp2(y log2 e) - 1 with the software exp2 of the raster
+//   Adam       m' = b1 m + (1 - b1) g, v' = b2 v + (1 - b2) g^2,
+//              p' = p - lr (m' c1) / (sqrt(v' c2) + eps), c1, c2 the bias
+//              corrections of the step (inputs, like b1, 1 - b1, b2, 1 - b2)
+//   bounds     of the new fp32 values of each block, every step.
+
+namespace {
+
+struct QuantConst {
+  float l2c[6];  // RN(2 / ((2k + 1) ln 2)), k = 0..5
+  float ln2, sqrt2;
+  QuantConst() {
+    const double ln2d = std::log(2.0);
+    for (int k = 0; k < 6; ++k) l2c[k] = (float)(2.0 / ((2.0 * k + 1.0) * ln2d));
+    ln2 = (float)ln2d;
+    sqrt2 = (float)std::sqrt(2.0);
+  }
+};
+const QuantConst QC;
+
+}  // namespace
+
+// log2 of y >= 1 (finite): y = m 2^e with m in (sqrt(1/2), sqrt(2)] (exact),
+// s = (m - 1) / (m + 1), log2(m) = 2 atanh(s) / ln 2 as a Horner polynomial
+// in s^2 with the coefficients above.
+float log2_spec(float y) {
+  int e;
+  float m = std::frexp(y, &e);  // y = m 2^e, m in [1/2, 1)
+  m = m * 2.0f;
+  e -= 1;                       // m in [1, 2)
+  if (m > QC.sqrt2) {
+    m = m * 0.5f;
+    e += 1;
+  }
+  const float s = (m - 1.0f) / (m + 1.0f);
+  const float s2 = s * s;
+  float p = QC.l2c[5];
+  for (int k = 4; k >= 0; --k) p = std::fmaf(p, s2, QC.l2c[k]);
+  return (float)e + s * p;
+}
+inline float log1p_spec(float z) { return QC.ln2 * log2_spec(1.0f + z); }
+inline float expm1_spec(float y) { return exp2_spec(y * KC.l2e) - 1.0f; }
+
+inline uint32_t q_encode(float x, float lo, float d, float Q) {
+  if (!(d > 0.0f)) return 0u;
+  const float t = std::rint(((x - lo) / d) * Q);
+  return t < 0.0f ? 0u : (t > Q ? (uint32_t)Q : (uint32_t)t);
+}
+inline float q_decode(uint32_t q, float lo, float d, float Q) { return lo + d * ((float)q / Q); }
+
+inline float m_to_log(float m, float e) { return m >= 0.0f ? log1p_spec(m / e) : -log1p_spec(-m / e); }
+inline float m_from_log(float y, float e) { return y >= 0.0f ? e * expm1_spec(y) : -(e * expm1_spec(-y)); }
+inline float v_to_log(float v, float e) { return log1p_spec(std::sqrt(v) / e); }
+inline float v_from_log(float y, float e) {
+  const float s = e * expm1_spec(y);
+  return s * s;
+}
+
+OR_API float or_log2_spec(float y) { return log2_spec(y); }
+OR_API float or_log1p_spec(float z) { return log1p_spec(z); }
+OR_API float or_expm1_spec(float y) { return expm1_spec(y); }
+
+// Block codes of fp32 planes x [U][N] (row stride N): codes [U][Npad] (16 or
+// 8 bit, stored as uint32 here), bounds [U][nblk][2].
+OR_API int or_quant_encode(const float* x, int64_t U, int64_t N, int bits, uint32_t* codes, float* bounds) {
+  const int64_t nblk = (N + 255) / 256, Npad = nblk * 256;
+  const float Q = (float)((1u << bits) - 1u);
+  for (int64_t u = 0; u < U; ++u)
+    for (int64_t b = 0; b < nblk; ++b) {
+      const int64_t g0 = b * 256, g1 = std::min(N, g0 + 256);
+      float lo = x[u * N + g0], hi = lo;
+      for (int64_t g = g0; g < g1; ++g) {
+        lo = std::min(lo, x[u * N + g]);
+        hi = std::max(hi, x[u * N + g]);
+      }
+      const float d = hi - lo;
+      for (int64_t g = g0; g < g0 + 256; ++g)
+        codes[u * Npad + g] = g < g1 ? q_encode(x[u * N + g], lo, d, Q) : 0u;
+      bounds[2 * (u * nblk + b)] = lo;
+      bounds[2 * (u * nblk + b) + 1] = hi;
+    }
+  return 0;
+}
+
+// Decoded fp32 planes of block codes (inverse layout of or_quant_encode).
+OR_API int or_quant_decode(const uint32_t* codes, const float* bounds, int64_t U, int64_t N, int bits, float* x) {
+  const int64_t nblk = (N + 255) / 256, Npad = nblk * 256;
+  const float Q = (float)((1u << bits) - 1u);
+  for (int64_t u = 0; u < U; ++u)
+    for (int64_t g = 0; g < N; ++g) {
+      const int64_t b = g / 256;
+      const float lo = bounds[2 * (u * nblk + b)], hi = bounds[2 * (u * nblk + b) + 1];
+      x[u * N + g] = q_decode(codes[u * Npad + g], lo, hi - lo, Q);
+    }
+  return 0;
+}
+
+// One Adam step (number `step`, from 1) over U planes of N units, in place:
+// 16-bit value codes, 8-bit log codes of m and v, fp32 gradients grad [U][N]
+// (row stride N). The fp32 constants of the step are the roundings of
+// lr, beta1, 1 - beta1, beta2, 1 - beta2, 1 / (1 - beta1^step),
+// 1 / (1 - beta2^step), eps and the code scale, each computed in double.
+OR_API int or_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint32_t* pc, float* pb, uint32_t* mc,
+                            float* mb, uint32_t* vc, float* vb, double lr_d, double beta1, double beta2,
+                            double eps_d, double scale_d, int64_t step) {
+  const float lr = (float)lr_d, b1 = (float)beta1, ob1 = (float)(1.0 - beta1), b2 = (float)beta2,
+              ob2 = (float)(1.0 - beta2), c1 = (float)(1.0 / (1.0 - std::pow(beta1, (double)step))),
+              c2 = (float)(1.0 / (1.0 - std::pow(beta2, (double)step))), eps = (float)eps_d,
+              ec = (float)scale_d;
+  const int64_t nblk = (N + 255) / 256, Npad = nblk * 256;
+  const float Q16 = 65535.0f, Q8 = 255.0f;
+  std::vector<float> np(256), ny(256), vy(256);
+  for (int64_t u = 0; u < U; ++u)
+    for (int64_t b = 0; b < nblk; ++b) {
+      const int64_t g0 = b * 256, g1 = std::min(N, g0 + 256), n = g1 - g0;
+      float* B[3] = {pb + 2 * (u * nblk + b), mb + 2 * (u * nblk + b), vb + 2 * (u * nblk + b)};
+      for (int64_t k = 0; k < n; ++k) {
+        const int64_t c = u * Npad + g0 + k;
+        const float ph = q_decode(pc[c], B[0][0], B[0][1] - B[0][0], Q16);
+        const float mh = m_from_log(q_decode(mc[c], B[1][0], B[1][1] - B[1][0], Q8), ec);
+        const float vh = v_from_log(q_decode(vc[c], B[2][0], B[2][1] - B[2][0], Q8), ec);
+        const float g = grad[u * N + g0 + k];
+        const float m1 = b1 * mh + ob1 * g;
+        const float v1 = b2 * vh + ob2 * (g * g);
+        const float a = m1 * c1;
+        const float den = std::sqrt(v1 * c2) + eps;
+        np[k] = ph - lr * (a / den);
+        ny[k] = m_to_log(m1, ec);
+        vy[k] = v_to_log(v1, ec);
+      }
+      const std::vector<float>* vals[3] = {&np, &ny, &vy};
+      uint32_t* codes[3] = {pc, mc, vc};
+      const float Qs[3] = {Q16, Q8, Q8};
+      for (int t = 0; t < 3; ++t) {
+        const std::vector<float>& y = *vals[t];
+        float lo = y[0], hi = y[0];
+        for (int64_t k = 1; k < n; ++k) {
+          lo = std::min(lo, y[k]);
+          hi = std::max(hi, y[k]);
+        }
+        const float d = hi - lo;
+        for (int64_t k = 0; k < 256; ++k) codes[t][u * Npad + g0 + k] = k < n ? q_encode(y[k], lo, d, Qs[t]) : 0u;
+        B[t][0] = lo;
+        B[t][1] = hi;
+      }
+    }
+  return 0;
+}

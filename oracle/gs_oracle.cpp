@@ -1283,10 +1283,11 @@ const QuantConst QC;
 
 }  // namespace
 
-// log2 of y >= 1 (finite): y = m 2^e with m in (sqrt(1/2), sqrt(2)] (exact),
+// log2 of y >= 1: y = m 2^e with m in (sqrt(1/2), sqrt(2)] (exact),
 // s = (m - 1) / (m + 1), log2(m) = 2 atanh(s) / ln 2 as a Horner polynomial
-// in s^2 with the coefficients above.
+// in s^2 with the coefficients above; log2(+inf) = +inf.
 float log2_spec(float y) {
+  if (!(y <= std::numeric_limits<float>::max())) return y;  // +inf (and NaN) pass through
   int e;
   float m = std::frexp(y, &e);  // y = m 2^e, m in [1/2, 1)
   m = m * 2.0f;

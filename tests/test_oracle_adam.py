@@ -28,6 +28,7 @@ def test_log2_spec_against_float64():
     worst = max(_ulp_err(oracle.log2_spec(y), np.log2(np.float64(F32(y)))) for y in ys)
     assert worst <= 3.0, worst
     assert oracle.log2_spec(1.0) == 0.0 and oracle.log2_spec(1024.0) == 10.0
+    assert oracle.log2_spec(float("inf")) == float("inf")
 
 
 def test_log1p_and_expm1_spec_against_float64():

@@ -306,6 +306,9 @@ def run_ours(args):
         line["importance_pass"] = importance_pass(R, params, cams, bg, per_kernel["raster_fwd"] / len(poses),
                                                   peak_alu, fwd_ms)
 
+    if not args.no_adam:
+        line["adam_sh_quant"] = adam_pass(R, params, peaks)
+
     if args.multiview and world == 1:
         line["multiview"] = multiview(args, peaks)
 
@@ -357,6 +360,34 @@ def importance_pass(R, params, cams, bg, ops_per_view, peak_alu, fwd_ms, reps=10
             "roofline": {"bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
                          "frac": achieved / peak_alu, "ops": "the forward's spec operations (21 E + 8 B)"},
             "views": len(cams), "reps": reps}
+
+
+def adam_pass(R, params, peaks, reps=20):
+    """The fused quantised-SH Adam step (gs_adam_sh_quant) on the bench model:
+    45 unit planes x 1M Gaussians, with the last backward's gradients."""
+    import torch
+    from differentiable_tile_rasterizer_b200.pipeline import QuantizedSHAdam
+    opt = QuantizedSHAdam(R.N, R.sh_degree, lr=1e-3)
+    opt.load(params.sh)
+    d_sh = R.grads["sh"]
+    for _ in range(3):
+        opt.step(d_sh)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        opt.step(d_sh)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    units = opt.U * opt.N
+    nbytes = units * (4 + 2 + 1 + 1) + opt.U * opt.nblk * 256 * (2 + 1 + 1) + 3 * opt.U * opt.nblk * 8 * 2
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"units": units, "ms_per_step": ms, "bytes_per_step": nbytes,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"],
+                         "bytes": "4 B gradient + 4 B codes read, 4 B codes written per unit, + block bounds"},
+            "state_bytes_per_unit": 4.0 + 3 * 8 * 2 / 256.0}
 
 
 def multiview(args, peaks):
@@ -466,6 +497,7 @@ def main():
     ap.add_argument("--ref-tile-stride", type=int, default=32,
                     help="reference arm: sample every n-th tile per step")
     ap.add_argument("--no-importance", action="store_true", help="skip timing the importance pass")
+    ap.add_argument("--no-adam", action="store_true", help="skip timing the quantised SH Adam step")
     ap.add_argument("--multiview", action="store_true",
                     help="also time the eight-view 4K workload with the one-pass multi-view preprocess")
     ap.add_argument("--cpu-tile-stride", type=int, default=1,

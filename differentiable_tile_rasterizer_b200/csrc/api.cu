@@ -234,6 +234,42 @@ GS_API int gs_accumulate_grad2d_norm(const float* grad2d, const int32_t* tiles_t
                                         static_cast<cudaStream_t>(stream)));
 }
 
+GS_API int gs_quant_encode(const float* x, int64_t U, int64_t N, int bits, void* codes, float* bounds,
+                           void* stream) {
+  if (U < 0 || N < 0 || (bits != 8 && bits != 16) || (U * N > 0 && (!x || !codes || !bounds)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_quant_encode(x, U, N, bits, codes, bounds, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_quant_decode(const void* codes, const float* bounds, int64_t U, int64_t N, int bits, float* x,
+                           void* stream) {
+  if (U < 0 || N < 0 || (bits != 8 && bits != 16) || (U * N > 0 && (!x || !codes || !bounds)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_quant_decode(codes, bounds, U, N, bits, x, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* value_codes, float* value_bounds,
+                            uint8_t* m_codes, float* m_bounds, uint8_t* v_codes, float* v_bounds,
+                            const gs_adam_config* cfg, void* stream) {
+  if (!cfg || U < 0 || N < 0 || cfg->step < 1 || !(cfg->code_scale > 0.0) ||
+      (U * N > 0 && (!grad || !value_codes || !value_bounds || !m_codes || !m_bounds || !v_codes || !v_bounds)))
+    return GS_ERR_INVALID_ARGUMENT;
+  // the fp32 constants of the step, each rounded from double
+  const double t = (double)cfg->step;
+  const float hp[10] = {(float)cfg->lr,
+                       (float)cfg->beta1,
+                       (float)(1.0 - cfg->beta1),
+                       (float)cfg->beta2,
+                       (float)(1.0 - cfg->beta2),
+                       (float)(1.0 / (1.0 - std::pow(cfg->beta1, t))),
+                       (float)(1.0 / (1.0 - std::pow(cfg->beta2, t))),
+                       (float)cfg->eps,
+                       (float)cfg->code_scale,
+                       (float)(1.0 / cfg->code_scale)};
+  return cuda_status(launch_adam_sh_quant(grad, U, N, value_codes, value_bounds, m_codes, m_bounds, v_codes,
+                                          v_bounds, hp, static_cast<cudaStream_t>(stream)));
+}
+
 GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const float* quats,
                              const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                              const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,

@@ -92,6 +92,16 @@ cudaError_t launch_grad2d_norm(const float4* grad2d, const int32_t* tiles, const
                                const int32_t* n_active, int64_t n_records, float* norm_sum, int32_t* view_count,
                                cudaStream_t s);
 
+// adam.cu: block codes (256 units per block, row stride quant_blocks(N) * 256)
+int64_t quant_blocks(int64_t N);
+cudaError_t launch_quant_encode(const float* x, int64_t U, int64_t N, int bits, void* codes, float* bounds,
+                                cudaStream_t s);
+cudaError_t launch_quant_decode(const void* codes, const float* bounds, int64_t U, int64_t N, int bits, float* x,
+                                cudaStream_t s);
+// hp = {lr, b1, 1 - b1, b2, 1 - b2, c1, c2, eps, code scale e, 1 / e}
+cudaError_t launch_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* pc, float* pb, uint8_t* mc,
+                                 float* mb, uint8_t* vc, float* vb, const float hp[10], cudaStream_t s);
+
 // binsort.cu
 struct BinSortPlan {
   int64_t n, capacity, tiles;

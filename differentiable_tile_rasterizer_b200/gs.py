@@ -24,7 +24,8 @@ GS_ERR_DEVICE_TIMEOUT = 4
 GS_ERR_UNSUPPORTED = 5
 
 EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_preprocess_multiview",
-            "gs_bin_sort", "gs_bin_sort_async", "gs_accumulate_grad2d_norm",
+            "gs_bin_sort", "gs_bin_sort_async", "gs_accumulate_grad2d_norm", "gs_quant_encode",
+            "gs_quant_decode", "gs_adam_sh_quant",
             "gs_rasterize_fwd", "gs_rasterize_fwd_importance", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
             "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
@@ -35,6 +36,11 @@ class GsError(RuntimeError):
     def __init__(self, fn: str, status: int, msg: str):
         super().__init__(f"{fn}: status {status} ({msg})")
         self.status = status
+
+
+class GsAdamConfig(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("code_scale", ctypes.c_double), ("step", ctypes.c_int64)]
 
 
 class GsCamera(ctypes.Structure):
@@ -79,6 +85,9 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_preprocess.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, PCAM, PPROJ, P]
         L.gs_preprocess_multiview.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, ctypes.c_int, P, P]
         L.gs_accumulate_grad2d_norm.argtypes = [P, P, P, P, I64, P, P, P]
+        L.gs_quant_encode.argtypes = [P, I64, I64, ctypes.c_int, P, P, P]
+        L.gs_quant_decode.argtypes = [P, P, I64, I64, ctypes.c_int, P, P]
+        L.gs_adam_sh_quant.argtypes = [P, I64, I64, P, P, P, P, P, P, ctypes.POINTER(GsAdamConfig), P]
         L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
         L.gs_bin_sort_async.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, P, P, PSZ, P]
         L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P]
@@ -94,7 +103,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_debug_kernel_launches.argtypes = []
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
         L.gs_debug_set_stalled_sort_tile.restype = None
-        for name in ["gs_cull", "gs_preprocess", "gs_preprocess_multiview", "gs_bin_sort", "gs_accumulate_grad2d_norm", "gs_bin_sort_async", "gs_rasterize_fwd",
+        for name in ["gs_cull", "gs_preprocess", "gs_preprocess_multiview", "gs_bin_sort", "gs_accumulate_grad2d_norm",
+                     "gs_quant_encode", "gs_quant_decode", "gs_adam_sh_quant", "gs_bin_sort_async", "gs_rasterize_fwd",
                      "gs_rasterize_fwd_importance",
                      "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
             getattr(L, name).restype = ctypes.c_int
@@ -187,6 +197,23 @@ def gs_preprocess_multiview(means, log_scales, quats, opacity_logits, sh, sh_deg
     _check("gs_preprocess_multiview", load().gs_preprocess_multiview(
         _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
         ctypes.cast(cam_arr, P), V, ctypes.cast(out_arr, P), _stream(stream)))
+
+
+def gs_quant_encode(x, U, N, bits, codes, bounds, stream=None):
+    _check("gs_quant_encode", load().gs_quant_encode(_p(x), int(U), int(N), int(bits), _p(codes), _p(bounds),
+                                                     _stream(stream)))
+
+
+def gs_quant_decode(codes, bounds, U, N, bits, x, stream=None):
+    _check("gs_quant_decode", load().gs_quant_decode(_p(codes), _p(bounds), int(U), int(N), int(bits), _p(x),
+                                                     _stream(stream)))
+
+
+def gs_adam_sh_quant(grad, U, N, pc, pb, mc, mb, vc, vb, lr, beta1, beta2, eps, code_scale, step, stream=None):
+    cfg = GsAdamConfig(float(lr), float(beta1), float(beta2), float(eps), float(code_scale), int(step))
+    _check("gs_adam_sh_quant", load().gs_adam_sh_quant(
+        _p(grad), int(U), int(N), _p(pc), _p(pb), _p(mc), _p(mb), _p(vc), _p(vb), ctypes.byref(cfg),
+        _stream(stream)))
 
 
 def gs_accumulate_grad2d_norm(grad2d, tiles_touched, active_idx, n_active, n_records, norm_sum, view_count,

@@ -347,3 +347,45 @@ class MultiViewRenderer:
 
     def check(self) -> list:
         return [R.check() for R in self.views]
+
+
+class QuantizedSHAdam:
+    """Adam over the view-dependent SH coefficients kept as 16-bit block codes,
+    with both moments as 8-bit block codes of their logarithms
+    (gs_adam_sh_quant). Planes 3 .. 3K - 1 of the SH parameters (the DC plane
+    stays in fp32); 256 consecutive Gaussians of a plane share a (lo, hi)."""
+
+    def __init__(self, N: int, sh_degree: int, lr=2.5e-3 / 20.0, beta1=0.9, beta2=0.999, eps=1e-15,
+                 code_scale=1e-15, device=None):
+        if sh_degree < 1:
+            raise ValueError("no view-dependent SH coefficients at degree 0")
+        d = torch.device(device or "cuda")
+        self.N, self.K = int(N), (sh_degree + 1) ** 2
+        self.U = 3 * (self.K - 1)
+        self.nblk = (self.N + 255) // 256
+        pad = self.nblk * 256
+        self.pc = torch.zeros((self.U, pad), dtype=torch.int16, device=d)  # uint16 codes
+        self.mc = torch.zeros((self.U, pad), dtype=torch.uint8, device=d)
+        self.vc = torch.zeros((self.U, pad), dtype=torch.uint8, device=d)
+        self.pb = torch.zeros((self.U, self.nblk, 2), dtype=torch.float32, device=d)
+        self.mb = torch.zeros_like(self.pb)
+        self.vb = torch.zeros_like(self.pb)
+        self.lr, self.beta1, self.beta2, self.eps, self.code_scale = lr, beta1, beta2, eps, code_scale
+        self.step_count = 0
+
+    def load(self, sh: torch.Tensor):
+        """Codes of the SH planes 3.. of sh [3K][N] (moments reset to zero)."""
+        gs.gs_quant_encode(sh[3:], self.U, self.N, 16, self.pc, self.pb)
+        for t in (self.mc, self.vc, self.mb, self.vb):
+            t.zero_()
+        self.step_count = 0
+
+    def step(self, d_sh: torch.Tensor):
+        """One Adam step from the gradients d_sh [3K][N] (planes 3.. are used)."""
+        self.step_count += 1
+        gs.gs_adam_sh_quant(d_sh[3:], self.U, self.N, self.pc, self.pb, self.mc, self.mb, self.vc, self.vb,
+                            self.lr, self.beta1, self.beta2, self.eps, self.code_scale, self.step_count)
+
+    def store(self, sh: torch.Tensor):
+        """Decoded values into the SH planes 3.. of sh [3K][N] (for rendering)."""
+        gs.gs_quant_decode(self.pc, self.pb, self.U, self.N, 16, sh[3:])

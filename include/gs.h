@@ -174,6 +174,58 @@ GS_API int gs_accumulate_grad2d_norm(const float* grad2d, const int32_t* tiles_t
                                      const int32_t* active_idx, const int32_t* n_active, int64_t n_records,
                                      float* norm_sum, int32_t* view_count, void* stream);
 
+/* ---- Quantised SH training state (Spirula Studio page, sections
+ * "先算一笔账", "一个开关" and the section on 8-bit Adam states): view-dependent
+ * SH coefficients stored as 16-bit linear block codes, both Adam moments as
+ * 8-bit linear block codes of their logarithms, gradients in fp32. A block is
+ * 256 consecutive Gaussians of one unit plane (the transposed layout the page
+ * describes); planes are [U][N] with U = 3 (K - 1) at SH degree with K
+ * coefficients (the DC plane is not quantised), codes at row stride
+ * Npad = 256 * ceil(N / 256), bounds [U][ceil(N / 256)][2] = (lo, hi) fp32.
+ * Code, per block: step = (hi - lo) / Q, inv = Q / (hi - lo) (both 0 when
+ * hi == lo: every code 0), Q = 2^bits - 1; q = rint((x - lo) * inv) clamped
+ * to [0, Q]; decode lo + step * q (one multiplication per unit, as the page
+ * says); fp32 without fused multiply-add. The page prints only the moment transform
+ * log1p(sqrt(g2) / eps) and the decode; the rest is fixed as written here. */
+
+/* Block codes of fp32 planes x [U][N] (row stride N); bits 8 or 16
+ * (codes uint8 or uint16 [U][Npad]). Padding codes are 0. Asynchronous. */
+GS_API int gs_quant_encode(const float* x, int64_t U, int64_t N, int bits, void* codes, float* bounds,
+                           void* stream);
+
+/* Decoded fp32 planes x [U][N] of block codes. Asynchronous. */
+GS_API int gs_quant_decode(const void* codes, const float* bounds, int64_t U, int64_t N, int bits, float* x,
+                           void* stream);
+
+/* Hyperparameters of one Adam step (step counts from 1). */
+typedef struct gs_adam_config {
+  double lr, beta1, beta2, eps;
+  double code_scale; /* e of the moment codes, > 0 */
+  int64_t step;
+} gs_adam_config;
+
+/* One fused Adam step over quantised SH state, in place. Per unit: decode
+ * the value p (16-bit), m from y_m = sign(m) log1p(|m| r) and v from
+ * y_v = log1p(sqrt(v) r) (8-bit codes of y; r = 1 / e rounded from double,
+ * decoded as e expm1(|y|) with y's sign); then
+ *   m' = b1 m + (1 - b1) g,  v' = b2 v + (1 - b2) g^2,
+ *   p' = p - lr (m' c1) / (sqrt(v' c2) + eps),
+ * c1 = 1 / (1 - b1^step), c2 = 1 / (1 - b2^step); each block's new bounds
+ * are the min and max of its new values (of y for the moments) and the
+ * codes are rewritten. log1p(z) = ln 2 log2(1 + z) with a software log2
+ * (atanh series) and expm1(y) = exp2(y log2 e) - 1 with the software exp2
+ * of the raster, so the codes are reproducible bit for bit. The fp32
+ * constants are the roundings of lr, b1, 1 - b1, b2, 1 - b2, c1, c2, eps,
+ * e and 1 / e, each computed in double.
+ *   grad          [device] [U][N] fp32 (e.g. d_sh + 3 N of gs_rasterize_bwd)
+ *   value_codes   [device] [U][Npad] u16, value_bounds [U][nblk][2]
+ *   m_codes, v_codes [device] [U][Npad] u8, m_bounds, v_bounds [U][nblk][2]
+ * A zero state (all codes 0, all bounds 0) is m = v = 0. One warp per block;
+ * HBM traffic 12 bytes per unit plus the bounds. Asynchronous. */
+GS_API int gs_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* value_codes, float* value_bounds,
+                            uint8_t* m_codes, float* m_bounds, uint8_t* v_codes, float* v_bounds,
+                            const gs_adam_config* cfg, void* stream);
+
 /* Views per gs_preprocess_multiview call. */
 #define GS_MAX_VIEWS 16
 

@@ -1254,12 +1254,14 @@ OR_API int or_project_f64(const double* means, const double* log_scales, const d
 //   block      256 consecutive Gaussians of one unit plane (the transposed
 //              layout); codes have row stride Npad = N rounded up to 256,
 //              bounds are [U][N/256 rounded up][2] = (lo, hi)
-//   code       q = rint(((x - lo) / (hi - lo)) * Q) clamped to [0, Q],
-//              Q = 2^bits - 1; decode lo + (hi - lo) * (q / Q); a block with
-//              hi == lo codes everything 0; fp32, no fused multiply-add
-//   moments    first moment m: y = sign(m) log1p(|m| / e); second moment v:
-//              y = log1p(sqrt(v) / e); e is the code scale (an input);
-//              decode through expm1
+//   code       per block step = (hi - lo) / Q and inv = Q / (hi - lo)
+//              (0 when hi == lo, and then every code is 0), Q = 2^bits - 1;
+//              q = rint((x - lo) * inv) clamped to [0, Q]; decode
+//              lo + step * q (the page: one multiplication per unit); fp32,
+//              no fused multiply-add
+//   moments    first moment m: y = sign(m) log1p(|m| r); second moment v:
+//              y = log1p(sqrt(v) r); e is the code scale (an input), r its
+//              reciprocal rounded from double; decode e expm1(|y|) (signed)
 //   log1p      ln 2 * log2(1 + z), log2 by the atanh series below; expm1 as
 //              exp2(y log2 e) - 1 with the software exp2 of the raster
 //   Adam       m' = b1 m + (1 - b1) g, v' = b2 v + (1 - b2) g^2,
@@ -1305,16 +1307,23 @@ float log2_spec(float y) {
 inline float log1p_spec(float z) { return QC.ln2 * log2_spec(1.0f + z); }
 inline float expm1_spec(float y) { return exp2_spec(y * KC.l2e) - 1.0f; }
 
-inline uint32_t q_encode(float x, float lo, float d, float Q) {
-  if (!(d > 0.0f)) return 0u;
-  const float t = std::rint(((x - lo) / d) * Q);
+// A block's code: its lower bound, step and inverse step.
+struct QBlock {
+  float lo, step, inv;
+};
+inline QBlock q_block(float lo, float hi, float Q) {
+  const float d = hi - lo;
+  return d > 0.0f ? QBlock{lo, d / Q, Q / d} : QBlock{lo, 0.0f, 0.0f};
+}
+inline uint32_t q_encode(float x, const QBlock& b, float Q) {
+  const float t = std::rint((x - b.lo) * b.inv);
   return t < 0.0f ? 0u : (t > Q ? (uint32_t)Q : (uint32_t)t);
 }
-inline float q_decode(uint32_t q, float lo, float d, float Q) { return lo + d * ((float)q / Q); }
+inline float q_decode(uint32_t q, const QBlock& b) { return b.lo + b.step * (float)q; }
 
-inline float m_to_log(float m, float e) { return m >= 0.0f ? log1p_spec(m / e) : -log1p_spec(-m / e); }
+inline float m_to_log(float m, float r) { return m >= 0.0f ? log1p_spec(m * r) : -log1p_spec(-m * r); }
 inline float m_from_log(float y, float e) { return y >= 0.0f ? e * expm1_spec(y) : -(e * expm1_spec(-y)); }
-inline float v_to_log(float v, float e) { return log1p_spec(std::sqrt(v) / e); }
+inline float v_to_log(float v, float r) { return log1p_spec(std::sqrt(v) * r); }
 inline float v_from_log(float y, float e) {
   const float s = e * expm1_spec(y);
   return s * s;
@@ -1337,9 +1346,9 @@ OR_API int or_quant_encode(const float* x, int64_t U, int64_t N, int bits, uint3
         lo = std::min(lo, x[u * N + g]);
         hi = std::max(hi, x[u * N + g]);
       }
-      const float d = hi - lo;
+      const QBlock qb = q_block(lo, hi, Q);
       for (int64_t g = g0; g < g0 + 256; ++g)
-        codes[u * Npad + g] = g < g1 ? q_encode(x[u * N + g], lo, d, Q) : 0u;
+        codes[u * Npad + g] = g < g1 ? q_encode(x[u * N + g], qb, Q) : 0u;
       bounds[2 * (u * nblk + b)] = lo;
       bounds[2 * (u * nblk + b) + 1] = hi;
     }
@@ -1353,8 +1362,8 @@ OR_API int or_quant_decode(const uint32_t* codes, const float* bounds, int64_t U
   for (int64_t u = 0; u < U; ++u)
     for (int64_t g = 0; g < N; ++g) {
       const int64_t b = g / 256;
-      const float lo = bounds[2 * (u * nblk + b)], hi = bounds[2 * (u * nblk + b) + 1];
-      x[u * N + g] = q_decode(codes[u * Npad + g], lo, hi - lo, Q);
+      const QBlock qb = q_block(bounds[2 * (u * nblk + b)], bounds[2 * (u * nblk + b) + 1], Q);
+      x[u * N + g] = q_decode(codes[u * Npad + g], qb);
     }
   return 0;
 }
@@ -1370,7 +1379,7 @@ OR_API int or_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint32_t* p
   const float lr = (float)lr_d, b1 = (float)beta1, ob1 = (float)(1.0 - beta1), b2 = (float)beta2,
               ob2 = (float)(1.0 - beta2), c1 = (float)(1.0 / (1.0 - std::pow(beta1, (double)step))),
               c2 = (float)(1.0 / (1.0 - std::pow(beta2, (double)step))), eps = (float)eps_d,
-              ec = (float)scale_d;
+              ec = (float)scale_d, er = (float)(1.0 / scale_d);
   const int64_t nblk = (N + 255) / 256, Npad = nblk * 256;
   const float Q16 = 65535.0f, Q8 = 255.0f;
   std::vector<float> np(256), ny(256), vy(256);
@@ -1378,19 +1387,21 @@ OR_API int or_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint32_t* p
     for (int64_t b = 0; b < nblk; ++b) {
       const int64_t g0 = b * 256, g1 = std::min(N, g0 + 256), n = g1 - g0;
       float* B[3] = {pb + 2 * (u * nblk + b), mb + 2 * (u * nblk + b), vb + 2 * (u * nblk + b)};
+      const QBlock qp = q_block(B[0][0], B[0][1], Q16), qm = q_block(B[1][0], B[1][1], Q8),
+                   qv = q_block(B[2][0], B[2][1], Q8);
       for (int64_t k = 0; k < n; ++k) {
         const int64_t c = u * Npad + g0 + k;
-        const float ph = q_decode(pc[c], B[0][0], B[0][1] - B[0][0], Q16);
-        const float mh = m_from_log(q_decode(mc[c], B[1][0], B[1][1] - B[1][0], Q8), ec);
-        const float vh = v_from_log(q_decode(vc[c], B[2][0], B[2][1] - B[2][0], Q8), ec);
+        const float ph = q_decode(pc[c], qp);
+        const float mh = m_from_log(q_decode(mc[c], qm), ec);
+        const float vh = v_from_log(q_decode(vc[c], qv), ec);
         const float g = grad[u * N + g0 + k];
         const float m1 = b1 * mh + ob1 * g;
         const float v1 = b2 * vh + ob2 * (g * g);
         const float a = m1 * c1;
         const float den = std::sqrt(v1 * c2) + eps;
         np[k] = ph - lr * (a / den);
-        ny[k] = m_to_log(m1, ec);
-        vy[k] = v_to_log(v1, ec);
+        ny[k] = m_to_log(m1, er);
+        vy[k] = v_to_log(v1, er);
       }
       const std::vector<float>* vals[3] = {&np, &ny, &vy};
       uint32_t* codes[3] = {pc, mc, vc};
@@ -1402,8 +1413,8 @@ OR_API int or_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint32_t* p
           lo = std::min(lo, y[k]);
           hi = std::max(hi, y[k]);
         }
-        const float d = hi - lo;
-        for (int64_t k = 0; k < 256; ++k) codes[t][u * Npad + g0 + k] = k < n ? q_encode(y[k], lo, d, Qs[t]) : 0u;
+        const QBlock qb = q_block(lo, hi, Qs[t]);
+        for (int64_t k = 0; k < 256; ++k) codes[t][u * Npad + g0 + k] = k < n ? q_encode(y[k], qb, Qs[t]) : 0u;
         B[t][0] = lo;
         B[t][1] = hi;
       }

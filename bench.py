@@ -125,11 +125,13 @@ def _dist_setup():
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (device times), on every rank."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 

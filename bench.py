@@ -313,6 +313,8 @@ def run_ours(args):
 
     if args.multiview and world == 1:
         line["multiview"] = multiview(args, peaks)
+    if args.interleaved > 0 and world == 1:
+        line["interleaved"] = interleaved(args, args.interleaved)
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
@@ -390,6 +392,85 @@ def adam_pass(R, params, peaks, reps=20):
                          "frac": achieved / peaks["hbm_gbs"],
                          "bytes": "4 B gradient + 4 B codes read, 4 B codes written per unit, + block bounds"},
             "state_bytes_per_unit": 4.0 + 3 * 8 * 2 / 256.0}
+
+
+def interleaved(args, G):
+    """The index-interleaved render with one exchange, G ranks emulated on
+    this GPU: each rank's phases timed with CUDA events, bytes exchanged
+    counted, and a G-GPU step modelled as the slowest rank's compute plus the
+    two exchanges at the measured 770 GB/s NVLink peer bandwidth per
+    direction (the exchanges themselves do not run here)."""
+    import torch
+    from differentiable_tile_rasterizer_b200 import synthetic
+    from differentiable_tile_rasterizer_b200.multigpu import WIRE, InterleavedRank, emulate, local_params
+    from differentiable_tile_rasterizer_b200.pipeline import GaussianParams
+    scene = synthetic.make_config(WORKLOAD_CONFIG)
+    cam = scene.cameras[0]
+    params = GaussianParams.from_scene(scene)
+    parts = [local_params(params, r, G) for r in range(G)]
+    ranks = [InterleavedRank(p.N, scene.sh_degree, cam.width, cam.height, r, G) for r, p in enumerate(parts)]
+    g = torch.from_numpy(scene.grad_image(0)).cuda()
+    bg = tuple(float(b) for b in scene.bg)
+    for _ in range(2):  # warm-up, sizes the receive buffers
+        emulate(ranks, parts, cam, bg, g)
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    reps = 5
+    t = {k: [0.0] * G for k in ("project_pack", "merge_sort_raster", "raster_bwd", "return_preprocess_bwd")}
+    for _ in range(reps):
+        packs = []
+        for r, (rk, p) in enumerate(zip(ranks, parts)):
+            a, b = ev(), ev()
+            a.record()
+            packs.append(rk.project_and_pack(p, cam))
+            b.record()
+            torch.cuda.synchronize()
+            t["project_pack"][r] += a.elapsed_time(b) / reps
+        offs = []
+        for send, counts in packs:
+            o = [0]
+            for v in counts:
+                o.append(o[-1] + v)
+            offs.append(o)
+        backs = []
+        for q, rq in enumerate(ranks):
+            recv = torch.cat([packs[s][0][offs[s][q] * WIRE: offs[s][q + 1] * WIRE] for s in range(G)])
+            a, b, c = ev(), ev(), ev()
+            a.record()
+            rq.receive_and_render(recv, [packs[s][1][q] for s in range(G)], cam, bg)
+            b.record()
+            backs.append(rq.backward_band(g))
+            c.record()
+            torch.cuda.synchronize()
+            t["merge_sort_raster"][q] += a.elapsed_time(b) / reps
+            t["raster_bwd"][q] += b.elapsed_time(c) / reps
+        for s_, rs in enumerate(ranks):
+            rows = []
+            for q in range(G):
+                back, rc = backs[q]
+                st = sum(rc[:s_])
+                rows.append(back[st: st + rc[s_]])
+            ret = torch.cat(rows).contiguous()
+            a, b = ev(), ev()
+            a.record()
+            rs.finish_backward(ret)
+            b.record()
+            torch.cuda.synchronize()
+            t["return_preprocess_bwd"][s_] += a.elapsed_time(b) / reps
+    per_rank = [sum(t[k][r] for k in t) for r in range(G)]
+    sent = [r.sent for r in ranks]
+    recvd = [r.n_recv for r in ranks]
+    # forward records out of each rank / into each rank, 64 B; gradients back, 48 B
+    fwd_bytes = max(max(s_ * WIRE for s_ in sent), max(r_ * WIRE for r_ in recvd))
+    bwd_bytes = max(max(r_ * 48 for r_ in recvd), max(s_ * 48 for s_ in sent))
+    link = 770e9
+    xchg_ms = 1e3 * (fwd_bytes + bwd_bytes) / link
+    step_ms = max(per_rank) + xchg_ms
+    return {"workload": "1m_1920x1080_sh3_pose0", "ranks": G, "emulated_on_one_gpu": True,
+            "ms_per_rank": per_rank, "phase_ms_per_rank": t, "records_sent": sent, "records_received": recvd,
+            "exchange_bytes_max_rank": {"forward": fwd_bytes, "backward": bwd_bytes},
+            "modelled": {"exchange_ms_at_770GBps": xchg_ms, "step_ms": step_ms, "frames_per_s": 1e3 / step_ms,
+                         "load_balance_max_over_mean": max(per_rank) / (sum(per_rank) / G)}}
 
 
 def multiview(args, peaks):
@@ -534,6 +615,8 @@ def main():
                     help="reference arm: sample every n-th tile per step")
     ap.add_argument("--no-importance", action="store_true", help="skip timing the importance pass")
     ap.add_argument("--no-adam", action="store_true", help="skip timing the quantised SH Adam step")
+    ap.add_argument("--interleaved", type=int, default=0,
+                    help="also emulate the index-interleaved render over this many ranks on one GPU")
     ap.add_argument("--multiview", action="store_true",
                     help="also time the eight-view 4K workload with the one-pass multi-view preprocess")
     ap.add_argument("--cpu-tile-stride", type=int, default=1,

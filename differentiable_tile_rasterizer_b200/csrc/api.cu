@@ -270,6 +270,49 @@ GS_API int gs_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* v
                                           v_bounds, hp, static_cast<cudaStream_t>(stream)));
 }
 
+GS_API int64_t gs_route_ctas(int64_t n) { return n < 0 ? 0 : route_ctas(n); }
+
+GS_API int gs_route_count(const gs_projected* rec, int64_t n, int n_ranks, int tiles_y, uint32_t* mask,
+                          uint32_t* cta_counts, int64_t* totals, void* stream) {
+  if (!records_ok(rec) || n < 0 || n >= (int64_t(1) << 31) || n_ranks < 1 || n_ranks > GS_MAX_RANKS ||
+      tiles_y < 1 || !totals || (n > 0 && (!mask || !cta_counts)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_route_count(to_records(rec), n, n_ranks, tiles_y, mask, cta_counts, totals,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_route_pack(const gs_projected* rec, const uint32_t* mask, int64_t n, int n_ranks, int rank,
+                         const uint32_t* cta_offsets, const int64_t* dst_offsets, void* send, int32_t* src_idx,
+                         void* stream) {
+  if (!records_ok(rec) || n < 0 || n >= (int64_t(1) << 31) || n_ranks < 1 || n_ranks > GS_MAX_RANKS || rank < 0 ||
+      rank >= n_ranks || (n > 0 && (!mask || !cta_offsets || !dst_offsets || !send || !src_idx)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_route_pack(to_records(rec), mask, n, n_ranks, rank, cta_offsets, dst_offsets,
+                                       static_cast<WireRecord*>(send), src_idx, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_merge_received(const void* recv, const int64_t* seg_offsets, int n_ranks, int64_t n_recv,
+                             int tile_row_lo, int tile_row_hi, const gs_projected* out, int32_t* perm,
+                             void* stream) {
+  if (!records_ok(out) || n_recv < 0 || n_recv >= (int64_t(1) << 31) || n_ranks < 1 || n_ranks > GS_MAX_RANKS ||
+      tile_row_lo < 0 || tile_row_hi < tile_row_lo || (n_recv > 0 && (!recv || !seg_offsets || !perm)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_merge(static_cast<const WireRecord*>(recv), seg_offsets, n_ranks, n_recv, tile_row_lo,
+                                  tile_row_hi, to_records(out), perm, static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_unmerge_grad2d(const float* grad2d, const int32_t* perm, int64_t n, float* back, void* stream) {
+  if (n < 0 || (n > 0 && (!grad2d || !perm || !back))) return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_unmerge_grad(reinterpret_cast<const float4*>(grad2d), perm, n,
+                                         reinterpret_cast<float4*>(back), static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_return_grad2d(const float* ret, const int32_t* src_idx, int64_t n, float* grad2d, void* stream) {
+  if (n < 0 || (n > 0 && (!ret || !src_idx || !grad2d))) return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_return_grad(reinterpret_cast<const float4*>(ret), src_idx, n,
+                                        reinterpret_cast<float4*>(grad2d), static_cast<cudaStream_t>(stream)));
+}
+
 GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const float* quats,
                              const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                              const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,

@@ -102,6 +102,30 @@ cudaError_t launch_quant_decode(const void* codes, const float* bounds, int64_t 
 cudaError_t launch_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* pc, float* pb, uint8_t* mc,
                                  float* mb, uint8_t* vc, float* vb, const float hp[10], cudaStream_t s);
 
+// exchange.cu: index-interleaved ranks and the one exchange of projected
+// records (bands of tile rows per rank).
+constexpr int kMaxRanks = 32;
+struct WireRecord {   // 64 bytes on the wire
+  float4 xyzo;
+  float4 conic;       // w: global Gaussian index (int bits)
+  float4 rgb;         // w: radius (int bits)
+  ushort4 rect;
+  uint2 pad;
+};
+static_assert(sizeof(WireRecord) == 64, "wire record layout");
+int64_t route_ctas(int64_t n);
+cudaError_t launch_route_count(const Records& rec, int64_t n, int G, int TH, uint32_t* mask, uint32_t* cta_counts,
+                               int64_t* totals, cudaStream_t s);
+cudaError_t launch_route_pack(const Records& rec, const uint32_t* mask, int64_t n, int G, int rank,
+                              const uint32_t* cta_offsets, const int64_t* dst_off, WireRecord* send,
+                              int32_t* src_idx, cudaStream_t s);
+cudaError_t launch_merge(const WireRecord* recv, const int64_t* seg_off, int G, int64_t n_recv, int y_lo, int y_hi,
+                         const Records& out, int32_t* perm, cudaStream_t s);
+cudaError_t launch_unmerge_grad(const float4* grad2d, const int32_t* perm, int64_t n, float4* back,
+                                cudaStream_t s);
+cudaError_t launch_return_grad(const float4* ret, const int32_t* src_idx, int64_t n, float4* grad2d,
+                               cudaStream_t s);
+
 // binsort.cu
 struct BinSortPlan {
   int64_t n, capacity, tiles;

@@ -25,11 +25,14 @@ GS_ERR_UNSUPPORTED = 5
 
 EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_preprocess_multiview",
             "gs_bin_sort", "gs_bin_sort_async", "gs_accumulate_grad2d_norm", "gs_quant_encode",
-            "gs_quant_decode", "gs_adam_sh_quant",
+            "gs_quant_decode", "gs_adam_sh_quant", "gs_route_ctas", "gs_route_count", "gs_route_pack",
+            "gs_merge_received", "gs_unmerge_grad2d", "gs_return_grad2d",
             "gs_rasterize_fwd", "gs_rasterize_fwd_importance", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
             "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
 GS_MAX_VIEWS = 16
+GS_WIRE_RECORD_BYTES = 64
+GS_MAX_RANKS = 32
 
 
 class GsError(RuntimeError):
@@ -88,6 +91,13 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_quant_encode.argtypes = [P, I64, I64, ctypes.c_int, P, P, P]
         L.gs_quant_decode.argtypes = [P, P, I64, I64, ctypes.c_int, P, P]
         L.gs_adam_sh_quant.argtypes = [P, I64, I64, P, P, P, P, P, P, ctypes.POINTER(GsAdamConfig), P]
+        L.gs_route_ctas.argtypes = [I64]
+        L.gs_route_ctas.restype = ctypes.c_int64
+        L.gs_route_count.argtypes = [PPROJ, I64, ctypes.c_int, ctypes.c_int, P, P, P, P]
+        L.gs_route_pack.argtypes = [PPROJ, P, I64, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
+        L.gs_merge_received.argtypes = [P, P, ctypes.c_int, I64, ctypes.c_int, ctypes.c_int, PPROJ, P, P]
+        L.gs_unmerge_grad2d.argtypes = [P, P, I64, P, P]
+        L.gs_return_grad2d.argtypes = [P, P, I64, P, P]
         L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
         L.gs_bin_sort_async.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, P, P, PSZ, P]
         L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, PCAM, P, P, P, P, P, P]
@@ -104,7 +114,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
         L.gs_debug_set_stalled_sort_tile.restype = None
         for name in ["gs_cull", "gs_preprocess", "gs_preprocess_multiview", "gs_bin_sort", "gs_accumulate_grad2d_norm",
-                     "gs_quant_encode", "gs_quant_decode", "gs_adam_sh_quant", "gs_bin_sort_async", "gs_rasterize_fwd",
+                     "gs_quant_encode", "gs_quant_decode", "gs_adam_sh_quant", "gs_route_count", "gs_route_pack",
+                     "gs_merge_received", "gs_unmerge_grad2d", "gs_return_grad2d", "gs_bin_sort_async", "gs_rasterize_fwd",
                      "gs_rasterize_fwd_importance",
                      "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
             getattr(L, name).restype = ctypes.c_int
@@ -214,6 +225,31 @@ def gs_adam_sh_quant(grad, U, N, pc, pb, mc, mb, vc, vb, lr, beta1, beta2, eps, 
     _check("gs_adam_sh_quant", load().gs_adam_sh_quant(
         _p(grad), int(U), int(N), _p(pc), _p(pb), _p(mc), _p(mb), _p(vc), _p(vb), ctypes.byref(cfg),
         _stream(stream)))
+
+
+def gs_route_count(rec: GsProjected, n, n_ranks, tiles_y, mask, cta_counts, totals, stream=None):
+    _check("gs_route_count", load().gs_route_count(ctypes.byref(rec), int(n), int(n_ranks), int(tiles_y), _p(mask),
+                                                   _p(cta_counts), _p(totals), _stream(stream)))
+
+
+def gs_route_pack(rec: GsProjected, mask, n, n_ranks, rank, cta_offsets, dst_offsets, send, src_idx, stream=None):
+    _check("gs_route_pack", load().gs_route_pack(ctypes.byref(rec), _p(mask), int(n), int(n_ranks), int(rank),
+                                                 _p(cta_offsets), _p(dst_offsets), _p(send), _p(src_idx),
+                                                 _stream(stream)))
+
+
+def gs_merge_received(recv, seg_offsets, n_ranks, n_recv, row_lo, row_hi, out: GsProjected, perm, stream=None):
+    _check("gs_merge_received", load().gs_merge_received(_p(recv), _p(seg_offsets), int(n_ranks), int(n_recv),
+                                                         int(row_lo), int(row_hi), ctypes.byref(out), _p(perm),
+                                                         _stream(stream)))
+
+
+def gs_unmerge_grad2d(grad2d, perm, n, back, stream=None):
+    _check("gs_unmerge_grad2d", load().gs_unmerge_grad2d(_p(grad2d), _p(perm), int(n), _p(back), _stream(stream)))
+
+
+def gs_return_grad2d(ret, src_idx, n, grad2d, stream=None):
+    _check("gs_return_grad2d", load().gs_return_grad2d(_p(ret), _p(src_idx), int(n), _p(grad2d), _stream(stream)))
 
 
 def gs_accumulate_grad2d_norm(grad2d, tiles_touched, active_idx, n_active, n_records, norm_sum, view_count,

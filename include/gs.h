@@ -226,6 +226,61 @@ GS_API int gs_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* v
                             uint8_t* m_codes, float* m_bounds, uint8_t* v_codes, float* v_bounds,
                             const gs_adam_config* cfg, void* stream);
 
+/* ---- Index-interleaved multi-GPU rendering with one exchange (BlitzGS
+ * write-up, section 2.1 "系统层级索引分割": Gaussians are dealt to GPUs by
+ * index, each GPU projects its own, and one centralised exchange routes the
+ * projected Gaussians to the GPUs that own the screen tiles they touch).
+ * Readings: rank r of G holds Gaussians g = l G + r (local record l) and owns
+ * the tile rows [floor(r TH / G), floor((r + 1) TH / G)); a record is sent to
+ * every rank whose rows its rect reaches; no cull. The collective is the
+ * caller's (counts, then one all-to-all of GS_WIRE_RECORD_BYTES-byte records;
+ * after the backward the reverse all-to-all of 12-float gradient rows). */
+#define GS_WIRE_RECORD_BYTES 64
+#define GS_MAX_RANKS 32
+
+/* CTAs of gs_route_count / gs_route_pack for n records (size of cta_counts
+ * is gs_route_ctas(n) * n_ranks). */
+GS_API int64_t gs_route_ctas(int64_t n);
+
+/* Which ranks each visible record (tiles_touched > 0) goes to.
+ *   mask        [device] [n] u32 out: bit q = sent to rank q
+ *   cta_counts  [device] [gs_route_ctas(n)][n_ranks] u32 out: per-CTA
+ *               exclusive offsets within each destination
+ *   totals      [device] [n_ranks] i64 out: records for each destination
+ * Asynchronous. */
+GS_API int gs_route_count(const gs_projected* rec, int64_t n, int n_ranks, int tiles_y, uint32_t* mask,
+                          uint32_t* cta_counts, int64_t* totals, void* stream);
+
+/* Packs the records for every destination into send (wire records,
+ * destination-major, each destination's records in ascending index);
+ * dst_offsets [device] [n_ranks] i64 = exclusive scan of totals;
+ * src_idx [device] [sum totals] i32 out = local record of each slot. The
+ * global index sent is l * n_ranks + rank. Asynchronous. */
+GS_API int gs_route_pack(const gs_projected* rec, const uint32_t* mask, int64_t n, int n_ranks, int rank,
+                         const uint32_t* cta_offsets, const int64_t* dst_offsets, void* send, int32_t* src_idx,
+                         void* stream);
+
+/* The received wire records (n_ranks segments, seg_offsets [device]
+ * [n_ranks + 1] i64, each ascending in global index) merged into records
+ * ordered by global index, rects clamped to the tile rows
+ * [tile_row_lo, tile_row_hi) (tiles_touched recomputed), so that bin/sort and
+ * raster on them give this rank's rows exactly as one GPU renders them.
+ *   out   records, capacity n_recv;  perm [device] [n_recv] i32 out: the
+ *         received position of each merged record. Asynchronous. */
+GS_API int gs_merge_received(const void* recv, const int64_t* seg_offsets, int n_ranks, int64_t n_recv,
+                             int tile_row_lo, int tile_row_hi, const gs_projected* out, int32_t* perm,
+                             void* stream);
+
+/* back[perm[i]] = grad2d[i] (12 floats per record): the merged records'
+ * 2-D gradients in received order, ready for the reverse exchange.
+ * Asynchronous. */
+GS_API int gs_unmerge_grad2d(const float* grad2d, const int32_t* perm, int64_t n, float* back, void* stream);
+
+/* grad2d[src_idx[j]] += ret[j] for the n returned gradient rows (vector
+ * atomics: a record sent to several ranks gets their sum). grad2d is the
+ * sender's [n_local][12] array, zeroed first. Asynchronous. */
+GS_API int gs_return_grad2d(const float* ret, const int32_t* src_idx, int64_t n, float* grad2d, void* stream);
+
 /* Views per gs_preprocess_multiview call. */
 #define GS_MAX_VIEWS 16
 

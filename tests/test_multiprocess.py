@@ -64,3 +64,45 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def _exchange_main(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from differentiable_tile_rasterizer_b200.multigpu import DistExchange
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ex = DistExchange()
+        # rank r sends (r + 1) * (q + 1) rows of 3 values to rank q, each row
+        # tagged (source, destination, row)
+        counts = [(rank + 1) * (q + 1) for q in range(world)]
+        rows = [torch.tensor([rank, q, k], dtype=torch.int64) for q in range(world) for k in range(counts[q])]
+        send = torch.stack(rows).reshape(-1)
+        recv_counts = ex.counts(counts, "cpu")
+        recv = ex.payload(send, counts, recv_counts, 3).reshape(-1, 3)
+        out.put((rank, recv_counts, recv.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_exchange_counts_and_payload_with_gloo():
+    world, port = 3, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_exchange_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = {r: (c, rows) for r, c, rows in (q.get(timeout=10) for _ in range(world))}
+    for dst in range(world):
+        counts, rows = res[dst]
+        assert counts == [(s + 1) * (dst + 1) for s in range(world)]
+        # segments in source order, rows in send order
+        want = [[s, dst, k] for s in range(world) for k in range((s + 1) * (dst + 1))]
+        assert rows == want

@@ -84,6 +84,57 @@ __device__ __forceinline__ float exp2_raster(float x) {
 
 __device__ __forceinline__ float exp_spec(float x) { return exp2_spec(__fmul_rn(x, kLog2e)); }
 
+// ---- packed fp32 pairs (the f32x2 instructions of sm_100): each half is
+// rounded exactly as the scalar round-to-nearest operation, so a pair of
+// pixels can run one instruction stream with unchanged results.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; add.rn.f32x2 rd, ra, rb;"
+      " mov.b64 {%0, %1}, rd;}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; sub.rn.f32x2 rd, ra, rb;"
+      " mov.b64 {%0, %1}, rd;}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; mul.rn.f32x2 rd, ra, rb;"
+      " mov.b64 {%0, %1}, rd;}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{.reg .b64 ra, rb, rc, rd; mov.b64 ra, {%2, %3}; mov.b64 rb, {%4, %5}; mov.b64 rc, {%6, %7};"
+      " fma.rn.f32x2 rd, ra, rb, rc; mov.b64 {%0, %1}, rd;}"
+      : "=f"(r.x), "=f"(r.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// exp2_raster on a pair (the same two results).
+__device__ __forceinline__ float2 exp2_raster2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -125.0f), fmaxf(x.y, -125.0f));
+  const float2 t = add2(xc, splat2(kRoundMagic));
+  const float2 n = sub2(t, splat2(kRoundMagic));
+  const float2 f = sub2(xc, n);
+  float2 p = splat2(kExp2C7);
+  p = fma2(p, f, splat2(kExp2C6));
+  p = fma2(p, f, splat2(kExp2C5));
+  p = fma2(p, f, splat2(kExp2C4));
+  p = fma2(p, f, splat2(kExp2C3));
+  p = fma2(p, f, splat2(kExp2C2));
+  p = fma2(p, f, splat2(kExp2C1));
+  p = fma2(p, f, splat2(1.0f));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 // SH basis at a unit direction, Y[0..K-1], in the specification's order.
 template <int K>
 __device__ __forceinline__ void sh_basis(float x, float y, float z, float* Y) {

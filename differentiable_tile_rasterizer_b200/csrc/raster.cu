@@ -323,101 +323,45 @@ __device__ __forceinline__ float warp_reduce9(const float v[9], int lane) {
   return w4 + __shfl_xor_sync(0xffffffffu, w4, 1);
 }
 
-// State of one pixel in the backward walk.
-struct BwdPixel {
-  float xc, yc;     // pixel centre
-  float T;          // transmittance in front of the current entry
-  float R0, R1, R2; // colour accumulated behind it (background included)
-  float g0, g1, g2; // dL/dimage
-  int last;         // 1 + list offset of its last blend (0: none)
+// State of a lane's two pixels in the backward walk: the same column, rows
+// r and r + 4, so dx is shared and everything else is a pair (packed fp32).
+struct BwdPair {
+  float xc;          // pixel centre column
+  float2 yc;         // pixel centre rows
+  float2 T;          // transmittance in front of the current entry
+  float2 R0, R1, R2; // colour accumulated behind it (background included)
+  float2 g0, g1, g2; // dL/dimage
+  int last0, last1;  // 1 + list offset of the last blend (0: none)
 };
 
-__device__ __forceinline__ BwdPixel load_bwd_pixel(const BwdArgs& a, int u, int v, size_t P) {
-  BwdPixel p;
-  p.xc = __fadd_rn((float)u, 0.5f);
-  p.yc = __fadd_rn((float)v, 0.5f);
-  p.R0 = a.bg0;
-  p.R1 = a.bg1;
-  p.R2 = a.bg2;
-  p.T = 1.0f;
-  p.g0 = p.g1 = p.g2 = 0.0f;
-  p.last = 0;
-  if (u < a.W && v < a.H) {
-    const size_t pix = (size_t)v * a.W + u;
-    p.T = a.final_T[pix];
-    p.last = a.last[pix];
-    p.g0 = a.dL_dimage[pix];
-    p.g1 = a.dL_dimage[P + pix];
-    p.g2 = a.dL_dimage[2 * P + pix];
+__device__ __forceinline__ BwdPair load_bwd_pair(const BwdArgs& a, int u, int v, size_t P) {
+  BwdPair q;
+  q.xc = __fadd_rn((float)u, 0.5f);
+  q.yc = make_float2(__fadd_rn((float)v, 0.5f), __fadd_rn((float)(v + 4), 0.5f));
+  q.R0 = splat2(a.bg0);
+  q.R1 = splat2(a.bg1);
+  q.R2 = splat2(a.bg2);
+  float T[2] = {1.0f, 1.0f}, g[2][3] = {{0.f, 0.f, 0.f}, {0.f, 0.f, 0.f}};
+  int last[2] = {0, 0};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int vv = v + 4 * h;
+    if (u < a.W && vv < a.H) {
+      const size_t pix = (size_t)vv * a.W + u;
+      T[h] = a.final_T[pix];
+      last[h] = a.last[pix];
+      g[h][0] = a.dL_dimage[pix];
+      g[h][1] = a.dL_dimage[P + pix];
+      g[h][2] = a.dL_dimage[2 * P + pix];
+    }
   }
-  return p;
-}
-
-// Alpha of one (pixel, entry) pair of the backward walk, recomputed exactly
-// as the forward computed it. A pair that was not a blend of the forward
-// (past the pixel's last blend, or alpha < 1/255) gets ab = 0.
-struct BwdEval {
-  float dx, dy, e, vv, ab;
-  bool contrib;
-};
-__device__ __forceinline__ BwdEval bwd_eval(const BwdPixel& p, const float4 g, const float4 co, int offk) {
-  BwdEval r;
-  r.dx = __fsub_rn(g.x, p.xc);
-  r.dy = __fsub_rn(g.y, p.yc);
-  float qv = __fmul_rn(g.z, r.dx);
-  qv = __fmaf_rn(g.w, r.dy, qv);
-  float p2 = __fmul_rn(r.dx, qv);
-  const float wv = __fmul_rn(co.x, r.dy);
-  p2 = __fmaf_rn(wv, r.dy, p2);
-  r.e = exp2_raster(p2);
-  r.vv = __fmul_rn(co.y, r.e);
-  const float alpha = fminf(r.vv, kAlphaMax);
-  r.contrib = offk < p.last && alpha >= kAlphaMin;
-  r.ab = r.contrib ? alpha : 0.0f;
-  return r;
-}
-
-// Step T and R of the pixel back over the entry and add its nine gradient
-// terms (mean2D x, y, opacity, conic A, B, C, colour r, g, b) to gv (kFirst:
-// gv is overwritten). With ab = 0 it leaves T and R unchanged and adds zeros.
-template <bool kFirst>
-__device__ __forceinline__ void bwd_grad(BwdPixel& p, const BwdEval& r, const float4 co, const float4 c,
-                                         float gv[9]) {
-  const float dx = r.dx, dy = r.dy, ab = r.ab;
-  const float oma = 1.0f - ab;
-  // transmittance in front of this entry (gradient values only)
-  p.T = r.contrib ? __fdividef(p.T, oma) : p.T;
-  const float wgt = ab * p.T;
-  const float Gk = p.T * (p.g0 * (c.x - p.R0) + p.g1 * (c.y - p.R1) + p.g2 * (c.z - p.R2));
-  const float Gm = (r.contrib && r.vv < kAlphaMax) ? Gk : 0.0f;  // no gradient through a clamped alpha
-  const float dp = Gm * ab;
-  const float A = co.z, B = co.w, Cc = c.w;
-  const float t0 = fmaf(A, dx, B * dy), t1 = fmaf(B, dx, Cc * dy);
-  const float ndp = -dp, hdx = -0.5f * dp * dx, ndx = ndp * dx, hdy = -0.5f * dp * dy;
-  if (kFirst) {
-    gv[0] = ndp * t0;
-    gv[1] = ndp * t1;
-    gv[2] = Gm * r.e;
-    gv[3] = hdx * dx;
-    gv[4] = ndx * dy;
-    gv[5] = hdy * dy;
-    gv[6] = p.g0 * wgt;
-    gv[7] = p.g1 * wgt;
-    gv[8] = p.g2 * wgt;
-  } else {
-    gv[0] = fmaf(ndp, t0, gv[0]);
-    gv[1] = fmaf(ndp, t1, gv[1]);
-    gv[2] = fmaf(Gm, r.e, gv[2]);
-    gv[3] = fmaf(hdx, dx, gv[3]);
-    gv[4] = fmaf(ndx, dy, gv[4]);
-    gv[5] = fmaf(hdy, dy, gv[5]);
-    gv[6] = fmaf(p.g0, wgt, gv[6]);
-    gv[7] = fmaf(p.g1, wgt, gv[7]);
-    gv[8] = fmaf(p.g2, wgt, gv[8]);
-  }
-  p.R0 = fmaf(c.x, ab, oma * p.R0);
-  p.R1 = fmaf(c.y, ab, oma * p.R1);
-  p.R2 = fmaf(c.z, ab, oma * p.R2);
+  q.T = make_float2(T[0], T[1]);
+  q.g0 = make_float2(g[0][0], g[1][0]);
+  q.g1 = make_float2(g[0][1], g[1][1]);
+  q.g2 = make_float2(g[0][2], g[1][2]);
+  q.last0 = last[0];
+  q.last1 = last[1];
+  return q;
 }
 
 // Backward CTA: 4 warps per tile, warp w owns the 8x8 block at
@@ -438,9 +382,8 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
   const int u = tx0 + (warp & 1) * 8 + (lane & 7), v = ty0 + (warp >> 1) * 8 + (lane >> 3);
   const uint2 range = a.ranges[tile];
   const size_t P = (size_t)a.W * a.H;
-  BwdPixel p0 = load_bwd_pixel(a, u, v, P);
-  BwdPixel p1 = load_bwd_pixel(a, u, v + 4, P);
-  const int warp_last = __reduce_max_sync(0xffffffffu, max(p0.last, p1.last));
+  BwdPair px = load_bwd_pair(a, u, v, P);
+  const int warp_last = __reduce_max_sync(0xffffffffu, max(px.last0, px.last1));
   const Reduce9Slot slot = reduce9_slot(lane);
   if (tid == 0) s_maxlast = 0;
   __syncthreads();
@@ -502,15 +445,57 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
         const int k = c0 + __ffs(msk) - 1;
         msk &= msk - 1;
         const int offk = n - 1 - done - k;
-        const float4 g = s_geo[k];
-        const float4 co = s_co[k];
-        const BwdEval e0 = bwd_eval(p0, g, co, offk), e1 = bwd_eval(p1, g, co, offk);
-        // no pixel of the warp blended this entry: T and R stay, no terms
-        if (!__any_sync(0xffffffffu, e0.contrib || e1.contrib)) continue;
-        const float4 c = s_rgb[k];
+        const float4 g = s_geo[k];   // px, py, a2, b2
+        const float4 co = s_co[k];   // c2, opacity, A, B
+        // alpha of both pixels, recomputed exactly as the forward computed
+        // it (the same operations; dx is common to the pair)
+        const float dx = __fsub_rn(g.x, px.xc);
+        const float2 dy = sub2(splat2(g.y), px.yc);
+        const float2 qv = fma2(splat2(g.w), dy, splat2(__fmul_rn(g.z, dx)));
+        float2 p2 = mul2(splat2(dx), qv);
+        p2 = fma2(mul2(splat2(co.x), dy), dy, p2);
+        const float2 e = exp2_raster2(p2);
+        const float2 vv = mul2(splat2(co.y), e);
+        const float al0 = fminf(vv.x, kAlphaMax), al1 = fminf(vv.y, kAlphaMax);
+        // a pair that was not a blend of the forward (past the pixel's last
+        // blend, or alpha < 1/255) runs with alpha 0: T and R stay, no terms
+        const bool b0 = offk < px.last0 && al0 >= kAlphaMin, b1 = offk < px.last1 && al1 >= kAlphaMin;
+        if (!__any_sync(0xffffffffu, b0 || b1)) continue;
+        const float2 ab = make_float2(b0 ? al0 : 0.0f, b1 ? al1 : 0.0f);
+        const float2 oma = sub2(splat2(1.0f), ab);
+        // transmittance in front of this entry (gradient values only)
+        px.T = make_float2(b0 ? __fdividef(px.T.x, oma.x) : px.T.x, b1 ? __fdividef(px.T.y, oma.y) : px.T.y);
+        const float2 wgt = mul2(ab, px.T);
+        const float4 c = s_rgb[k];   // r, g, b, C
+        float2 sg = mul2(px.g0, sub2(splat2(c.x), px.R0));
+        sg = fma2(px.g1, sub2(splat2(c.y), px.R1), sg);
+        sg = fma2(px.g2, sub2(splat2(c.z), px.R2), sg);
+        const float2 Gk = mul2(px.T, sg);
+        // no gradient through a clamped alpha
+        const float2 Gm = make_float2((b0 && vv.x < kAlphaMax) ? Gk.x : 0.0f, (b1 && vv.y < kAlphaMax) ? Gk.y : 0.0f);
+        const float2 dp = mul2(Gm, ab);
+        const float2 dpdy = mul2(dp, dy);
+        const float2 dpdy2 = mul2(dpdy, dy);
+        const float2 ge = mul2(Gm, e);
+        const float2 w0 = mul2(px.g0, wgt), w1 = mul2(px.g1, wgt), w2 = mul2(px.g2, wgt);
+        // the nine terms summed over the pair (mean2D x, y, opacity, conic
+        // A, B, C, colour r, g, b); dp/dpx = -(A dx + B dy), dp/dA = -dx^2/2,
+        // dp/dB = -dx dy, dp/dC = -dy^2/2
+        const float sdp = dp.x + dp.y, sdpdy = dpdy.x + dpdy.y;
+        const float A = co.z, B = co.w, Cc = c.w, dxs = dx * sdp;
         float gv[9];
-        bwd_grad<true>(p0, e0, co, c, gv);
-        bwd_grad<false>(p1, e1, co, c, gv);
+        gv[0] = -fmaf(A, dxs, B * sdpdy);
+        gv[1] = -fmaf(B, dxs, Cc * sdpdy);
+        gv[2] = ge.x + ge.y;
+        gv[3] = -0.5f * dx * dxs;
+        gv[4] = -dx * sdpdy;
+        gv[5] = -0.5f * (dpdy2.x + dpdy2.y);
+        gv[6] = w0.x + w0.y;
+        gv[7] = w1.x + w1.y;
+        gv[8] = w2.x + w2.y;
+        px.R0 = fma2(splat2(c.x), ab, mul2(oma, px.R0));
+        px.R1 = fma2(splat2(c.y), ab, mul2(oma, px.R1));
+        px.R2 = fma2(splat2(c.z), ab, mul2(oma, px.R2));
         const float tot = warp_reduce9(gv, lane);
         if (slot.owner) atomicAdd(&s_acc[k][slot.idx], tot);
       }

@@ -206,23 +206,14 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
       const int j = c0 + lane;
       const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy, 3.5f, 1.5f);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
-      // Branch-free body: a lane that skips the pair (alpha < 1/255) or has
-      // already stopped blends with alpha 0, which leaves C, T and the counts
-      // exactly as they were (colours are finite), so the warp never diverges.
-      while (msk) {
-        const int k = c0 + __ffs(msk) - 1;
-        msk &= msk - 1;
-        const float4 g = s_geo[k];
-        const float2 co = s_co[k];
+      // Entries are taken two at a time: their alphas at this pixel run as
+      // one packed pair (each half rounded as the scalar operation), then
+      // they blend in list order. Branch-free blend: a lane that skips an
+      // entry (alpha < 1/255) or has already stopped blends with alpha 0,
+      // which leaves C, T and the counts exactly as they were (colours are
+      // finite), so the warp never diverges.
+      auto blend_one = [&](int k, float alpha) {
         const float4 c = s_rgb[k];
-        const float dx = __fsub_rn(g.x, xc), dy = __fsub_rn(g.y, yc);
-        float qv = __fmul_rn(g.z, dx);
-        qv = __fmaf_rn(g.w, dy, qv);
-        float p2 = __fmul_rn(dx, qv);
-        const float wv = __fmul_rn(co.x, dy);
-        p2 = __fmaf_rn(wv, dy, p2);
-        const float e = exp2_raster(p2);
-        const float alpha = fminf(__fmul_rn(co.y, e), kAlphaMax);
         const bool blend = !done && alpha >= kAlphaMin;
         const float ab = blend ? alpha : 0.0f;
         const float wgt = __fmul_rn(ab, T);
@@ -239,6 +230,24 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
           for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
           if (lane == 0 && ws != 0.0f) atomicAdd(&s_imp[k], ws);
         }
+      };
+      while (msk) {
+        const int k1 = c0 + __ffs(msk) - 1;
+        msk &= msk - 1;
+        const bool has2 = msk != 0;  // the same for the whole warp
+        const int k2 = has2 ? c0 + __ffs(msk) - 1 : k1;
+        msk &= msk - 1;
+        const float4 g1 = s_geo[k1], g2 = s_geo[k2];
+        const float2 co1 = s_co[k1], co2 = s_co[k2];
+        const float2 dx = sub2(make_float2(g1.x, g2.x), splat2(xc));
+        const float2 dy = sub2(make_float2(g1.y, g2.y), splat2(yc));
+        const float2 qv = fma2(make_float2(g1.w, g2.w), dy, mul2(make_float2(g1.z, g2.z), dx));
+        float2 p2 = mul2(dx, qv);
+        p2 = fma2(mul2(make_float2(co1.x, co2.x), dy), dy, p2);
+        const float2 e = exp2_raster2(p2);
+        const float2 va = mul2(make_float2(co1.y, co2.y), e);
+        blend_one(k1, fminf(va.x, kAlphaMax));
+        if (has2) blend_one(k2, fminf(va.y, kAlphaMax));
       }
     }
   }

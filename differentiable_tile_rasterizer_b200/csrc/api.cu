@@ -186,18 +186,25 @@ GS_API int gs_bin_sort_async(const gs_projected* in, int64_t n, const gs_camera*
   return cuda_status(launch_publish(workspace, plan, result, static_cast<cudaStream_t>(stream)));
 }
 
+GS_API int gs_tile_order(const uint32_t* tile_ranges, int64_t n_tiles, uint32_t* order, void* stream) {
+  if (n_tiles < 0 || n_tiles >= (int64_t(1) << 31) || (n_tiles > 0 && (!tile_ranges || !order)))
+    return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_tile_order(tile_ranges, n_tiles, order, static_cast<cudaStream_t>(stream)));
+}
+
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,
-                            const gs_camera* cam, const float* bg, float* image, float* final_T,
+                            const uint32_t* tile_order, const gs_camera* cam, const float* bg, float* image, float* final_T,
                             int32_t* n_contrib, int32_t* last, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last)
     return GS_ERR_INVALID_ARGUMENT;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
-                                       n_contrib, last, nullptr, nullptr, static_cast<cudaStream_t>(stream)));
+                                       n_contrib, last, nullptr, nullptr, tile_order,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,
-                                       const gs_camera* cam, const float* bg, const int32_t* active_idx,
+                                       const uint32_t* tile_order, const gs_camera* cam, const float* bg, const int32_t* active_idx,
                                        float* image, float* final_T, int32_t* n_contrib, int32_t* last,
                                        float* importance, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last ||
@@ -205,21 +212,21 @@ GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* v
     return GS_ERR_INVALID_ARGUMENT;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
-                                       n_contrib, last, importance, active_idx,
+                                       n_contrib, last, importance, active_idx, tile_order,
                                        static_cast<cudaStream_t>(stream)));
 }
 
 GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,
-                               const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
-                               const float* final_T, const int32_t* last, const float* dL_dimage,
-                               float* grad2d, void* stream) {
+                               const uint32_t* tile_ranges, const uint32_t* tile_order, const gs_camera* cam,
+                               const float* bg, const float* final_T, const int32_t* last,
+                               const float* dL_dimage, float* grad2d, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || n_records < 0 || n_records >= (int64_t(1) << 31) || !tile_ranges ||
       !bg || !final_T || !last || !dL_dimage || (n_records > 0 && !grad2d))
     return GS_ERR_INVALID_ARGUMENT;
   if (n_records == 0) return GS_OK;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_bwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, final_T, last,
-                                       dL_dimage, reinterpret_cast<float4*>(grad2d), n_records,
+                                       dL_dimage, reinterpret_cast<float4*>(grad2d), n_records, tile_order,
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -337,8 +344,9 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
                             const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                             const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
                             const gs_camera* cam, const gs_projected* in, const uint32_t* vals,
-                            const uint32_t* tile_ranges, const float* bg, const float* final_T,
-                            const int32_t* last, const float* dL_dimage, float* grad2d, float* d_means,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order, const float* bg,
+                            const float* final_T, const int32_t* last, const float* dL_dimage,
+                            float* grad2d, float* d_means,
                             float* d_log_scales, float* d_quats, float* d_opacity_logits, float* d_sh,
                             void* stream) {
   if (sh_degree < 0) return GS_ERR_INVALID_ARGUMENT;
@@ -354,7 +362,7 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
   const float b[3] = {bg[0], bg[1], bg[2]};
   if (N > 0) {
     cudaError_t e = launch_raster_bwd(rec, vals, tile_ranges, dc, b, final_T, last, dL_dimage,
-                                      reinterpret_cast<float4*>(grad2d), N, s);
+                                      reinterpret_cast<float4*>(grad2d), N, tile_order, s);
     if (e != cudaSuccess) return GS_ERR_CUDA;
   }
   Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};

@@ -120,12 +120,41 @@ __device__ __forceinline__ bool region_hits(const float4 b, const float4 q1, con
 __device__ __forceinline__ float block_cx(int tx0, int w) { return (float)(tx0 + (w & 1) * 8) + 4.0f; }
 __device__ __forceinline__ float block_cy(int ty0, int w) { return (float)(ty0 + (w >> 1) * 4) + 2.0f; }
 
+// Tiles in descending order of log2 of their list length: a launch that takes
+// its CTAs' tiles in this order starts the longest lists first, so few long
+// CTAs are left running alone at the end. One CTA; counting sort over 33
+// buckets, the order inside a bucket unspecified (it does not change results).
+__global__ void __launch_bounds__(1024) tile_order_kernel(const uint2* ranges, int64_t TT, uint32_t* order) {
+  __shared__ uint32_t cnt[33];
+  if (threadIdx.x < 33) cnt[threadIdx.x] = 0;
+  __syncthreads();
+  for (int64_t t = threadIdx.x; t < TT; t += 1024) {
+    const uint32_t len = ranges[t].y - ranges[t].x;
+    atomicAdd(&cnt[len ? 32 - __clz(len) : 0], 1u);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t run = 0;
+    for (int b = 32; b >= 0; --b) {
+      const uint32_t c = cnt[b];
+      cnt[b] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int64_t t = threadIdx.x; t < TT; t += 1024) {
+    const uint32_t len = ranges[t].y - ranges[t].x;
+    order[atomicAdd(&cnt[len ? 32 - __clz(len) : 0], 1u)] = (uint32_t)t;
+  }
+}
+
 struct FwdArgs {
   const float4* xyzo;
   const float4* conic;
   const float4* rgb;
   const uint32_t* vals;
   const uint2* ranges;
+  const uint32_t* order;  // tile of CTA b (null: tile b)
   int W, H, TW;
   float bg0, bg1, bg2;
   float* image;
@@ -148,7 +177,9 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   __shared__ float4 s_box[kBatchF];  // blend region of each staged entry
   __shared__ float4 s_q1[kBatchF];
   __shared__ float4 s_q2[kBatchF];
-  const int tile = blockIdx.x;
+  const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
+  if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
+  const int tile = (int)tile_u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int du, dv;
   tile_pixel(tid, du, dv);
@@ -272,6 +303,7 @@ struct BwdArgs {
   const float4* rgb;
   const uint32_t* vals;
   const uint2* ranges;
+  const uint32_t* order;  // tile of CTA b (null: tile b)
   int W, H, TW;
   float bg0, bg1, bg2;
   const float* final_T;
@@ -385,7 +417,9 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
   __shared__ uint8_t s_hit[kBatchB];    // bit w: the entry can blend in warp w's block
   __shared__ float s_acc[kBatchB][9];   // per-batch gradient sums of the CTA ([slot][value]: conflict-free)
   __shared__ int s_maxlast;
-  const int tile = blockIdx.x;
+  const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
+  if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
+  const int tile = (int)tile_u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
   const int u = tx0 + (warp & 1) * 8 + (lane & 7), v = ty0 + (warp >> 1) * 8 + (lane >> 3);
@@ -536,10 +570,10 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], float* image, float* final_T,
                               int32_t* n_contrib, int32_t* last, float* importance, const int32_t* active_idx,
-                              cudaStream_t s) {
+                              const uint32_t* order, cudaStream_t s) {
   FwdArgs a;
   a.xyzo = rec.xyzo; a.conic = rec.conic; a.rgb = rec.rgb;
-  a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges);
+  a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges); a.order = order;
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.image = image; a.final_T = final_T; a.n_contrib = n_contrib; a.last = last;
@@ -555,16 +589,23 @@ cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const ui
 cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], const float* final_T,
                               const int32_t* last, const float* dL_dimage, float4* grad2d,
-                              int64_t n_records, cudaStream_t s) {
+                              int64_t n_records, const uint32_t* order, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(grad2d, 0, (size_t)n_records * 3 * sizeof(float4), s);
   if (e != cudaSuccess) return e;
   BwdArgs a;
   a.xyzo = rec.xyzo; a.conic = rec.conic; a.rgb = rec.rgb;
-  a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges);
+  a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges); a.order = order;
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d;
   raster_bwd_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_order(const uint32_t* ranges, int64_t TT, uint32_t* order, cudaStream_t s) {
+  if (TT == 0) return cudaSuccess;
+  tile_order_kernel<<<1, 1024, 0, s>>>(reinterpret_cast<const uint2*>(ranges), TT, order);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -108,6 +108,10 @@ class Rasterizer:
         self.n_contrib = torch.empty((height, width), **i32)
         self.last = torch.empty((height, width), **i32)
         self.ranges = torch.empty((self.TT, 2), **i32)
+        # Tiles longest list first (gs_tile_order), computed after every bin
+        # sort and given to the raster launches; None: CTA b takes tile b.
+        self.schedule_tiles = True
+        self.tile_order = torch.arange(max(self.TT, 1), **i32)
         self.grad2d = torch.empty((n, 12), **f32)
         self.grads = {"means": torch.empty((3, n), **f32), "log_scales": torch.empty((3, n), **f32),
                       "quats": torch.empty((4, n), **f32), "opacity_logits": torch.empty(n, **f32),
@@ -171,6 +175,9 @@ class Rasterizer:
         with self._timed("bin_sort"):
             return self._bin_sort(cam)
 
+    def _order(self):
+        return self.tile_order if self.schedule_tiles else None
+
     def _bin_sort(self, cam: gs.GsCamera):
         offs = self.offsets if self.want_offsets else None
         if self.deferred:
@@ -179,6 +186,8 @@ class Rasterizer:
             gs.gs_bin_sort_async(self._proj, self.N, cam, offs, self.keys, self.vals, self.capacity,
                                  self.ranges, self._results[self._n_pending], self.sort_ws)
             self._n_pending += 1
+            if self.schedule_tiles:
+                gs.gs_tile_order(self.ranges, self.TT, self.tile_order)
             return None
         st, ni = gs.gs_bin_sort(self._proj, self.N, cam, offs, self.keys, self.vals, self.capacity,
                                 self.ranges, self.sort_ws, raise_on_capacity=False)
@@ -187,6 +196,8 @@ class Rasterizer:
             st, ni = gs.gs_bin_sort(self._proj, self.N, cam, offs, self.keys, self.vals,
                                     self.capacity, self.ranges, self.sort_ws)
         self.n_instances = ni
+        if self.schedule_tiles:
+            gs.gs_tile_order(self.ranges, self.TT, self.tile_order)
         return ni
 
     def forward_importance(self, params: GaussianParams, cam, importance: torch.Tensor, bg=(0.0, 0.0, 0.0),
@@ -205,7 +216,8 @@ class Rasterizer:
         self.bin_sort(c)
         with self._timed("raster_fwd_importance"):
             gs.gs_rasterize_fwd_importance(self._proj, self.vals, self.ranges, c, self.bg, self.active_idx,
-                                           self.image, self.final_T, self.n_contrib, self.last, importance)
+                                           self.image, self.final_T, self.n_contrib, self.last, importance,
+                                           tile_order=self._order())
         return self.image
 
     def accumulate_grad_stats(self, norm_sum: torch.Tensor, view_count: torch.Tensor):
@@ -237,7 +249,7 @@ class Rasterizer:
     def raster_fwd(self, cam: gs.GsCamera, bg):
         with self._timed("raster_fwd"):
             gs.gs_rasterize_fwd(self._proj, self.vals, self.ranges, cam, bg, self.image, self.final_T,
-                                self.n_contrib, self.last)
+                                self.n_contrib, self.last, tile_order=self._order())
 
     # ------------------------------------------------------------------ public
     def forward(self, params: GaussianParams, cam, bg=(0.0, 0.0, 0.0), lod_dist=0.0,
@@ -262,12 +274,13 @@ class Rasterizer:
             gs.gs_rasterize_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
                                 self.N, act, na, mask, c, self._proj, self.vals, self.ranges, self.bg,
                                 self.final_T, self.last, dL_dimage, self.grad2d, g["means"],
-                                g["log_scales"], g["quats"], g["opacity_logits"], g["sh"])
+                                g["log_scales"], g["quats"], g["opacity_logits"], g["sh"],
+                                tile_order=self._order())
             return g
         # the same two parts as separate calls, so each can be timed
         with self._timed("raster_bwd"):
             gs.gs_rasterize_bwd_2d(self._proj, self.N, self.vals, self.ranges, c, self.bg, self.final_T,
-                                   self.last, dL_dimage, self.grad2d)
+                                   self.last, dL_dimage, self.grad2d, tile_order=self._order())
         with self._timed("preprocess_bwd"):
             gs.gs_preprocess_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
                                  self.N, act, na, mask, c, self._proj, self.grad2d, g["means"],
@@ -338,7 +351,8 @@ class MultiViewRenderer:
             with self._timed("bin_sort"):
                 R._bin_sort(c)
             with self._timed("raster_fwd"):
-                gs.gs_rasterize_fwd(R._proj, R.vals, R.ranges, c, bg, R.image, R.final_T, R.n_contrib, R.last)
+                gs.gs_rasterize_fwd(R._proj, R.vals, R.ranges, c, bg, R.image, R.final_T, R.n_contrib, R.last,
+                                    tile_order=R._order())
         return [R.image for R in self.views]
 
     def set_deferred(self, on: bool):

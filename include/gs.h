@@ -348,12 +348,26 @@ GS_API int gs_bin_sort_async(const gs_projected* in, int64_t n, const gs_camera*
                              uint64_t* keys, uint32_t* vals, int64_t capacity, uint32_t* tile_ranges,
                              int64_t* result, void* workspace, size_t* workspace_bytes, void* stream);
 
+/* Tile schedule for the raster launches: the tile indices ordered by
+ * descending floor(log2) of their list length (empty lists last), so that the
+ * CTAs that take the longest lists start first and the launch does not end on
+ * a few long tiles running alone (a longest-processing-time-first schedule;
+ * without it, CTA b takes tile b). The order within one length class is
+ * unspecified. The raster outputs do not depend on it.
+ *   tile_ranges  [device] [n_tiles] (start, end) u32 pairs from gs_bin_sort
+ *   order        [device] [n_tiles] u32 out: a permutation of 0 .. n_tiles - 1
+ * One CTA. Asynchronous; GS_ERR_INVALID_ARGUMENT on NULL pointers with
+ * n_tiles > 0 or n_tiles outside [0, 2^31). */
+GS_API int gs_tile_order(const uint32_t* tile_ranges, int64_t n_tiles, uint32_t* order, void* stream);
+
 /* Forward compositing (tiled rasterization with alpha blending). For each
  * pixel, over its tile's sorted list: alpha = min(0.99, o exp(p)) with
  * p = -1/2 (A dx^2 + C dy^2) - B dx dy, (dx, dy) = (px - u - 0.5, py - v - 0.5);
  * skip alpha < 1/255; C += T alpha c; T *= 1 - alpha; stop once T < 1e-4
  * (the crossing Gaussian is blended). out = C + T bg.
  *   vals, tile_ranges [device] from gs_bin_sort
+ *   tile_order   [device] [tiles] u32 from gs_tile_order, or NULL: the order
+ *                in which the CTAs take the tiles; it changes no output bit
  *   bg           [host] 3 floats
  *   image        [device] [3][H][W] out
  *   final_T      [device] [H][W] out
@@ -361,7 +375,8 @@ GS_API int gs_bin_sort_async(const gs_projected* in, int64_t n, const gs_camera*
  *   last         [device] [H][W] i32 out: 1 + list offset of the last blend
  * Asynchronous. */
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
-                            const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order,
+                            const gs_camera* cam, const float* bg,
                             float* image, float* final_T, int32_t* n_contrib, int32_t* last,
                             void* stream);
 
@@ -372,7 +387,8 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
  * view-level importance cull of gs_cull). The page prints no formula. It is
  * read as the sum over the view's pixels of the blend weight alpha * T of
  * each of the Gaussian's blends, with the forward's own fp32 values. The
- * image outputs equal gs_rasterize_fwd's bit for bit.
+ * image outputs equal gs_rasterize_fwd's bit for bit. tile_order as for
+ * gs_rasterize_fwd.
  *   active_idx   [device] [n_records] i32 or NULL: Gaussian of record i
  *                (from gs_cull; NULL: record i is Gaussian i)
  *   importance   [device] [N] f32 in/out: this view's weights are ADDED, so
@@ -380,7 +396,8 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
  * The sums are fp32 atomics in an unspecified order (a warp sum, a CTA sum,
  * then one atomic per (Gaussian, tile)). Asynchronous. */
 GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* vals,
-                                       const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                                       const uint32_t* tile_ranges, const uint32_t* tile_order,
+                                       const gs_camera* cam, const float* bg,
                                        const int32_t* active_idx, float* image, float* final_T,
                                        int32_t* n_contrib, int32_t* last, float* importance, void* stream);
 
@@ -392,6 +409,7 @@ GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* v
  *   params, sh_degree, N, active_idx, n_active: as given to gs_preprocess
  *   mask         [device] [N] u8 from gs_cull or NULL (all active)
  *   in           records from gs_preprocess
+ *   tile_order   as for gs_rasterize_fwd (any permutation, or NULL)
  *   final_T, last from gs_rasterize_fwd; dL_dimage [device] [3][H][W]
  *   grad2d       [device] [N][12] f32 out: (dpx, dpy, dopacity, 0,
  *                dA, dB, dC, 0, dr, dg, db, 0) per record
@@ -402,9 +420,9 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
                             const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                             const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
                             const gs_camera* cam, const gs_projected* in, const uint32_t* vals,
-                            const uint32_t* tile_ranges, const float* bg, const float* final_T,
-                            const int32_t* last, const float* dL_dimage, float* grad2d,
-                            float* d_means, float* d_log_scales, float* d_quats,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order, const float* bg,
+                            const float* final_T, const int32_t* last, const float* dL_dimage,
+                            float* grad2d, float* d_means, float* d_log_scales, float* d_quats,
                             float* d_opacity_logits, float* d_sh, void* stream);
 
 /* Part 1 of gs_rasterize_bwd alone: the back-to-front replay that writes the
@@ -412,7 +430,8 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
  * chaining them to the parameters. Same arguments as the corresponding ones
  * of gs_rasterize_bwd; n_records = N. Asynchronous. */
 GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,
-                               const uint32_t* tile_ranges, const gs_camera* cam, const float* bg,
+                               const uint32_t* tile_ranges, const uint32_t* tile_order,
+                               const gs_camera* cam, const float* bg,
                                const float* final_T, const int32_t* last, const float* dL_dimage,
                                float* grad2d, void* stream);
 

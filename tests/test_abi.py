@@ -56,3 +56,9 @@ def test_workspace_queries_need_no_gpu():
     with pytest.raises(gs.GsError):
         gs.gs_cull_workspace(10, cam)
 
+
+def test_tile_order_argument_checks_need_no_gpu():
+    L = gs.load()
+    assert L.gs_tile_order(None, -1, None, None) == gs.GS_ERR_INVALID_ARGUMENT
+    assert L.gs_tile_order(None, 10, None, None) == gs.GS_ERR_INVALID_ARGUMENT
+    assert L.gs_tile_order(None, 1 << 31, None, None) == gs.GS_ERR_INVALID_ARGUMENT

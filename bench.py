@@ -48,6 +48,40 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
+# Sources whose compiled code the raster kernels are: a traffic figure taken
+# with ncu counts only while their hash is the one recorded beside it.
+RASTER_SOURCES = ("differentiable_tile_rasterizer_b200/csrc/raster.cu",
+                  "differentiable_tile_rasterizer_b200/csrc/gs_device.cuh")
+TRAFFIC_PROFILE = "profiles/raster_kernels_1m_1080p_sh3.md"
+
+
+def raster_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in RASTER_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` (dram__bytes_read.sum +
+    dram__bytes_write.sum, averaged over the captured launches) from the
+    committed ncu summary, or None when the summary has no figure for it or
+    the kernel sources changed since it was taken. Summary line format:
+    `traffic <kernel> bytes_per_launch=<B> launches=<n> source=<hash>`."""
+    p = os.path.join(ROOT, TRAFFIC_PROFILE)
+    if not os.path.exists(p):
+        return None
+    want = raster_source_hash()
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 5 and f[0] == "traffic" and f[1] == kernel + "_kernel":
+            kv = dict(t.split("=", 1) for t in f[2:] if "=" in t)
+            if kv.get("source") == want:
+                return float(kv["bytes_per_launch"])
+    return None
+
+
 class ClockSampler:
     """nvidia-smi clock and throttle samples during the timed region."""
 
@@ -276,7 +310,7 @@ def run_ours(args):
         ops_per_launch = per_kernel[dom] / len(poses)
         achieved = ops_per_launch / (avg_ms * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
-                "frac": achieved / peak_alu, "traffic": None,
+                "frac": achieved / peak_alu, "traffic": profiled_traffic(dom),
                 "peak_source": f"148 SMs x 128 fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz (fp32 ops, FMA = 1)",
                 "ops_per_launch": ops_per_launch, "avg_launch_ms": avg_ms}
     else:

@@ -3,8 +3,9 @@
 // linear block codes of the logarithms of both Adam moments, one (lo, hi)
 // pair per 256 consecutive Gaussians of a unit plane, fp32 gradients.
 //
-// One warp per block of 256 units; lane l takes units l, l + 32, ..., so
-// every load and store of the warp is one contiguous run. The warp decodes,
+// One warp per block of 256 units; lane l takes the 8 consecutive units
+// 8 l .. 8 l + 7, so its codes move as one 16-byte and two 8-byte words and
+// every access of the warp is one contiguous run. The warp decodes,
 // steps, finds the new bounds with shuffles and re-encodes, all in fp32 in
 // the order fixed by the specification (no fused multiply-add except in the
 // log2 polynomial, where it is part of the definition). HBM-bound: per unit
@@ -70,6 +71,7 @@ __device__ __forceinline__ uint32_t q_encode(float x, const QBlock& b, float Q) 
 __device__ __forceinline__ float q_decode(uint32_t q, const QBlock& b) {
   return __fadd_rn(b.lo, __fmul_rn(b.step, (float)q));
 }
+__device__ __forceinline__ float q_decode_f(float q, const QBlock& b) { return __fadd_rn(b.lo, __fmul_rn(b.step, q)); }
 // r = 1 / e, the code scale's reciprocal
 // (one log1p / expm1 per unit, the sign applied after: the same values as
 // the two-branch form, -0 included)
@@ -143,62 +145,132 @@ struct AdamArgs {
   uint8_t* vc;
   float2* vb;
   float lr, b1, ob1, b2, ob2, c1, c2, eps, ec, er;
+  bool vec_codes;  // pc 16-byte, mc and vc 8-byte aligned
+  bool vec_grad;   // grad 16-byte aligned and N % 4 == 0
 };
 
-__global__ void __launch_bounds__(256) adam_sh_quant_kernel(AdamArgs a) {
-  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (wid >= a.U * a.nblk) return;  // whole warps
-  const int lane = threadIdx.x & 31;
+// (float)q of a code q < 2^23, exactly: q placed in the mantissa of 2^23,
+// minus 2^23 (the byte permute builds the bit pattern in one instruction).
+__device__ __forceinline__ float code_u8(uint32_t w, int k) {
+  return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540u + (uint32_t)k)), 8388608.0f);
+}
+__device__ __forceinline__ float code_u16(uint32_t w, int hi) {
+  return __fsub_rn(__uint_as_float(__byte_perm(w, 0x4B000000u, hi ? 0x7432u : 0x7410u)), 8388608.0f);
+}
+// q_encode with one conversion: round to nearest even and saturate to
+// [0, 2^32 - 1] (NaN -> 0), then clamp to Q; the same code for every input.
+__device__ __forceinline__ uint32_t q_encode_fast(float x, const QBlock& b, uint32_t Q) {
+  return min(__float2uint_rn(__fmul_rn(__fsub_rn(x, b.lo), b.inv)), Q);
+}
+
+// Lane l of the warp takes the units 8 l .. 8 l + 7 of the block (so the
+// codes of a lane are one 16-byte and two 8-byte words). kFull: all 256
+// units of the block are valid.
+template <bool kFull>
+__device__ __forceinline__ void adam_block(const AdamArgs& a, int64_t wid, int lane) {
   const int64_t u = wid / a.nblk, g0 = (wid % a.nblk) * kBlockUnits;
-  const int64_t row = u * a.nblk * kBlockUnits + g0;
-  const int n = (int)(a.N - g0 < kBlockUnits ? a.N - g0 : kBlockUnits);
+  const int64_t row = u * a.nblk * kBlockUnits + g0 + 8 * lane;
+  const int n = kFull ? kBlockUnits : (int)(a.N - g0);
+  const int i0 = 8 * lane;
   const QBlock qp = q_block(a.pb[wid], 65535.0f), qm = q_block(a.mb[wid], 255.0f), qv = q_block(a.vb[wid], 255.0f);
-  // every load of the lane first (independent, all in flight together)
-  uint32_t cp[kUnitsPerLane], cm[kUnitsPerLane], cv[kUnitsPerLane];
-  float gr[kUnitsPerLane];
+  // codes: rows are padded to whole blocks, so the lane's 8 codes are in
+  // bounds whether or not they are valid units
+  uint32_t wp[4], wm[2], wv[2];
+  if (a.vec_codes) {
+    const uint4 p4 = *reinterpret_cast<const uint4*>(a.pc + row);
+    const uint2 m2 = *reinterpret_cast<const uint2*>(a.mc + row);
+    const uint2 v2 = *reinterpret_cast<const uint2*>(a.vc + row);
+    wp[0] = p4.x; wp[1] = p4.y; wp[2] = p4.z; wp[3] = p4.w;
+    wm[0] = m2.x; wm[1] = m2.y; wv[0] = v2.x; wv[1] = v2.y;
+  } else {
 #pragma unroll
-  for (int k = 0; k < kUnitsPerLane; ++k) {
-    const int i = lane + 32 * k;
-    const bool ok = i < n;
-    cp[k] = ok ? a.pc[row + i] : 0u;
-    cm[k] = ok ? a.mc[row + i] : 0u;
-    cv[k] = ok ? a.vc[row + i] : 0u;
-    gr[k] = ok ? a.grad[u * a.N + g0 + i] : 0.0f;
-  }
-  float np[kUnitsPerLane], my[kUnitsPerLane], vy[kUnitsPerLane];
+    for (int k = 0; k < 4; ++k) wp[k] = (uint32_t)a.pc[row + 2 * k] | ((uint32_t)a.pc[row + 2 * k + 1] << 16);
 #pragma unroll
-  for (int k = 0; k < kUnitsPerLane; ++k) {
-    const int i = lane + 32 * k;
-    np[k] = my[k] = vy[k] = 0.0f;
-    if (i < n) {
-      const float ph = q_decode(cp[k], qp);
-      const float mh = m_from_log(q_decode(cm[k], qm), a.ec);
-      const float vh = v_from_log(q_decode(cv[k], qv), a.ec);
-      const float g = gr[k];
-      const float m1 = __fadd_rn(__fmul_rn(a.b1, mh), __fmul_rn(a.ob1, g));
-      const float v1 = __fadd_rn(__fmul_rn(a.b2, vh), __fmul_rn(a.ob2, __fmul_rn(g, g)));
-      const float num = __fmul_rn(m1, a.c1);
-      const float den = __fadd_rn(__fsqrt_rn(__fmul_rn(v1, a.c2)), a.eps);
-      np[k] = __fsub_rn(ph, __fmul_rn(a.lr, __fdiv_rn(num, den)));
-      my[k] = m_to_log(m1, a.er);
-      vy[k] = v_to_log(v1, a.er);
+    for (int k = 0; k < 2; ++k) {
+      wm[k] = (uint32_t)a.mc[row + 4 * k] | ((uint32_t)a.mc[row + 4 * k + 1] << 8) |
+              ((uint32_t)a.mc[row + 4 * k + 2] << 16) | ((uint32_t)a.mc[row + 4 * k + 3] << 24);
+      wv[k] = (uint32_t)a.vc[row + 4 * k] | ((uint32_t)a.vc[row + 4 * k + 1] << 8) |
+              ((uint32_t)a.vc[row + 4 * k + 2] << 16) | ((uint32_t)a.vc[row + 4 * k + 3] << 24);
     }
   }
-  const float2 nb = warp_bounds(np, lane, n), nm = warp_bounds(my, lane, n), nv = warp_bounds(vy, lane, n);
-  const QBlock q16 = q_block(nb, 65535.0f), qm8 = q_block(nm, 255.0f), qv8 = q_block(nv, 255.0f);
+  const float* gsrc = a.grad + u * a.N + g0 + i0;
+  float gr[8];
+  if (a.vec_grad && (kFull || i0 + 8 <= n)) {
+    const float4 g0v = *reinterpret_cast<const float4*>(gsrc), g1v = *reinterpret_cast<const float4*>(gsrc + 4);
+    gr[0] = g0v.x; gr[1] = g0v.y; gr[2] = g0v.z; gr[3] = g0v.w;
+    gr[4] = g1v.x; gr[5] = g1v.y; gr[6] = g1v.z; gr[7] = g1v.w;
+  } else {
 #pragma unroll
-  for (int k = 0; k < kUnitsPerLane; ++k) {
-    const int i = lane + 32 * k;
-    const bool ok = i < n;
-    a.pc[row + i] = (uint16_t)(ok ? q_encode(np[k], q16, 65535.0f) : 0u);
-    a.mc[row + i] = (uint8_t)(ok ? q_encode(my[k], qm8, 255.0f) : 0u);
-    a.vc[row + i] = (uint8_t)(ok ? q_encode(vy[k], qv8, 255.0f) : 0u);
+    for (int k = 0; k < 8; ++k) gr[k] = (kFull || i0 + k < n) ? gsrc[k] : 0.0f;
+  }
+  float np[8], my[8], vy[8];
+  float plo = inf_f(), phi = -inf_f(), mlo = inf_f(), mhi = -inf_f(), vlo = inf_f(), vhi = -inf_f();
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float ph = q_decode_f(code_u16(wp[k >> 1], k & 1), qp);
+    const float mh = m_from_log(q_decode_f(code_u8(wm[k >> 2], k & 3), qm), a.ec);
+    const float vh = v_from_log(q_decode_f(code_u8(wv[k >> 2], k & 3), qv), a.ec);
+    const float g = gr[k];
+    const float m1 = __fadd_rn(__fmul_rn(a.b1, mh), __fmul_rn(a.ob1, g));
+    const float v1 = __fadd_rn(__fmul_rn(a.b2, vh), __fmul_rn(a.ob2, __fmul_rn(g, g)));
+    const float num = __fmul_rn(m1, a.c1);
+    const float den = __fadd_rn(__fsqrt_rn(__fmul_rn(v1, a.c2)), a.eps);
+    np[k] = __fsub_rn(ph, __fmul_rn(a.lr, __fdiv_rn(num, den)));
+    my[k] = m_to_log(m1, a.er);
+    vy[k] = v_to_log(v1, a.er);
+    if (kFull || i0 + k < n) {
+      plo = fminf(plo, np[k]); phi = fmaxf(phi, np[k]);
+      mlo = fminf(mlo, my[k]); mhi = fmaxf(mhi, my[k]);
+      vlo = fminf(vlo, vy[k]); vhi = fmaxf(vhi, vy[k]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    plo = fminf(plo, __shfl_xor_sync(0xffffffffu, plo, o));
+    phi = fmaxf(phi, __shfl_xor_sync(0xffffffffu, phi, o));
+    mlo = fminf(mlo, __shfl_xor_sync(0xffffffffu, mlo, o));
+    mhi = fmaxf(mhi, __shfl_xor_sync(0xffffffffu, mhi, o));
+    vlo = fminf(vlo, __shfl_xor_sync(0xffffffffu, vlo, o));
+    vhi = fmaxf(vhi, __shfl_xor_sync(0xffffffffu, vhi, o));
+  }
+  const float2 nb = make_float2(plo, phi), nm = make_float2(mlo, mhi), nv = make_float2(vlo, vhi);
+  const QBlock q16 = q_block(nb, 65535.0f), qm8 = q_block(nm, 255.0f), qv8 = q_block(nv, 255.0f);
+  uint32_t op[4] = {0u, 0u, 0u, 0u}, om[2] = {0u, 0u}, ov[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (kFull || i0 + k < n) {  // invalid units keep code 0
+      op[k >> 1] |= q_encode_fast(np[k], q16, 65535u) << (16 * (k & 1));
+      om[k >> 2] |= q_encode_fast(my[k], qm8, 255u) << (8 * (k & 3));
+      ov[k >> 2] |= q_encode_fast(vy[k], qv8, 255u) << (8 * (k & 3));
+    }
+  }
+  if (a.vec_codes) {
+    *reinterpret_cast<uint4*>(a.pc + row) = make_uint4(op[0], op[1], op[2], op[3]);
+    *reinterpret_cast<uint2*>(a.mc + row) = make_uint2(om[0], om[1]);
+    *reinterpret_cast<uint2*>(a.vc + row) = make_uint2(ov[0], ov[1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      a.pc[row + k] = (uint16_t)(op[k >> 1] >> (16 * (k & 1)));
+      a.mc[row + k] = (uint8_t)(om[k >> 2] >> (8 * (k & 3)));
+      a.vc[row + k] = (uint8_t)(ov[k >> 2] >> (8 * (k & 3)));
+    }
   }
   if (lane == 0) {
     a.pb[wid] = nb;
     a.mb[wid] = nm;
     a.vb[wid] = nv;
   }
+}
+
+__global__ void __launch_bounds__(256) adam_sh_quant_kernel(AdamArgs a) {
+  const int64_t wid = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (wid >= a.U * a.nblk) return;  // whole warps
+  const int lane = threadIdx.x & 31;
+  if ((wid % a.nblk) * kBlockUnits + kBlockUnits <= a.N)
+    adam_block<true>(a, wid, lane);
+  else
+    adam_block<false>(a, wid, lane);
 }
 
 unsigned warps_grid(int64_t warps) { return (unsigned)((warps + 7) / 8); }
@@ -261,6 +333,9 @@ cudaError_t launch_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16
   a.eps = hp[7];
   a.ec = hp[8];
   a.er = hp[9];
+  a.vec_codes = reinterpret_cast<uintptr_t>(pc) % 16 == 0 && reinterpret_cast<uintptr_t>(mc) % 8 == 0 &&
+                reinterpret_cast<uintptr_t>(vc) % 8 == 0;
+  a.vec_grad = reinterpret_cast<uintptr_t>(grad) % 16 == 0 && N % 4 == 0;
   adam_sh_quant_kernel<<<warps_grid(U * a.nblk), 256, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();

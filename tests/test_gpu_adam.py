@@ -117,3 +117,38 @@ def test_adam_argument_checks():
         gs.gs_quant_encode(t, 1, 16, 12, t, t)  # bits
     with pytest.raises(gs.GsError):
         gs.gs_adam_sh_quant(t, 1, 16, t, t, t, t, t, t, 1e-3, 0.9, 0.999, 1e-15, 1e-15, 0)  # step 0
+
+
+@pytest.mark.parametrize("U,N,off", [(5, 3 * 256 + 100, 1), (3, 512, 3), (4, 1001, 2)])
+def test_adam_unaligned_buffers_take_the_scalar_path(U, N, off):
+    # codes and gradients at odd element offsets into larger buffers: not
+    # 16/8-byte aligned, so the kernel takes its element-wise loads and stores
+    rng = np.random.default_rng(120 + off)
+    x = _planes(rng, U, N)
+    pc, pb = oracle.quant_encode(x, 16)
+    z = np.zeros((U, N), np.float32)
+    mc, mb = oracle.quant_encode(z, 8)
+    vc, vb = oracle.quant_encode(z, 8)
+    st = {"pc": pc, "pb": pb, "mc": mc, "mb": mb, "vc": vc, "vb": vb}
+    g = _gpu_state(st)
+    L = pc.size
+
+    def shifted(t):
+        big = torch.zeros(L + 16, dtype=t.dtype, device="cuda")
+        v = big[off: off + L]
+        v.copy_(t.reshape(-1))
+        return v
+
+    sp, sm, sv = shifted(g["pc"]), shifted(g["mc"]), shifted(g["vc"])
+    assert sp.data_ptr() % 16 and sm.data_ptr() % 8
+    for step in range(1, 4):
+        gr = _grads(rng, U, N)
+        gbig = torch.zeros(U * N + 8, dtype=torch.float32, device="cuda")
+        gt = gbig[off: off + U * N]
+        gt.copy_(torch.from_numpy(gr.reshape(-1)))
+        oracle.adam_sh_quant(gr, st, HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["scale"], step)
+        gs.gs_adam_sh_quant(gt, U, N, sp, g["pb"], sm, g["mb"], sv, g["vb"],
+                            HP["lr"], HP["beta1"], HP["beta2"], HP["eps"], HP["scale"], step)
+        torch.cuda.synchronize()
+        _compare({"pc": sp.view(U, -1), "mc": sm.view(U, -1), "vc": sv.view(U, -1), "pb": g["pb"], "mb": g["mb"],
+                  "vb": g["vb"]}, st, f"step {step}")

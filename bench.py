@@ -2,9 +2,9 @@
 """Benchmark: forward + backward frames/s of the tile rasterizer.
 
 Workload (default): 1M Gaussians, SH degree 3, 1920x1080, four camera poses
-per step; each pose runs the whole path through the C ABI -- cull (gates off),
-preprocess, bin/sort, rasterize forward, rasterize backward (2-D part and
-parameter part). Inputs are synthetic and resident in HBM before timing; the
+per step; each pose runs the whole path through the C ABI -- preprocess,
+bin/sort, tile order, rasterize forward, rasterize backward (2-D part and
+parameter part); both cull gates are off, so no cull runs. Inputs are synthetic and resident in HBM before timing; the
 236 MB parameter set is larger than the 126 MB L2, so no flush is needed.
 
 Prints one JSON line on rank 0. Under torchrun (N > 1) each rank renders its

@@ -194,31 +194,31 @@ GS_API int gs_tile_order(const uint32_t* tile_ranges, int64_t n_tiles, uint32_t*
 
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,
                             const uint32_t* tile_order, const gs_camera* cam, const float* bg, float* image, float* final_T,
-                            int32_t* n_contrib, int32_t* last, void* stream) {
+                            int32_t* n_contrib, int32_t* last, uint8_t* hit_bits, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last)
     return GS_ERR_INVALID_ARGUMENT;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
-                                       n_contrib, last, nullptr, nullptr, tile_order,
+                                       n_contrib, last, nullptr, nullptr, tile_order, hit_bits,
                                        static_cast<cudaStream_t>(stream)));
 }
 
 GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* vals, const uint32_t* tile_ranges,
                                        const uint32_t* tile_order, const gs_camera* cam, const float* bg, const int32_t* active_idx,
                                        float* image, float* final_T, int32_t* n_contrib, int32_t* last,
-                                       float* importance, void* stream) {
+                                       float* importance, uint8_t* hit_bits, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last ||
       !importance)
     return GS_ERR_INVALID_ARGUMENT;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
-                                       n_contrib, last, importance, active_idx, tile_order,
+                                       n_contrib, last, importance, active_idx, tile_order, hit_bits,
                                        static_cast<cudaStream_t>(stream)));
 }
 
 GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,
-                               const uint32_t* tile_ranges, const uint32_t* tile_order, const gs_camera* cam,
-                               const float* bg, const float* final_T, const int32_t* last,
+                               const uint32_t* tile_ranges, const uint32_t* tile_order, const uint8_t* hit_bits,
+                               const gs_camera* cam, const float* bg, const float* final_T, const int32_t* last,
                                const float* dL_dimage, float* grad2d, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || n_records < 0 || n_records >= (int64_t(1) << 31) || !tile_ranges ||
       !bg || !final_T || !last || !dL_dimage || (n_records > 0 && !grad2d))
@@ -226,7 +226,7 @@ GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const 
   if (n_records == 0) return GS_OK;
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_bwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, final_T, last,
-                                       dL_dimage, reinterpret_cast<float4*>(grad2d), n_records, tile_order,
+                                       dL_dimage, reinterpret_cast<float4*>(grad2d), n_records, tile_order, hit_bits,
                                        static_cast<cudaStream_t>(stream)));
 }
 
@@ -344,7 +344,8 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
                             const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                             const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
                             const gs_camera* cam, const gs_projected* in, const uint32_t* vals,
-                            const uint32_t* tile_ranges, const uint32_t* tile_order, const float* bg,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order, const uint8_t* hit_bits,
+                            const float* bg,
                             const float* final_T, const int32_t* last, const float* dL_dimage,
                             float* grad2d, float* d_means,
                             float* d_log_scales, float* d_quats, float* d_opacity_logits, float* d_sh,
@@ -362,7 +363,7 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
   const float b[3] = {bg[0], bg[1], bg[2]};
   if (N > 0) {
     cudaError_t e = launch_raster_bwd(rec, vals, tile_ranges, dc, b, final_T, last, dL_dimage,
-                                      reinterpret_cast<float4*>(grad2d), N, tile_order, s);
+                                      reinterpret_cast<float4*>(grad2d), N, tile_order, hit_bits, s);
     if (e != cudaSuccess) return GS_ERR_CUDA;
   }
   Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};

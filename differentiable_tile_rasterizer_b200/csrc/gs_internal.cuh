@@ -154,13 +154,13 @@ cudaError_t launch_publish(void* ws, const BinSortPlan& plan, int64_t* result, c
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], float* image, float* final_T,
                               int32_t* n_contrib, int32_t* last, float* importance, const int32_t* active_idx,
-                              const uint32_t* order, cudaStream_t s);
+                              const uint32_t* order, uint8_t* hits, cudaStream_t s);
 // Tiles by descending log2 of their list length (order [TT]); the raster
 // launches take their CTAs' tiles in this order (order == nullptr: tile b).
 cudaError_t launch_tile_order(const uint32_t* ranges, int64_t TT, uint32_t* order, cudaStream_t s);
 cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], const float* final_T,
                               const int32_t* last, const float* dL_dimage, float4* grad2d,
-                              int64_t n_records, const uint32_t* order, cudaStream_t s);
+                              int64_t n_records, const uint32_t* order, const uint8_t* hits, cudaStream_t s);
 
 }  // namespace gs

@@ -163,6 +163,7 @@ struct FwdArgs {
   int32_t* last;
   float* importance;           // kImp: [N] += sum over pixels of alpha * T
   const int32_t* active_idx;   // record -> Gaussian, or null (identity)
+  uint8_t* hits;               // [entries] or null: bit w = warp w's block can blend the entry
 };
 
 // kImp also accumulates each Gaussian's importance weight (the sum over the
@@ -177,6 +178,9 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   __shared__ float4 s_box[kBatchF];  // blend region of each staged entry
   __shared__ float4 s_q1[kBatchF];
   __shared__ float4 s_q2[kBatchF];
+  // per batch parity: warp w's region ballot of chunk c (0 for chunks the
+  // warp did not test: its pixels had all stopped)
+  __shared__ uint32_t s_wm[2][kBlock / 32][kBatchF / 32];
   const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
   if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
   const int tile = (int)tile_u;
@@ -206,11 +210,25 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
       have_staged = false;
     }
   };
+  // hit byte of the entry this thread staged in the batch at `hbase`, from
+  // the eight warps' ballots of parity `par`
+  auto write_hits = [&](int hbase, int par) {
+    if (a.hits && hbase >= 0 && hbase + tid < n) {
+      uint32_t h = 0;
+#pragma unroll
+      for (int w = 0; w < kBlock / 32; ++w) h |= ((s_wm[par][w][tid >> 5] >> lane) & 1u) << w;
+      a.hits[range.x + hbase + tid] = (uint8_t)h;
+    }
+  };
   // (The forward stages with plain gathers: with five CTAs per SM the
   // others cover a staging CTA's latency.)
-  for (int base = 0; base < n; base += kBatchF) {
+  int par = 0, last_staged = -1;
+  for (int base = 0; base < n; base += kBatchF, par ^= 1) {
     if (__syncthreads_count(done) == kBlock) break;
     flush();  // the previous batch's sums are complete (barrier above)
+    write_hits(base - kBatchF, par ^ 1);  // and its ballots
+    last_staged = base;
+    if (a.hits && tid < (kBlock / 32) * (kBatchF / 32)) (&s_wm[par][0][0])[tid] = 0u;
     if (base + tid < n) {
       const int e = tid;
       const uint32_t i = a.vals[range.x + base + e];
@@ -237,6 +255,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
       const int j = c0 + lane;
       const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy, 3.5f, 1.5f);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
+      if (a.hits && lane == 0) s_wm[par][warp][c0 >> 5] = msk;
       // Entries are taken two at a time: their alphas at this pixel run as
       // one packed pair (each half rounded as the scalar operation), then
       // they blend in list order. Branch-free blend: a lane that skips an
@@ -282,9 +301,10 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
       }
     }
   }
-  if (kImp) {
+  if (kImp || a.hits) {
     __syncthreads();
     flush();
+    write_hits(last_staged, (last_staged / kBatchF) & 1);  // the last staged batch
   }
   if (inside) {
     const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
@@ -310,6 +330,7 @@ struct BwdArgs {
   const int32_t* last;
   const float* dL_dimage;
   float4* grad2d;  // [n][3]
+  const uint8_t* hits;  // [entries] from the forward, or null
 };
 
 // Where the multi-value butterfly below leaves its results: lane `lane` ends
@@ -565,19 +586,160 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
   cp_async_wait_all();  // no copy outlives the CTA
 }
 
+// cp.async groups: wait until at most one (the newest) is still in flight.
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// Backward with the forward's hit bytes: warp w (the 8x8 block of forward
+// warps f and f + 2, f = (w & 1) | (w >> 1) << 2) walks its own list
+// entries back to front from the last blend of its pixels, 32 per chunk
+// (lane l: offset warp_last - 1 - 32 c - l). Only the entries whose byte has
+// bit f or f + 2 set are fetched: by cp.async into the warp's own
+// double-buffered slots, one chunk ahead. The warps of a CTA share no data
+// and never wait for each other. Per pixel the operations, and the entries
+// that blend, are those of raster_bwd_kernel, so every pixel's terms are
+// the same values; the warp sums go to the global gradient rows directly.
+__global__ void __launch_bounds__(kBlockB, 8) raster_bwd_hits_kernel(BwdArgs a) {
+  constexpr int kWarps = kBlockB / 32;
+  __shared__ float4 s_raw[kWarps][2][3][32];  // xyzo, conic, rgb of the hit entries of two chunks
+  __shared__ float s_acc[kWarps][32][9];      // the chunk's warp sums ([slot][value])
+  const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
+  if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
+  const int tile = (int)tile_u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
+  const int u = tx0 + (warp & 1) * 8 + (lane & 7), v = ty0 + (warp >> 1) * 8 + (lane >> 3);
+  const uint2 range = a.ranges[tile];
+  const size_t P = (size_t)a.W * a.H;
+  BwdPair px = load_bwd_pair(a, u, v, P);
+  const int warp_last = __reduce_max_sync(0xffffffffu, max(px.last0, px.last1));
+  if (warp_last == 0) return;  // no pixel of the block blended anything
+  const Reduce9Slot slot = reduce9_slot(lane);
+  const int f = (warp & 1) | ((warp >> 1) << 2);
+  const uint32_t fbits = (1u << f) | (1u << (f + 2));
+  const uint32_t* lv = a.vals + range.x;
+  const uint8_t* hb = a.hits + range.x;
+  float4(*raw)[3][32] = s_raw[warp];
+  float(*acc)[9] = s_acc[warp];
+  // lane's entry of chunk c: its record index and whether the block can blend it
+  auto meta = [&](int c, uint32_t& idx, bool& hit) {
+    const int off = warp_last - 1 - 32 * c - lane;
+    const bool in = off >= 0;
+    const uint32_t b = in ? (uint32_t)hb[off] : 0u;
+    idx = in ? lv[off] : 0u;
+    hit = (b & fbits) != 0u;
+  };
+  auto fetch = [&](int buf, uint32_t idx, bool hit) {
+    if (hit) {
+      cp_async16(&raw[buf][0][lane], a.xyzo + idx);
+      cp_async16(&raw[buf][1][lane], a.conic + idx);
+      cp_async16(&raw[buf][2][lane], a.rgb + idx);
+    }
+    cp_async_commit();
+  };
+  const int nchunks = (warp_last + 31) >> 5;
+  uint32_t i_cur, i_nxt;
+  bool h_cur, h_nxt;
+  meta(0, i_cur, h_cur);
+  fetch(0, i_cur, h_cur);
+  meta(1, i_nxt, h_nxt);
+  for (int c = 0; c < nchunks; ++c) {
+    const int buf = c & 1;
+    fetch(buf ^ 1, i_nxt, h_nxt);  // chunk c + 1 in flight (its buffer was freed after chunk c - 1)
+    const uint32_t i_this = i_cur;
+    const bool h_this = h_cur;
+    i_cur = i_nxt;
+    h_cur = h_nxt;
+    meta(c + 2, i_nxt, h_nxt);
+    cp_async_wait_1();  // this lane's copies of chunk c have landed
+    __syncwarp();       // and every lane's
+    unsigned msk = __ballot_sync(0xffffffffu, h_this);
+    unsigned summed = 0u;
+    while (msk) {
+      const int k = __ffs(msk) - 1;
+      msk &= msk - 1;
+      const int offk = warp_last - 1 - 32 * c - k;
+      const float4 G = raw[buf][0][k];  // px, py, depth, opacity
+      const float4 Q = raw[buf][1][k];  // A, B, C
+      const float a2 = __fmul_rn(Q.x, kHalfNegLog2e), b2 = __fmul_rn(Q.y, kNegLog2e),
+                  c2 = __fmul_rn(Q.z, kHalfNegLog2e);
+      const float dx = __fsub_rn(G.x, px.xc);
+      const float2 dy = sub2(splat2(G.y), px.yc);
+      const float2 qv = fma2(splat2(b2), dy, splat2(__fmul_rn(a2, dx)));
+      float2 p2 = mul2(splat2(dx), qv);
+      p2 = fma2(mul2(splat2(c2), dy), dy, p2);
+      const float2 e = exp2_raster2(p2);
+      const float2 vv = mul2(splat2(G.w), e);
+      const float al0 = fminf(vv.x, kAlphaMax), al1 = fminf(vv.y, kAlphaMax);
+      const bool b0 = offk < px.last0 && al0 >= kAlphaMin, b1 = offk < px.last1 && al1 >= kAlphaMin;
+      if (!__any_sync(0xffffffffu, b0 || b1)) continue;
+      const float2 ab = make_float2(b0 ? al0 : 0.0f, b1 ? al1 : 0.0f);
+      const float2 oma = sub2(splat2(1.0f), ab);
+      px.T = make_float2(b0 ? __fdividef(px.T.x, oma.x) : px.T.x, b1 ? __fdividef(px.T.y, oma.y) : px.T.y);
+      const float2 wgt = mul2(ab, px.T);
+      const float4 cc = raw[buf][2][k];  // r, g, b
+      float2 sg = mul2(px.g0, sub2(splat2(cc.x), px.R0));
+      sg = fma2(px.g1, sub2(splat2(cc.y), px.R1), sg);
+      sg = fma2(px.g2, sub2(splat2(cc.z), px.R2), sg);
+      const float2 Gk = mul2(px.T, sg);
+      const float2 Gm = make_float2((b0 && vv.x < kAlphaMax) ? Gk.x : 0.0f, (b1 && vv.y < kAlphaMax) ? Gk.y : 0.0f);
+      const float2 dp = mul2(Gm, ab);
+      const float2 dpdy = mul2(dp, dy);
+      const float2 dpdy2 = mul2(dpdy, dy);
+      const float2 ge = mul2(Gm, e);
+      const float2 w0 = mul2(px.g0, wgt), w1 = mul2(px.g1, wgt), w2 = mul2(px.g2, wgt);
+      const float sdp = dp.x + dp.y, sdpdy = dpdy.x + dpdy.y;
+      const float A = Q.x, B = Q.y, Cc = Q.z, dxs = dx * sdp;
+      float gv[9];
+      gv[0] = -fmaf(A, dxs, B * sdpdy);
+      gv[1] = -fmaf(B, dxs, Cc * sdpdy);
+      gv[2] = ge.x + ge.y;
+      gv[3] = -0.5f * dx * dxs;
+      gv[4] = -dx * sdpdy;
+      gv[5] = -0.5f * (dpdy2.x + dpdy2.y);
+      gv[6] = w0.x + w0.y;
+      gv[7] = w1.x + w1.y;
+      gv[8] = w2.x + w2.y;
+      px.R0 = fma2(splat2(cc.x), ab, mul2(oma, px.R0));
+      px.R1 = fma2(splat2(cc.y), ab, mul2(oma, px.R1));
+      px.R2 = fma2(splat2(cc.z), ab, mul2(oma, px.R2));
+      const float tot = warp_reduce9(gv, lane);
+      if (slot.owner) acc[k][slot.idx] = tot;
+      summed |= 1u << k;
+    }
+    __syncwarp();
+    if ((summed >> lane) & 1u) {
+      float r[9];
+      bool any = false;
+#pragma unroll
+      for (int j = 0; j < 9; ++j) {
+        r[j] = acc[lane][j];
+        any |= r[j] != 0.0f;
+      }
+      if (any) {
+        float4* dst = a.grad2d + 3 * (size_t)i_this;
+        atomicAdd(dst, make_float4(r[0], r[1], r[2], 0.f));
+        atomicAdd(dst + 1, make_float4(r[3], r[4], r[5], 0.f));
+        atomicAdd(dst + 2, make_float4(r[6], r[7], r[8], 0.f));
+      }
+    }
+    __syncwarp();  // the chunk's slots and sums are free again
+  }
+  cp_async_wait_all();  // no copy outlives the warp
+}
+
 }  // namespace
 
 cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], float* image, float* final_T,
                               int32_t* n_contrib, int32_t* last, float* importance, const int32_t* active_idx,
-                              const uint32_t* order, cudaStream_t s) {
+                              const uint32_t* order, uint8_t* hits, cudaStream_t s) {
   FwdArgs a;
   a.xyzo = rec.xyzo; a.conic = rec.conic; a.rgb = rec.rgb;
   a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges); a.order = order;
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.image = image; a.final_T = final_T; a.n_contrib = n_contrib; a.last = last;
-  a.importance = importance; a.active_idx = active_idx;
+  a.importance = importance; a.active_idx = active_idx; a.hits = hits;
   if (importance)
     raster_fwd_kernel<true><<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
   else
@@ -589,7 +751,7 @@ cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const ui
 cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const uint32_t* ranges,
                               const DevCam& cam, const float bg[3], const float* final_T,
                               const int32_t* last, const float* dL_dimage, float4* grad2d,
-                              int64_t n_records, const uint32_t* order, cudaStream_t s) {
+                              int64_t n_records, const uint32_t* order, const uint8_t* hits, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(grad2d, 0, (size_t)n_records * 3 * sizeof(float4), s);
   if (e != cudaSuccess) return e;
   BwdArgs a;
@@ -597,8 +759,11 @@ cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const ui
   a.vals = vals; a.ranges = reinterpret_cast<const uint2*>(ranges); a.order = order;
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
-  a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d;
-  raster_bwd_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
+  a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d; a.hits = hits;
+  if (hits)
+    raster_bwd_hits_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
+  else
+    raster_bwd_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
   count_launches(1);
   return cudaGetLastError();
 }

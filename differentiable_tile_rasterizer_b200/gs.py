@@ -101,13 +101,13 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_bin_sort.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, PI64, P, PSZ, P]
         L.gs_bin_sort_async.argtypes = [PPROJ, I64, PCAM, P, P, P, I64, P, P, P, PSZ, P]
         L.gs_tile_order.argtypes = [P, I64, P, P]
-        L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, P, PCAM, P, P, P, P, P, P]
-        L.gs_rasterize_fwd_importance.argtypes = [PPROJ, P, P, P, PCAM, P, P, P, P, P, P, P, P]
-        L.gs_rasterize_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P, P, P, P,
+        L.gs_rasterize_fwd.argtypes = [PPROJ, P, P, P, PCAM, P, P, P, P, P, P, P]
+        L.gs_rasterize_fwd_importance.argtypes = [PPROJ, P, P, P, PCAM, P, P, P, P, P, P, P, P, P]
+        L.gs_rasterize_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P, P, P, P, P,
                                        P, P, P, P, P, P, P, P, P, P]
         L.gs_preprocess_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P,
                                         P, P, P, P, P, P]
-        L.gs_rasterize_bwd_2d.argtypes = [PPROJ, I64, P, P, P, PCAM, P, P, P, P, P, P]
+        L.gs_rasterize_bwd_2d.argtypes = [PPROJ, I64, P, P, P, P, PCAM, P, P, P, P, P, P]
         L.gs_cull_noalloc.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P]
         L.gs_cull_noalloc.restype = ctypes.c_int
         L.gs_debug_kernel_launches.restype = ctypes.c_int64
@@ -298,38 +298,39 @@ def gs_tile_order(tile_ranges, n_tiles, order, stream=None):
 
 
 def gs_rasterize_fwd(rec: GsProjected, vals, tile_ranges, cam: GsCamera, bg, image, final_T,
-                     n_contrib, last, stream=None, tile_order=None):
+                     n_contrib, last, stream=None, tile_order=None, hit_bits=None):
     bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
     _check("gs_rasterize_fwd", load().gs_rasterize_fwd(
         ctypes.byref(rec), _p(vals), _p(tile_ranges), _p(tile_order), ctypes.byref(cam), ctypes.cast(bgv, P),
-        _p(image), _p(final_T), _p(n_contrib), _p(last), _stream(stream)))
+        _p(image), _p(final_T), _p(n_contrib), _p(last), _p(hit_bits), _stream(stream)))
 
 
 def gs_rasterize_fwd_importance(rec: GsProjected, vals, tile_ranges, cam: GsCamera, bg, active_idx, image,
-                                final_T, n_contrib, last, importance, stream=None, tile_order=None):
+                                final_T, n_contrib, last, importance, stream=None, tile_order=None, hit_bits=None):
     bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
     _check("gs_rasterize_fwd_importance", load().gs_rasterize_fwd_importance(
         ctypes.byref(rec), _p(vals), _p(tile_ranges), _p(tile_order), ctypes.byref(cam), ctypes.cast(bgv, P), _p(active_idx),
-        _p(image), _p(final_T), _p(n_contrib), _p(last), _p(importance), _stream(stream)))
+        _p(image), _p(final_T), _p(n_contrib), _p(last), _p(importance), _p(hit_bits), _stream(stream)))
 
 
 def gs_rasterize_bwd(means, log_scales, quats, opacity_logits, sh, sh_degree, N, active_idx, n_active,
                      mask, cam: GsCamera, rec: GsProjected, vals, tile_ranges, bg, final_T, last,
                      dL_dimage, grad2d, d_means, d_log_scales, d_quats, d_opacity_logits, d_sh,
-                     stream=None, tile_order=None):
+                     stream=None, tile_order=None, hit_bits=None):
     bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
     _check("gs_rasterize_bwd", load().gs_rasterize_bwd(
         _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
         _p(active_idx), _p(n_active), _p(mask), ctypes.byref(cam), ctypes.byref(rec), _p(vals),
-        _p(tile_ranges), _p(tile_order), ctypes.cast(bgv, P), _p(final_T), _p(last), _p(dL_dimage),
+        _p(tile_ranges), _p(tile_order), _p(hit_bits), ctypes.cast(bgv, P), _p(final_T), _p(last), _p(dL_dimage),
         _p(grad2d), _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
 
 
 def gs_rasterize_bwd_2d(rec: GsProjected, n_records, vals, tile_ranges, cam: GsCamera, bg, final_T, last,
-                        dL_dimage, grad2d, stream=None, tile_order=None):
+                        dL_dimage, grad2d, stream=None, tile_order=None, hit_bits=None):
     bgv = (ctypes.c_float * 3)(*[float(b) for b in bg])
     _check("gs_rasterize_bwd_2d", load().gs_rasterize_bwd_2d(
-        ctypes.byref(rec), int(n_records), _p(vals), _p(tile_ranges), _p(tile_order), ctypes.byref(cam),
+        ctypes.byref(rec), int(n_records), _p(vals), _p(tile_ranges), _p(tile_order), _p(hit_bits),
+        ctypes.byref(cam),
         ctypes.cast(bgv, P), _p(final_T), _p(last), _p(dL_dimage), _p(grad2d), _stream(stream)))
 
 

@@ -113,7 +113,7 @@ class InterleavedRank:
         back with the received counts as the splits)."""
         B = self.band
         gs.gs_rasterize_bwd_2d(B._proj, B.N, B.vals, B.ranges, B.cam, B.bg, B.final_T, B.last, dL_dimage,
-                               B.grad2d, tile_order=B._order())
+                               B.grad2d, tile_order=B._order(), hit_bits=B._hits_in())
         back = torch.empty((max(self.n_recv, 1), 12), dtype=torch.float32, device=self.dev)
         gs.gs_unmerge_grad2d(B.grad2d, self.perm, self.n_recv, back)
         return back[: self.n_recv], self.recv_counts

@@ -79,7 +79,8 @@ def _u8(n, dev):
 class Rasterizer:
     """Buffers and calls for rendering one view of N Gaussians at W x H.
 
-    forward() runs cull -> preprocess -> bin_sort -> rasterize_fwd and keeps
+    forward() runs cull (when a gate is on) -> preprocess -> bin_sort ->
+    tile_order -> rasterize_fwd and keeps
     what backward() needs; backward() runs rasterize_bwd. Buffers are
     allocated once (the instance capacity grows when gs_bin_sort reports it
     is too small) and reused across calls.
@@ -112,6 +113,11 @@ class Rasterizer:
         # sort and given to the raster launches; None: CTA b takes tile b.
         self.schedule_tiles = True
         self.tile_order = torch.arange(max(self.TT, 1), **i32)
+        # The forward writes one byte per list entry with the pixel blocks it
+        # may blend in, and the backward walks only those (gs_rasterize_fwd's
+        # hit_bits). False: the backward tests every entry itself.
+        self.use_hit_bits = True
+        self._hits_fresh = False  # hit_bits hold the current lists' bytes
         self.grad2d = torch.empty((n, 12), **f32)
         self.grads = {"means": torch.empty((3, n), **f32), "log_scales": torch.empty((3, n), **f32),
                       "quats": torch.empty((4, n), **f32), "opacity_logits": torch.empty(n, **f32),
@@ -152,6 +158,7 @@ class Rasterizer:
         cap = int(cap)
         self.keys = torch.empty(max(cap, 1), dtype=torch.int64, device=self.dev)
         self.vals = torch.empty(max(cap, 1), dtype=torch.int32, device=self.dev)
+        self.hit_bits = torch.empty(max(cap, 1), dtype=torch.uint8, device=self.dev)
         probe = gs.GsCamera()
         probe.width, probe.height = self.W, self.H
         self.sort_ws = _u8(gs.gs_bin_sort_workspace(self.N, probe, cap), self.dev)
@@ -163,6 +170,15 @@ class Rasterizer:
             gs.gs_cull(params.means, params.importance if importance_q > 0 else None, self.N, cam,
                        lod_dist, importance_q, self.mask, self.active_idx, self.n_active, self.cull_ws)
         self.culled = True
+
+    def _gate(self, params: GaussianParams, cam: gs.GsCamera, lod_dist, importance_q):
+        """The cull of forward(): with both gates off every Gaussian is active
+        and its active list would be the identity, so the records are
+        indexed by Gaussian directly and no cull runs."""
+        if lod_dist > 0 or importance_q > 0:
+            self.cull(params, cam, lod_dist, importance_q)
+        else:
+            self.culled = False
 
     def preprocess(self, params: GaussianParams, cam: gs.GsCamera):
         act = self.active_idx if self.culled else None
@@ -178,8 +194,21 @@ class Rasterizer:
     def _order(self):
         return self.tile_order if self.schedule_tiles else None
 
+    def _hits(self):
+        """hit_bits for a forward (which writes them)."""
+        if not self.use_hit_bits:
+            return None
+        self._hits_fresh = True
+        return self.hit_bits
+
+    def _hits_in(self):
+        """hit_bits for a backward: only when a forward wrote them for the
+        current lists."""
+        return self.hit_bits if self.use_hit_bits and self._hits_fresh else None
+
     def _bin_sort(self, cam: gs.GsCamera):
         offs = self.offsets if self.want_offsets else None
+        self._hits_fresh = False
         if self.deferred:
             if self._n_pending == self._results.shape[0]:
                 self.check()
@@ -211,13 +240,14 @@ class Rasterizer:
         if importance.dtype != torch.float32 or importance.numel() != self.N or not importance.is_cuda:
             raise ValueError("importance must be a float32 CUDA tensor of N elements")
         self.params, self.cam, self.bg = params, c, tuple(float(b) for b in bg)
-        self.cull(params, c, lod_dist, importance_q)
+        self._gate(params, c, lod_dist, importance_q)
         self.preprocess(params, c)
         self.bin_sort(c)
         with self._timed("raster_fwd_importance"):
-            gs.gs_rasterize_fwd_importance(self._proj, self.vals, self.ranges, c, self.bg, self.active_idx,
+            gs.gs_rasterize_fwd_importance(self._proj, self.vals, self.ranges, c, self.bg,
+                                           self.active_idx if self.culled else None,
                                            self.image, self.final_T, self.n_contrib, self.last, importance,
-                                           tile_order=self._order())
+                                           tile_order=self._order(), hit_bits=self._hits())
         return self.image
 
     def accumulate_grad_stats(self, norm_sum: torch.Tensor, view_count: torch.Tensor):
@@ -249,7 +279,7 @@ class Rasterizer:
     def raster_fwd(self, cam: gs.GsCamera, bg):
         with self._timed("raster_fwd"):
             gs.gs_rasterize_fwd(self._proj, self.vals, self.ranges, cam, bg, self.image, self.final_T,
-                                self.n_contrib, self.last, tile_order=self._order())
+                                self.n_contrib, self.last, tile_order=self._order(), hit_bits=self._hits())
 
     # ------------------------------------------------------------------ public
     def forward(self, params: GaussianParams, cam, bg=(0.0, 0.0, 0.0), lod_dist=0.0,
@@ -258,7 +288,7 @@ class Rasterizer:
         if (c.width, c.height) != (self.W, self.H):
             raise ValueError("camera size differs from the rasterizer's")
         self.params, self.cam, self.bg = params, c, tuple(float(b) for b in bg)
-        self.cull(params, c, lod_dist, importance_q)
+        self._gate(params, c, lod_dist, importance_q)
         self.preprocess(params, c)
         self.bin_sort(c)
         self.raster_fwd(c, self.bg)
@@ -275,12 +305,13 @@ class Rasterizer:
                                 self.N, act, na, mask, c, self._proj, self.vals, self.ranges, self.bg,
                                 self.final_T, self.last, dL_dimage, self.grad2d, g["means"],
                                 g["log_scales"], g["quats"], g["opacity_logits"], g["sh"],
-                                tile_order=self._order())
+                                tile_order=self._order(), hit_bits=self._hits_in())
             return g
         # the same two parts as separate calls, so each can be timed
         with self._timed("raster_bwd"):
             gs.gs_rasterize_bwd_2d(self._proj, self.N, self.vals, self.ranges, c, self.bg, self.final_T,
-                                   self.last, dL_dimage, self.grad2d, tile_order=self._order())
+                                   self.last, dL_dimage, self.grad2d, tile_order=self._order(),
+                                   hit_bits=self._hits_in())
         with self._timed("preprocess_bwd"):
             gs.gs_preprocess_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
                                  self.N, act, na, mask, c, self._proj, self.grad2d, g["means"],
@@ -352,7 +383,7 @@ class MultiViewRenderer:
                 R._bin_sort(c)
             with self._timed("raster_fwd"):
                 gs.gs_rasterize_fwd(R._proj, R.vals, R.ranges, c, bg, R.image, R.final_T, R.n_contrib, R.last,
-                                    tile_order=R._order())
+                                    tile_order=R._order(), hit_bits=R._hits())
         return [R.image for R in self.views]
 
     def set_deferred(self, on: bool):

@@ -373,12 +373,21 @@ GS_API int gs_tile_order(const uint32_t* tile_ranges, int64_t n_tiles, uint32_t*
  *   final_T      [device] [H][W] out
  *   n_contrib    [device] [H][W] i32 out: blended Gaussians
  *   last         [device] [H][W] i32 out: 1 + list offset of the last blend
+ *   hit_bits     [device] [n_instances] u8 out, or NULL: one byte per sorted
+ *                list entry (indexed as vals); bit f set when the entry may
+ *                blend in the 8x4 pixel block f of its tile (block f at
+ *                column (f & 1) * 8, row (f >> 1) * 4), clear when it cannot
+ *                blend there or when the block's pixels had all stopped
+ *                before it. The backward's input of the same name. Written
+ *                at least for every entry up to each tile's last blend;
+ *                entries after the point where all of a tile's pixels
+ *                stopped may be left as they were.
  * Asynchronous. */
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
                             const uint32_t* tile_ranges, const uint32_t* tile_order,
                             const gs_camera* cam, const float* bg,
                             float* image, float* final_T, int32_t* n_contrib, int32_t* last,
-                            void* stream);
+                            uint8_t* hit_bits, void* stream);
 
 /* Importance pass: gs_rasterize_fwd plus the cross-view visibility weight
  * of every Gaussian (BlitzGS write-up, section 2.2 "模型层级重要性评分传递":
@@ -387,8 +396,8 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
  * view-level importance cull of gs_cull). The page prints no formula. It is
  * read as the sum over the view's pixels of the blend weight alpha * T of
  * each of the Gaussian's blends, with the forward's own fp32 values. The
- * image outputs equal gs_rasterize_fwd's bit for bit. tile_order as for
- * gs_rasterize_fwd.
+ * image outputs equal gs_rasterize_fwd's bit for bit. tile_order and
+ * hit_bits as for gs_rasterize_fwd.
  *   active_idx   [device] [n_records] i32 or NULL: Gaussian of record i
  *                (from gs_cull; NULL: record i is Gaussian i)
  *   importance   [device] [N] f32 in/out: this view's weights are ADDED, so
@@ -399,7 +408,8 @@ GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* v
                                        const uint32_t* tile_ranges, const uint32_t* tile_order,
                                        const gs_camera* cam, const float* bg,
                                        const int32_t* active_idx, float* image, float* final_T,
-                                       int32_t* n_contrib, int32_t* last, float* importance, void* stream);
+                                       int32_t* n_contrib, int32_t* last, float* importance,
+                                       uint8_t* hit_bits, void* stream);
 
 /* Backward pass: exact derivatives of the forward with every discrete decision
  * held fixed (visibility, tile lists, skips, the 0.99 clamp -- zero gradient
@@ -410,6 +420,12 @@ GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* v
  *   mask         [device] [N] u8 from gs_cull or NULL (all active)
  *   in           records from gs_preprocess
  *   tile_order   as for gs_rasterize_fwd (any permutation, or NULL)
+ *   hit_bits     [device] the forward's hit_bits for the same lists, or NULL.
+ *                Given, each warp walks its own 8x8 block's entries and
+ *                fetches only those with its blocks' bits set, with no
+ *                CTA-wide barrier; NULL, the kernel tests every entry's
+ *                blend region itself. The results are the same either way
+ *                up to the order of the fp32 atomic sums.
  *   final_T, last from gs_rasterize_fwd; dL_dimage [device] [3][H][W]
  *   grad2d       [device] [N][12] f32 out: (dpx, dpy, dopacity, 0,
  *                dA, dB, dC, 0, dr, dg, db, 0) per record
@@ -420,7 +436,8 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
                             const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                             const int32_t* active_idx, const int32_t* n_active, const uint8_t* mask,
                             const gs_camera* cam, const gs_projected* in, const uint32_t* vals,
-                            const uint32_t* tile_ranges, const uint32_t* tile_order, const float* bg,
+                            const uint32_t* tile_ranges, const uint32_t* tile_order,
+                            const uint8_t* hit_bits, const float* bg,
                             const float* final_T, const int32_t* last, const float* dL_dimage,
                             float* grad2d, float* d_means, float* d_log_scales, float* d_quats,
                             float* d_opacity_logits, float* d_sh, void* stream);
@@ -431,7 +448,7 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
  * of gs_rasterize_bwd; n_records = N. Asynchronous. */
 GS_API int gs_rasterize_bwd_2d(const gs_projected* in, int64_t n_records, const uint32_t* vals,
                                const uint32_t* tile_ranges, const uint32_t* tile_order,
-                               const gs_camera* cam, const float* bg,
+                               const uint8_t* hit_bits, const gs_camera* cam, const float* bg,
                                const float* final_T, const int32_t* last, const float* dL_dimage,
                                float* grad2d, void* stream);
 

@@ -10,7 +10,7 @@ import torch
 import oracle
 from differentiable_tile_rasterizer_b200 import gs, synthetic as S
 from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, Rasterizer
-from tests.gpu_helpers import assert_bits, gpu_forward
+from tests.gpu_helpers import assert_bits, gpu_forward, grad_tol_check
 
 pytestmark = pytest.mark.gpu
 
@@ -62,9 +62,16 @@ def test_deferred_views_match_checked_views():
         assert counts[p] == Rs.n_instances
         assert_bits(out[p][0].cpu().numpy(), Rs.image.cpu().numpy(), f"image {p}")
         assert_bits(out[p][1].cpu().numpy(), Rs.final_T.cpu().numpy(), f"T {p}")
+        # same kernels on the same inputs; only the order of the fp32 atomic
+        # sums differs, so both runs are held to the oracle's gradients with
+        # the suite's tolerance (relative plus a floor from the summed magnitudes)
+        sub = S.Scene(sc.name, sc.N, sc.sh_degree, sc.means, sc.log_scales, sc.quats, sc.opacity_logits, sc.sh,
+                      [sc.cameras[p]], sc.bg, True)
+        ref = oracle.render(sub)
+        ob = oracle.backward(sub, sub.cameras[0], ref["rec"], ref["bins"], sc.grad_image(p))
         for k, v in Rs.grads.items():
-            # same kernels on the same inputs; only the order of float atomics differs
-            np.testing.assert_allclose(out[p][2][k].cpu().numpy(), v.cpu().numpy(), rtol=1e-4, atol=1e-6)
+            grad_tol_check(out[p][2][k].cpu().numpy(), ob["d_" + k], ob["m_" + k], what=f"deferred {k} {p}")
+            grad_tol_check(v.cpu().numpy(), ob["d_" + k], ob["m_" + k], what=f"checked {k} {p}")
 
 
 def test_deferred_capacity_failure_leaves_tiles_empty_then_recovers():

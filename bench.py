@@ -53,6 +53,9 @@ def _peaks():
 RASTER_SOURCES = ("differentiable_tile_rasterizer_b200/csrc/raster.cu",
                   "differentiable_tile_rasterizer_b200/csrc/gs_device.cuh")
 TRAFFIC_PROFILE = "profiles/raster_kernels_1m_1080p_sh3.md"
+# the kernel each timed raster stage launches (the backward walks the
+# forward's hit bytes)
+KERNEL_OF_STAGE = {"raster_fwd": "raster_fwd_kernel", "raster_bwd": "raster_bwd_hits_kernel"}
 
 
 def raster_source_hash() -> str:
@@ -63,19 +66,20 @@ def raster_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` (dram__bytes_read.sum +
+def profiled_traffic(stage: str):
+    """DRAM bytes per launch of the kernel of `stage` (dram__bytes_read.sum +
     dram__bytes_write.sum, averaged over the captured launches) from the
     committed ncu summary, or None when the summary has no figure for it or
     the kernel sources changed since it was taken. Summary line format:
     `traffic <kernel> bytes_per_launch=<B> launches=<n> source=<hash>`."""
     p = os.path.join(ROOT, TRAFFIC_PROFILE)
-    if not os.path.exists(p):
+    kernel = KERNEL_OF_STAGE.get(stage)
+    if kernel is None or not os.path.exists(p):
         return None
     want = raster_source_hash()
     for line in open(p):
         f = line.split()
-        if len(f) >= 5 and f[0] == "traffic" and f[1] == kernel + "_kernel":
+        if len(f) >= 5 and f[0] == "traffic" and f[1] == kernel:
             kv = dict(t.split("=", 1) for t in f[2:] if "=" in t)
             if kv.get("source") == want:
                 return float(kv["bytes_per_launch"])
@@ -309,7 +313,7 @@ def run_ours(args):
     if dom in per_kernel:
         ops_per_launch = per_kernel[dom] / len(poses)
         achieved = ops_per_launch / (avg_ms * 1e-3) / 1e12
-        roof = {"kernel": dom, "bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
+        roof = {"kernel": dom, "kernel_name": KERNEL_OF_STAGE[dom], "bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
                 "frac": achieved / peak_alu, "traffic": profiled_traffic(dom),
                 "peak_source": f"148 SMs x 128 fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz (fp32 ops, FMA = 1)",
                 "ops_per_launch": ops_per_launch, "avg_launch_ms": avg_ms}

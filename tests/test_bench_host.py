@@ -16,7 +16,7 @@ def test_traffic_line_applies_only_to_matching_sources(tmp_path, monkeypatch):
     assert len(h) == 16
     prof = tmp_path / "p.md"
     prof.write_text("text\n"
-                    f"    traffic raster_bwd_kernel bytes_per_launch=123.5 launches=4 source={h}\n"
+                    f"    traffic raster_bwd_hits_kernel bytes_per_launch=123.5 launches=4 source={h}\n"
                     "    traffic raster_fwd_kernel bytes_per_launch=77 launches=4 source=0000000000000000\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "TRAFFIC_PROFILE", "p.md")

@@ -149,19 +149,57 @@ __global__ void __launch_bounds__(1024) scan_partials_kernel(int64_t* partials, 
   if (threadIdx.x == 0) *total = carry;
 }
 
+// Row j of a CTA's tile holds elements base + j kScanBlock + [0, kScanBlock):
+// every load and store is coalesced. Each warp scans its 32 elements of every
+// row with shuffles; one warp then scans the (row, warp) totals in element
+// order, so the whole tile needs two CTA barriers.
 __global__ void __launch_bounds__(kScanBlock) scan_down_kernel(const int32_t* tiles, const uint32_t* order,
                                                                int64_t n, const int64_t* partials,
                                                                int32_t* offsets) {
-  __shared__ int64_t scratch[kScanBlock / 32 + 1];
+  constexpr int kWarps = kScanBlock / 32;
+  constexpr int kParts = kScanItems * kWarps;  // (row, warp) pieces in element order
+  static_assert(kParts == 4 * 32, "one warp scans the pieces, four per lane");
+  __shared__ int64_t s_part[kParts];
   const int64_t base = (int64_t)blockIdx.x * kScanTile;
-  int64_t run = partials[blockIdx.x];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t ex[kScanItems];  // the element first, then its exclusive prefix in the warp's row
+#pragma unroll
   for (int j = 0; j < kScanItems; ++j) {
     const int64_t r = base + j * kScanBlock + threadIdx.x;
-    const int64_t v = r < n ? (int64_t)tiles[order ? order[r] : r] : 0;
-    int64_t t;
-    const int64_t ex = block_exclusive_scan<int64_t, kScanBlock>(v, t, scratch);
-    if (r < n) offsets[r] = (int32_t)(run + ex);
-    run += t;
+    ex[j] = r < n ? tiles[order ? order[r] : r] : 0;
+  }
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j) {
+    int32_t x = ex[j];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    ex[j] = x - ex[j];
+    if (lane == 31) s_part[j * kWarps + warp] = x;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int64_t a0 = s_part[4 * lane], a1 = s_part[4 * lane + 1], a2 = s_part[4 * lane + 2],
+                  a3 = s_part[4 * lane + 3];
+    int64_t x = a0 + a1 + a2 + a3;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    const int64_t e = x - (a0 + a1 + a2 + a3) + partials[blockIdx.x];
+    s_part[4 * lane] = e;
+    s_part[4 * lane + 1] = e + a0;
+    s_part[4 * lane + 2] = e + a0 + a1;
+    s_part[4 * lane + 3] = e + a0 + a1 + a2;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kScanItems; ++j) {
+    const int64_t r = base + j * kScanBlock + threadIdx.x;
+    if (r < n) offsets[r] = (int32_t)(s_part[j * kWarps + warp] + ex[j]);
   }
 }
 

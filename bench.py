@@ -274,30 +274,58 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # ---- timed region: whole steps, device-resident inputs. The bin/sort
-    # results (instance counts, statuses) stay on the device and are checked
-    # once after the region (Rasterizer.check raises on any failure).
+    # results (instance counts, statuses) stay on the device (deferred mode),
+    # so a whole step has no host round trip and is captured once as a CUDA
+    # graph (every launch and memset of the 4 poses), then replayed K times.
+    # The slots of the last replay are checked after the region
+    # (Rasterizer.check raises on any failure).
     R.deferred = True
-    R.stage_events = {}
-    launches0 = gs.gs_debug_kernel_launches()
+    R.check()
+    graph = torch.cuda.CUDAGraph()
+    l0 = gs.gs_debug_kernel_launches()
+    with torch.cuda.graph(graph):
+        step()
+    launches_per_step = gs.gs_debug_kernel_launches() - l0
+    slots = R._n_pending
+    graph.replay()  # one more untimed step, through the graph
+    torch.cuda.synchronize()
     _barrier(world)
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         ev0.record()
         for _ in range(args.steps):
-            step()
+            graph.replay()
         ev1.record()
         torch.cuda.synchronize()
     _barrier(world)
-    launches = gs.gs_debug_kernel_launches() - launches0
+    launches = launches_per_step * args.steps
+    R._n_pending = slots
     R.check()
     elapsed_ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
-    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in R.stage_events.items()}
-    stage_n = {k: len(v) for k, v in R.stage_events.items()}
-    R.stage_events = None
     frames = args.steps * len(poses) * world
     value = 1000.0 * frames / elapsed_ms
     ms_per_step = elapsed_ms / args.steps
+    del graph
+
+    # ---- the same steps launched one call at a time, with CUDA events
+    # around every stage: the per-stage times and the dominant kernel's
+    # launch duration for the roofline
+    R.stage_events = {}
+    _barrier(world)
+    torch.cuda.synchronize()
+    es0, es1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es0.record()
+    for _ in range(args.steps):
+        step()
+    es1.record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    R.check()
+    stage_loop_ms = _max_over_ranks(es0.elapsed_time(es1), world) / args.steps
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in R.stage_events.items()}
+    stage_n = {k: len(v) for k, v in R.stage_events.items()}
+    R.stage_events = None
 
     # ---- roofline of the dominant kernel
     peaks = _peaks()
@@ -338,7 +366,12 @@ def run_ours(args):
             "work_per_step": {"V": sum(c["V"] for c in counts), "I": sum(c["I"] for c in counts),
                               "E": E, "E_bwd": Eb, "B": B},
             "stages_ms_per_step": {k: v / args.steps for k, v in stage_ms.items()},
-            "roofline": roof, "gpu_launches": int(launches), "clocks": clocks}
+            "timing": {"value": "one CUDA graph per step (all launches of the 4 poses), replayed K times",
+                       "stages": "a second loop of K steps launched call by call, CUDA events around each "
+                                 "stage (the roofline's launch duration)",
+                       "stage_loop_ms_per_step": stage_loop_ms},
+            "roofline": roof, "gpu_launches": int(launches), "gpu_launches_per_step": int(launches_per_step),
+            "clocks": clocks}
 
     # ---- the importance pass: the forward that also sums alpha*T per Gaussian
     if not args.no_importance:

@@ -216,7 +216,7 @@ def run_reference(args):
         return
     import oracle
     from differentiable_tile_rasterizer_b200 import synthetic
-    scene = synthetic.make_config(WORKLOAD_CONFIG)
+    scene = synthetic.make_config(args.workload)
     for _ in range(args.warmup):
         cpu_sample(scene, tile_stride=args.ref_tile_stride)
     frames = []
@@ -248,7 +248,10 @@ def run_ours(args):
 
     world, rank, local = _dist_setup()
     gs.load(build_if_missing=False)
-    scene = synthetic.make_config(WORKLOAD_CONFIG)
+    scene = synthetic.make_config(args.workload)
+    lod, quant = float(scene.lod_dist), float(scene.importance_q)
+    if args.workload != WORKLOAD_CONFIG:  # another stated workload: the GPU step alone
+        args.no_importance = args.no_adam = args.no_e2e = args.no_cpu = True
     poses = scene.cameras
     cams = [gs.camera(c) for c in poses]
     params = GaussianParams.from_scene(scene)
@@ -259,7 +262,7 @@ def run_ours(args):
 
     def step():
         for p, c in enumerate(cams):
-            R.forward(params, c, bg)
+            R.forward(params, c, bg, lod, quant)
             R.backward(gimg[p])
 
     # warm-up (also settles the instance capacity)
@@ -269,7 +272,7 @@ def run_ours(args):
     # work counts per pose (deterministic; measured outside the timed region)
     counts = []
     for p, c in enumerate(cams):
-        R.forward(params, c, bg)
+        R.forward(params, c, bg, lod, quant)
         counts.append(R.work_counts())
     torch.cuda.synchronize()
 
@@ -304,6 +307,8 @@ def run_ours(args):
     R.check()
     elapsed_ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
     frames = args.steps * len(poses) * world
+    params_mb = sum(t.numel() * t.element_size() for t in
+                    (params.means, params.log_scales, params.quats, params.opacity_logits, params.sh)) / 1e6
     value = 1000.0 * frames / elapsed_ms
     ms_per_step = elapsed_ms / args.steps
     del graph
@@ -359,7 +364,9 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": scene.name, "gaussians": scene.N, "sh_degree": scene.sh_degree,
                        "width": W, "height": H, "poses_per_step": len(poses),
-                       "l2": "inputs larger than L2 (236 MB of parameters), no flush",
+                       "l2": (f"inputs larger than L2 ({params_mb:.0f} MB of parameters), no flush" if params_mb > 126
+                              else f"inputs smaller than L2 ({params_mb:.0f} MB of parameters): L2-warm, no flush"),
+                       "cull": {"lod_dist": lod, "importance_q": quant} if (lod > 0 or quant > 0) else "gates off",
                        "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
             "blends_per_s": 1000.0 * B * args.steps * world / elapsed_ms,
             "evaluated_pairs_per_s": 1000.0 * E * args.steps * world / elapsed_ms,
@@ -677,6 +684,9 @@ def e2e(args, scene, R, gimg, cams, bg, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--workload", type=int, default=WORKLOAD_CONFIG, choices=[1, 2, 3],
+                    help="stated workload: 1 (100K, 800x800), 2 (1M, 1080p, 4 poses; the default and the "
+                         "metric's), 3 (6M city with both cull gates); 1 and 3 time the GPU step alone")
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")

@@ -30,6 +30,9 @@ namespace {
 constexpr int kScanBlock = 256;
 constexpr int kScanItems = 16;
 constexpr int kScanTile = kScanBlock * kScanItems;
+constexpr int kVisTile = 1024;  // records per CTA of the visible-record compaction
+constexpr int kVisRows = kVisTile / kScanBlock;
+constexpr int kEmitChunk = 256;  // instances per warp of the emission
 constexpr int kSortBlock = 256;
 constexpr int kSortItems = 16;
 constexpr int kSortTile = kSortBlock * kSortItems;  // 4096
@@ -46,11 +49,15 @@ constexpr uint32_t kInvisibleKey = 0xffffffffu;
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 int64_t scan_blocks(int64_t n) { return (n + kScanTile - 1) / kScanTile; }
+int64_t vis_blocks(int64_t n) { return (n + kVisTile - 1) / kVisTile; }
+int64_t emit_chunks(int64_t capacity) { return (capacity + kEmitChunk - 1) / kEmitChunk + 1; }
+// entries of the partials buffer: the scans' and the compaction's blocks
+int64_t partial_slots(int64_t n) { return std::max(scan_blocks(n), vis_blocks(n)) + 1; }
 int64_t sort_tiles(int64_t n) { return (n + kSortTile - 1) / kSortTile; }
 
 struct SortWs {
   int64_t* partials;   // [scan blocks + 1]
-  int64_t* total;      // [1]
+  int64_t* total;      // [2]: instances, then visible records
   int32_t* status;     // [1]
   uint32_t* hist;      // [kMaxPasses][kRadix]
   uint32_t* counters;  // [64], directly followed by the look-back words
@@ -59,6 +66,7 @@ struct SortWs {
   uint32_t* dval[2];   // [n] record indices
   int32_t* doff;       // [n] instance offsets in depth order
   int32_t* dtiles;     // [n] tiles_touched in depth order
+  int32_t* chunk_g;    // [emit chunks] depth position of each emit chunk's first instance
   uint32_t* tkey[2];   // [capacity] tile ids
   uint32_t* tval[2];   // [capacity] record indices
 };
@@ -73,7 +81,7 @@ SortWs carve(void* ws, const BinSortPlan& p) {
   char* c = static_cast<char*>(ws);
   SortWs w;
   w.partials = reinterpret_cast<int64_t*>(c);
-  c += align256((size_t)(scan_blocks(p.n) + 1) * sizeof(int64_t));
+  c += align256((size_t)partial_slots(p.n) * sizeof(int64_t));
   w.total = reinterpret_cast<int64_t*>(c);
   c += 256;
   w.status = reinterpret_cast<int32_t*>(c);
@@ -93,6 +101,8 @@ SortWs carve(void* ws, const BinSortPlan& p) {
   c += align256((size_t)p.n * sizeof(int32_t));
   w.dtiles = reinterpret_cast<int32_t*>(c);
   c += align256((size_t)p.n * sizeof(int32_t));
+  w.chunk_g = reinterpret_cast<int32_t*>(c);
+  c += align256((size_t)emit_chunks(p.capacity) * sizeof(int32_t));
   for (int k = 0; k < 2; ++k) {
     w.tkey[k] = reinterpret_cast<uint32_t*>(c);
     c += align256((size_t)p.capacity * sizeof(uint32_t));
@@ -122,8 +132,10 @@ __device__ __forceinline__ int64_t live_instances(const int64_t* total, int64_t 
 // ---------------------------------------------------------------- scans
 // Exclusive scan of tiles[order[r]] (order == nullptr: identity).
 __global__ void __launch_bounds__(kScanBlock) scan_reduce_kernel(const int32_t* tiles, const uint32_t* order,
-                                                                 int64_t n, int64_t* partials) {
+                                                                 int64_t n, const int64_t* n_dev,
+                                                                 int64_t* partials) {
   __shared__ int64_t scratch[kScanBlock / 32 + 1];
+  if (n_dev && *n_dev < n) n = *n_dev;  // elements past the device count are 0
   const int64_t base = (int64_t)blockIdx.x * kScanTile;
   int64_t s = 0;
 #pragma unroll 4
@@ -155,11 +167,13 @@ __global__ void __launch_bounds__(1024) scan_partials_kernel(int64_t* partials, 
 // order, so the whole tile needs two CTA barriers.
 __global__ void __launch_bounds__(kScanBlock) scan_down_kernel(const int32_t* tiles, const uint32_t* order,
                                                                int64_t n, const int64_t* partials,
-                                                               int32_t* offsets) {
+                                                               int32_t* offsets, int32_t* chunk_g,
+                                                               int64_t n_chunks, const int64_t* n_dev) {
   constexpr int kWarps = kScanBlock / 32;
   constexpr int kParts = kScanItems * kWarps;  // (row, warp) pieces in element order
   static_assert(kParts == 4 * 32, "one warp scans the pieces, four per lane");
   __shared__ int64_t s_part[kParts];
+  if (n_dev && *n_dev < n) n = *n_dev;  // elements past the device count are 0 (and not written)
   const int64_t base = (int64_t)blockIdx.x * kScanTile;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t ex[kScanItems];  // the element first, then its exclusive prefix in the warp's row
@@ -199,77 +213,149 @@ __global__ void __launch_bounds__(kScanBlock) scan_down_kernel(const int32_t* ti
 #pragma unroll
   for (int j = 0; j < kScanItems; ++j) {
     const int64_t r = base + j * kScanBlock + threadIdx.x;
-    if (r < n) offsets[r] = (int32_t)(s_part[j * kWarps + warp] + ex[j]);
+    if (r < n) {
+      const int64_t off = s_part[j * kWarps + warp] + ex[j];
+      offsets[r] = (int32_t)off;
+      if (chunk_g) {  // element r holds the first instance of every emit chunk that starts in its range
+        const int64_t end = off + tiles[order ? order[r] : r];
+        for (int64_t b = (off + kEmitChunk - 1) / kEmitChunk; b * kEmitChunk < end && b < n_chunks; ++b)
+          chunk_g[b] = (int32_t)r;
+      }
+    }
   }
 }
 
 // ---------------------------------------------------------------- keys
-__global__ void __launch_bounds__(256) depth_keys_kernel(const float4* xyzo, const int32_t* tiles, int64_t n,
-                                                         uint32_t* key, uint32_t* val) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  key[i] = tiles[i] > 0 ? __float_as_uint(xyzo[i].z) : kInvisibleKey;
-  val[i] = (uint32_t)i;
+// The depth sort takes the visible records only (tiles_touched > 0),
+// compacted in record order: equal depths then keep record order, so the
+// sorted order equals that of a stable sort of all records with the
+// invisible ones keyed last, and a cull that leaves few records visible
+// sorts few keys. Two passes over tiles_touched: visible records per scan
+// block (then scan_partials_kernel), and the compacted keys and values.
+__global__ void __launch_bounds__(kScanBlock) vis_count_kernel(const int32_t* tiles, int64_t n, int64_t* partials) {
+  __shared__ int64_t scratch[kScanBlock / 32 + 1];
+  const int64_t base = (int64_t)blockIdx.x * kVisTile;
+  int64_t c = 0;
+#pragma unroll
+  for (int j = 0; j < kVisRows; ++j) {
+    const int64_t r = base + j * kScanBlock + threadIdx.x;
+    if (r < n && tiles[r] > 0) ++c;
+  }
+  const int64_t tot = block_sum<int64_t, kScanBlock>(c, scratch);
+  if (threadIdx.x == 0) partials[blockIdx.x] = tot;
 }
 
-// Instances of the Gaussians in depth order, tiles row-major in each rect.
-// A warp writes the instances of its 32 consecutive Gaussians as one
-// contiguous run (their offsets are consecutive), each lane finding the
-// Gaussian of its instance by a binary search over the warp's prefix sums,
-// so the stores coalesce however many tiles each Gaussian touches.
+// Row j of a CTA holds records base + j kScanBlock + [0, kScanBlock): a
+// ballot per warp row, then one warp scans the (row, warp) counts, one per
+// lane.
+__global__ void __launch_bounds__(kScanBlock) vis_compact_kernel(const float4* xyzo, const int32_t* tiles, int64_t n,
+                                                                 const int64_t* partials, uint32_t* key,
+                                                                 uint32_t* val) {
+  constexpr int kWarps = kScanBlock / 32;
+  static_assert(kVisRows * kWarps == 32, "one warp scans the pieces, one per lane");
+  __shared__ int64_t s_part[32];
+  const int64_t base = (int64_t)blockIdx.x * kVisTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t vis[kVisRows];  // ballot of the warp's row j
+#pragma unroll
+  for (int j = 0; j < kVisRows; ++j) {
+    const int64_t r = base + j * kScanBlock + threadIdx.x;
+    vis[j] = __ballot_sync(0xffffffffu, r < n && tiles[r] > 0);
+    if (lane == 0) s_part[j * kWarps + warp] = __popc(vis[j]);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int64_t a = s_part[lane];
+    int64_t x = a;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    s_part[lane] = x - a + partials[blockIdx.x];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kVisRows; ++j) {
+    if ((vis[j] >> lane) & 1u) {
+      const int64_t r = base + j * kScanBlock + threadIdx.x;
+      const int64_t pos = s_part[j * kWarps + warp] + __popc(vis[j] & lt);
+      key[pos] = __float_as_uint(xyzo[r].z);
+      val[pos] = (uint32_t)r;
+    }
+  }
+}
+
+// Instances of the Gaussians in depth order, tiles row-major in each rect,
+// partitioned by instance: warp w writes instances [w C, (w + 1) C) with
+// C = kEmitChunk, so a Gaussian that touches thousands of tiles is shared by
+// many warps (near-camera Gaussians sort next to each other, and giving each
+// warp whole Gaussians left a few warps with most of the instances). The
+// scan of the depth-order counts records the Gaussian of every chunk's first
+// instance; the warp walks windows of 32 consecutive Gaussians from it, each
+// lane finding the Gaussian of its instance by a binary search over the
+// window's offsets; the stores of every step are 32 consecutive slots.
 __global__ void __launch_bounds__(256) emit_kernel(const uint32_t* order, const int32_t* doff,
-                                                   const int32_t* dtiles, const ushort4* rect, int64_t n,
-                                                   int TW, const int64_t* total, int64_t capacity,
-                                                   int32_t* status, uint32_t* tkey, uint32_t* tval) {
+                                                   const int32_t* dtiles, const int32_t* chunk_g,
+                                                   const ushort4* rect, int64_t n, const int64_t* nvis, int TW,
+                                                   const int64_t* total,
+                                                   int64_t capacity, int32_t* status, uint32_t* tkey,
+                                                   uint32_t* tval) {
   if (*status != 0) return;  // the depth order is not valid
-  if (*total > capacity) {    // nothing is emitted or sorted
+  const int64_t I = *total;
+  if (I > capacity) {  // nothing is emitted or sorted
     if (blockIdx.x == 0 && threadIdx.x == 0) *status = GS_ERR_CAPACITY;
     return;
   }
-  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int lane = threadIdx.x & 31;
-  const int64_t r0 = r - lane;
-  if (r0 >= n) return;  // warp-uniform
-  int t = 0, x0 = 0, y0 = 0, bw = 1;
-  uint32_t i = 0;
-  if (r < n) {
-    t = dtiles[r];
-    i = order[r];
-    if (t > 0 && i < n) {
-      const ushort4 b = rect[i];
-      x0 = b.x;
-      y0 = b.y;
-      bw = (int)b.z - (int)b.x;
+  const int64_t chunk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t q0 = chunk * kEmitChunk;
+  if (q0 >= I) return;  // warp-uniform
+  const int64_t q1 = q0 + kEmitChunk < I ? q0 + kEmitChunk : I;
+  const int64_t nd = *nvis < n ? *nvis : n;  // depth positions past the visible records hold nothing
+  // the depth position whose instances hold q0 (written by the scan)
+  int64_t q = q0;
+  for (int64_t g = chunk_g[chunk]; q < q1; g += 32) {
+    const int64_t gl = g + lane;
+    int32_t off = INT32_MAX;  // lanes past the records never match
+    int t = 0, x0 = 0, y0 = 0, bw = 1;
+    uint32_t i = 0;
+    if (gl < nd) {
+      off = doff[gl];
+      t = dtiles[gl];
+      i = order[gl];
+      if (t > 0 && i < n) {
+        const ushort4 b = rect[i];
+        x0 = b.x;
+        y0 = b.y;
+        bw = (int)b.z - (int)b.x;
+      }
     }
-  }
-  const int64_t base = doff[r0];
-  int inc = t;
+    // the window's instances end where its last Gaussian's end (or all end)
+    const int64_t end = __shfl_sync(0xffffffffu, gl < nd ? (int64_t)off + t : I, 31);
+    const int64_t qe = end < q1 ? end : q1;
+    for (int64_t qs = q; qs < qe; qs += 32) {
+      const int64_t qq = qs + lane;
+      int L = 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += v;
-  }
-  const int ex = inc - t;
-  const int wtotal = __shfl_sync(0xffffffffu, inc, 31);  // instances of the warp
-  for (int p0 = 0; p0 < wtotal; p0 += 32) {
-    const int q = p0 + lane;
-    int L = 0;
-#pragma unroll
-    for (int st = 16; st > 0; st >>= 1) {
-      const int c = L + st;
-      if (__shfl_sync(0xffffffffu, ex, c) <= q) L = c;
+      for (int st = 16; st > 0; st >>= 1) {
+        const int c = L + st;
+        if ((int64_t)__shfl_sync(0xffffffffu, off, c) <= qq) L = c;
+      }
+      const int32_t offL = __shfl_sync(0xffffffffu, off, L);
+      const uint32_t iL = __shfl_sync(0xffffffffu, i, L);
+      const int x0L = __shfl_sync(0xffffffffu, x0, L);
+      const int y0L = __shfl_sync(0xffffffffu, y0, L);
+      const int bwL = __shfl_sync(0xffffffffu, bw, L);
+      if (qq < qe) {
+        const int li = (int)(qq - offL);
+        const int row = li / bwL;
+        tkey[qq] = (uint32_t)((y0L + row) * TW + x0L + (li - row * bwL));
+        tval[qq] = iL;
+      }
     }
-    const int exL = __shfl_sync(0xffffffffu, ex, L);
-    const uint32_t iL = __shfl_sync(0xffffffffu, i, L);
-    const int x0L = __shfl_sync(0xffffffffu, x0, L);
-    const int y0L = __shfl_sync(0xffffffffu, y0, L);
-    const int bwL = __shfl_sync(0xffffffffu, bw, L);
-    if (q < wtotal) {
-      const int li = q - exL;
-      const int row = li / bwL;
-      tkey[base + q] = (uint32_t)((y0L + row) * TW + x0L + (li - row * bwL));
-      tval[base + q] = iL;
-    }
+    q = qe;  // the next window starts where this one's instances end
   }
 }
 
@@ -468,14 +554,15 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, const
                                                      const int32_t* status, int64_t TT, uint2* ranges) {
   if (*status != 0) return;
   const int64_t n = live_instances(n_dev, cap);
-  const int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= n) return;
-  const uint64_t tile = keys[k] >> 32;
-  if (tile >= (uint64_t)TT) return;
-  const uint64_t prev = k > 0 ? (keys[k - 1] >> 32) : ~0ull;
-  const uint64_t next = k + 1 < n ? (keys[k + 1] >> 32) : ~0ull;
-  if (prev != tile) ranges[tile].x = (uint32_t)k;
-  if (next != tile) ranges[tile].y = (uint32_t)(k + 1);
+  // grid-stride: the grid is sized for a bound, the count is on the device
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
+    const uint64_t tile = keys[k] >> 32;
+    if (tile >= (uint64_t)TT) continue;
+    const uint64_t prev = k > 0 ? (keys[k - 1] >> 32) : ~0ull;
+    const uint64_t next = k + 1 < n ? (keys[k + 1] >> 32) : ~0ull;
+    if (prev != tile) ranges[tile].x = (uint32_t)k;
+    if (next != tile) ranges[tile].y = (uint32_t)(k + 1);
+  }
 }
 
 // One LSD sort over `passes` 8-bit digits starting at bit 0, keys/values
@@ -534,9 +621,10 @@ BinSortPlan binsort_plan(int64_t n, int64_t capacity, int64_t tiles) {
   while ((int64_t(1) << tb) < tiles) ++tb;
   p.tile_bits = tb;
   p.passes = (tb + 7) / 8;  // tile-digit passes over the instances
-  p.bytes = align256((size_t)(scan_blocks(n) + 1) * sizeof(int64_t)) + 256 + 256 +
+  p.bytes = align256((size_t)partial_slots(n) * sizeof(int64_t)) + 256 + 256 +
             align256(kMaxPasses * kRadix * sizeof(uint32_t)) + align256(lookback_words(p) * sizeof(uint32_t)) +
             4 * align256((size_t)n * sizeof(uint32_t)) + 2 * align256((size_t)n * sizeof(int32_t)) +
+            align256((size_t)emit_chunks(capacity) * sizeof(int32_t)) +
             4 * align256((size_t)capacity * sizeof(uint32_t));
   return p;
 }
@@ -559,26 +647,33 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
   const int64_t nb = scan_blocks(n);
   int launched = 0;
   if (offsets && nb > 0) {  // record-order offsets, on request
-    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, nullptr, n, w.partials);
+    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, nullptr, n, nullptr, w.partials);
     scan_partials_kernel<<<1, 1024, 0, s>>>(w.partials, nb, w.total);
-    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, nullptr, n, w.partials, offsets);
+    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(rec.tiles, nullptr, n, w.partials, offsets, nullptr, 0,
+                                                         nullptr);
     launched += 3;
   }
   if (n > 0) {
-    depth_keys_kernel<<<grid_for(n, 256), 256, 0, s>>>(rec.xyzo, rec.tiles, n, w.dkey[0], w.dval[0]);
-    // 4 passes: dkey[0] -> [1] -> [0] -> [1] -> [0]
+    // the visible records' depth keys, compacted; their count in nvis
+    int64_t* nvis = w.total + 1;
+    const int64_t nv = vis_blocks(n);
+    vis_count_kernel<<<(unsigned)nv, kScanBlock, 0, s>>>(rec.tiles, n, w.partials);
+    scan_partials_kernel<<<1, 1024, 0, s>>>(w.partials, nv, nvis);
+    vis_compact_kernel<<<(unsigned)nv, kScanBlock, 0, s>>>(rec.xyzo, rec.tiles, n, w.partials, w.dkey[0], w.dval[0]);
+    // 4 passes over the nvis keys: dkey[0] -> [1] -> [0] -> [1] -> [0]
     // the last pass also writes tiles_touched in depth order (dtiles)
-    const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, nullptr, kDepthPasses, w.dkey[0],
+    const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, nvis, kDepthPasses, w.dkey[0],
                               nullptr, w.dval[0], rec.xyzo, n, rec.tiles, w.dtiles, stall_tile, s);
     if (k < 0) return cudaErrorLaunchFailure;
-    launched += 1 + k;
-    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials);
+    launched += 3 + k;
+    scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.total + 1, w.partials);
     launched += 1;
   }
   scan_partials_kernel<<<1, 1024, 0, s>>>(w.partials, nb, w.total);
   launched += 1;
   if (nb > 0) {
-    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials, w.doff);
+    scan_down_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.partials, w.doff, w.chunk_g,
+                                                         emit_chunks(plan.capacity), w.total + 1);
     launched += 1;
   }
   count_launches(launched);
@@ -595,7 +690,8 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
   if (e != cudaSuccess) return e;
   int launched = 0;
   if (n > 0) {
-    emit_kernel<<<grid_for(n, 256), 256, 0, s>>>(w.dval[0], w.doff, w.dtiles, rec.rect, n, cam.TW, w.total, cap,
+    emit_kernel<<<grid_for((cap + kEmitChunk - 1) / kEmitChunk * 32, 256), 256, 0, s>>>(
+        w.dval[0], w.doff, w.dtiles, w.chunk_g, rec.rect, n, w.total + 1, cam.TW, w.total, cap,
                                                  w.status, w.tkey[0], w.tval[0]);
     ++launched;
   }
@@ -610,7 +706,8 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
       if (k < 0) return cudaErrorLaunchFailure;
       launched += k;
     }
-    ranges_kernel<<<grid_for(cap, 256), 256, 0, s>>>(keys, w.total, cap, w.status, TT,
+    ranges_kernel<<<(unsigned)std::min<int64_t>(grid_for(cap, 256), 148 * 16), 256, 0, s>>>(keys, w.total, cap,
+                                                                                          w.status, TT,
                                                       reinterpret_cast<uint2*>(ranges));
     ++launched;
   }

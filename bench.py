@@ -675,8 +675,42 @@ def e2e(args, scene, R, gimg, cams, bg, world):
     torch.cuda.synchronize()
     R.check()
     ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    # the bound: the same copies with no compute, each direction alone and
+    # both at once
+    def copies(b, h2d_on, d2h_on):
+        if h2d_on:
+            with torch.cuda.stream(up):
+                for k in keys:
+                    getattr(dev[b], k).copy_(host[k], non_blocking=True)
+                for p in range(len(cams)):
+                    dg[b][p].copy_(host_g[p], non_blocking=True)
+        if d2h_on:
+            with torch.cuda.stream(down):
+                for p in range(len(cams)):
+                    out_img[p].copy_(img[b][p], non_blocking=True)
+                for k, v in acc[b].items():
+                    out_grads[k].copy_(v, non_blocking=True)
+        comp.wait_stream(up)
+        comp.wait_stream(down)
+
+    reps = max(3, min(args.steps, 20))
+    copy_ms = {}
+    for name, hd in (("h2d", (True, False)), ("d2h", (False, True)), ("both", (True, True))):
+        copies(0, *hd)
+        torch.cuda.synchronize()
+        ec0, ec1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ec0.record(comp)
+        for s in range(reps):
+            copies(s & 1, *hd)
+        ec1.record(comp)
+        torch.cuda.synchronize()
+        copy_ms[name] = _max_over_ranks(ec0.elapsed_time(ec1), world) / reps
     return {"value": 1000.0 * args.steps * len(cams) * world / ms, "unit": "frames/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms / args.steps,
+            "copies_alone_ms_per_step": copy_ms,
+            "copy_bound": "max(h2d, d2h) alone if the link were full duplex; e2e within a step of compute plus "
+                          "the copies",
             "overlap": "H2D and D2H on their own streams; inputs/outputs double-buffered on the device",
             "result_read_back": "4 images + the parameter gradients summed over the step's 4 poses"}
 

@@ -163,7 +163,7 @@ struct FwdArgs {
   int32_t* last;
   float* importance;           // kImp: [N] += sum over pixels of alpha * T
   const int32_t* active_idx;   // record -> Gaussian, or null (identity)
-  uint8_t* hits;               // [entries] or null: bit w = warp w's block can blend the entry
+  uint8_t* hits;               // [entries] or null: bit w = the entry blended in warp w's block
 };
 
 // kImp also accumulates each Gaussian's importance weight (the sum over the
@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   __shared__ float4 s_box[kBatchF];  // blend region of each staged entry
   __shared__ float4 s_q1[kBatchF];
   __shared__ float4 s_q2[kBatchF];
-  // per batch parity: warp w's region ballot of chunk c (0 for chunks the
-  // warp did not test: its pixels had all stopped)
+  // per batch parity: the entries of chunk c that blended at some pixel of
+  // warp w (0 for chunks the warp did not reach: its pixels had all stopped)
   __shared__ uint32_t s_wm[2][kBlock / 32][kBatchF / 32];
   const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
   if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
       const int j = c0 + lane;
       const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy, 3.5f, 1.5f);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
-      if (a.hits && lane == 0) s_wm[par][warp][c0 >> 5] = msk;
+      unsigned blended = 0u;  // bit k - c0: entry k blended at a pixel of the warp
       // Entries are taken two at a time: their alphas at this pixel run as
       // one packed pair (each half rounded as the scalar operation), then
       // they blend in list order. Branch-free blend: a lane that skips an
@@ -274,6 +274,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
         cnt += blend ? 1 : 0;
         lst = blend ? base + k + 1 : lst;
         done = done || T < kTMin;
+        if (a.hits && __any_sync(0xffffffffu, blend)) blended |= 1u << (k - c0);
         if (kImp && __any_sync(0xffffffffu, blend)) {
           float ws = wgt;
 #pragma unroll
@@ -299,6 +300,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
         blend_one(k1, fminf(va.x, kAlphaMax));
         if (has2) blend_one(k2, fminf(va.y, kAlphaMax));
       }
+      if (a.hits && lane == 0) s_wm[par][warp][c0 >> 5] = blended;
     }
   }
   if (kImp || a.hits) {

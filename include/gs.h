@@ -374,14 +374,13 @@ GS_API int gs_tile_order(const uint32_t* tile_ranges, int64_t n_tiles, uint32_t*
  *   n_contrib    [device] [H][W] i32 out: blended Gaussians
  *   last         [device] [H][W] i32 out: 1 + list offset of the last blend
  *   hit_bits     [device] [n_instances] u8 out, or NULL: one byte per sorted
- *                list entry (indexed as vals); bit f set when the entry may
- *                blend in the 8x4 pixel block f of its tile (block f at
- *                column (f & 1) * 8, row (f >> 1) * 4), clear when it cannot
- *                blend there or when the block's pixels had all stopped
- *                before it. The backward's input of the same name. Written
- *                at least for every entry up to each tile's last blend;
- *                entries after the point where all of a tile's pixels
- *                stopped may be left as they were.
+ *                list entry (indexed as vals); bit f set when the entry
+ *                blended at some pixel of the 8x4 block f of its tile (block
+ *                f at column (f & 1) * 8, row (f >> 1) * 4), clear otherwise.
+ *                The backward's input of the same name. Written at least for
+ *                every entry up to each tile's last blend; entries after the
+ *                point where all of a tile's pixels stopped may be left as
+ *                they were.
  * Asynchronous. */
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
                             const uint32_t* tile_ranges, const uint32_t* tile_order,
@@ -422,9 +421,9 @@ GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* v
  *   tile_order   as for gs_rasterize_fwd (any permutation, or NULL)
  *   hit_bits     [device] the forward's hit_bits for the same lists, or NULL.
  *                Given, each warp walks its own 8x8 block's entries and
- *                fetches only those with its blocks' bits set, with no
- *                CTA-wide barrier; NULL, the kernel tests every entry's
- *                blend region itself. The results are the same either way
+ *                fetches only those that blended in one of its two 8x4
+ *                halves, with no CTA-wide barrier; NULL, the kernel tests
+ *                every entry's blend region itself. The results are the same either way
  *                up to the order of the fp32 atomic sums.
  *   final_T, last from gs_rasterize_fwd; dL_dimage [device] [3][H][W]
  *   grad2d       [device] [N][12] f32 out: (dpx, dpy, dopacity, 0,

@@ -1,9 +1,10 @@
 """The forward's hit bytes (one per sorted list entry: the 8x4 pixel blocks
-of its tile where it may blend) and the backward that walks only them.
+of its tile where it blended) and the backward that walks only them.
 
 - Every entry up to a tile's deepest last blend gets a byte (the same bytes
   whatever the buffer held before).
-- The block of every pixel has its bit set at the pixel's last blend.
+- The block of every pixel has its bit set at the pixel's last blend, and
+  each pixel's block has at least n_contrib set bits before its last.
 - The backward gives the oracle's gradients within the suite's tolerance
   with the bytes and without them (its own region tests), and the forward
   outputs do not depend on whether the bytes are written."""
@@ -60,6 +61,13 @@ def test_hit_bytes_written_and_set_at_each_last_blend(seed, W, H):
     bits = (ha[entry] >> block[ys, xs]) & 1
     assert bits.all(), f"{int((bits == 0).sum())} last blends outside their block's bits"
     assert len(ys) > 1000
+    # every blend of a pixel is an entry with its block's bit: per pixel, the
+    # set bits of its block among entries [0, last) are at least n_contrib
+    nc = Ra.n_contrib.cpu().numpy()
+    for y, x in list(zip(ys, xs))[::97]:
+        s0 = ranges[tile[y, x], 0]
+        setb = int(((ha[s0: s0 + last[y, x]] >> block[y, x]) & 1).sum())
+        assert setb >= nc[y, x], (y, x, setb, nc[y, x])
 
 
 @pytest.mark.parametrize("name", ["ragged", "dense_sh3"])

@@ -58,3 +58,47 @@ def test_graph_replay_of_a_step_matches_direct_calls():
     for n in NAMES:
         grad_tol_check(R.grads[n].cpu().numpy(), ob["d_" + n], ob["m_" + n], what=f"{n} after replay")
     del graph
+
+
+def test_graph_of_poses_on_their_own_streams():
+    # one Rasterizer and stream per pose, forked from and joined to the
+    # capture stream: each pose's replayed image equals its direct render
+    sc = S.random_scene(2500, 144, 112, sh_degree=1, seed=161, n_poses=3, log_scale=(-2.2, 0.4))
+    params = GaussianParams.from_scene(sc)
+    cams = [gs.camera(c) for c in sc.cameras]
+    gimg = [torch.from_numpy(sc.grad_image(p)).cuda() for p in range(3)]
+    Rs = [Rasterizer(sc.N, sc.sh_degree, sc.cameras[0].width, sc.cameras[0].height, capacity=64 * sc.N)
+          for _ in cams]
+    streams = [torch.cuda.Stream() for _ in cams]
+
+    def step():
+        cur = torch.cuda.current_stream()
+        for p, c in enumerate(cams):
+            streams[p].wait_stream(cur)
+            with torch.cuda.stream(streams[p]):
+                Rs[p].forward(params, c, sc.bg)
+                Rs[p].backward(gimg[p])
+        for st in streams:
+            cur.wait_stream(st)
+
+    step()
+    torch.cuda.synchronize()
+    direct = [R.image.clone() for R in Rs]
+    for R in Rs:
+        R.deferred = True
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for R in Rs:
+        R.image.zero_()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    for p, R in enumerate(Rs):
+        R._n_pending = 1
+        assert R.check()[0] > 0
+        assert_bits(R.image.cpu().numpy(), direct[p].cpu().numpy(), f"image pose {p}")
+    ref = oracle.render(S.Scene(sc.name, sc.N, sc.sh_degree, sc.means, sc.log_scales, sc.quats,
+                                sc.opacity_logits, sc.sh, [sc.cameras[1]], sc.bg, True))
+    assert_bits(Rs[1].image.cpu().numpy(), ref["fwd"]["image"], "pose 1 against the oracle")
+    del graph

@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
       const int j = c0 + lane;
       const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy, 3.5f, 1.5f);
       unsigned msk = __ballot_sync(0xffffffffu, rel);
-      unsigned blended = 0u;  // bit k - c0: entry k blended at a pixel of the warp
+      unsigned blended = 0u;  // bit k - c0: entry k blended at this lane's pixel (OR-ed over the warp below)
       // Entries are taken two at a time: their alphas at this pixel run as
       // one packed pair (each half rounded as the scalar operation), then
       // they blend in list order. Branch-free blend: a lane that skips an
@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
         cnt += blend ? 1 : 0;
         lst = blend ? base + k + 1 : lst;
         done = done || T < kTMin;
-        if (a.hits && __any_sync(0xffffffffu, blend)) blended |= 1u << (k - c0);
+        blended |= (blend ? 1u : 0u) << (k - c0);
         if (kImp && __any_sync(0xffffffffu, blend)) {
           float ws = wgt;
 #pragma unroll
@@ -300,7 +300,10 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
         blend_one(k1, fminf(va.x, kAlphaMax));
         if (has2) blend_one(k2, fminf(va.y, kAlphaMax));
       }
-      if (a.hits && lane == 0) s_wm[par][warp][c0 >> 5] = blended;
+      if (a.hits) {
+        blended = __reduce_or_sync(0xffffffffu, blended);
+        if (lane == 0) s_wm[par][warp][c0 >> 5] = blended;
+      }
     }
   }
   if (kImp || a.hits) {

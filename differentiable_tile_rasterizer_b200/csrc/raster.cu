@@ -591,6 +591,12 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
   cp_async_wait_all();  // no copy outlives the CTA
 }
 
+// Warps (8x8 blocks) per CTA of the hit-byte backward. Its warps share
+// nothing, so a CTA of one warp frees its slot as soon as its block is done
+// instead of waiting for the tile's other three blocks.
+constexpr int kHitsWarps = 1;
+static_assert(4 % kHitsWarps == 0, "a tile's four blocks split evenly over the CTAs");
+
 // cp.async groups: wait until at most one (the newest) is still in flight.
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
@@ -603,14 +609,16 @@ __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_
 // and never wait for each other. Per pixel the operations, and the entries
 // that blend, are those of raster_bwd_kernel, so every pixel's terms are
 // the same values; the warp sums go to the global gradient rows directly.
-__global__ void __launch_bounds__(kBlockB, 8) raster_bwd_hits_kernel(BwdArgs a) {
-  constexpr int kWarps = kBlockB / 32;
-  __shared__ float4 s_raw[kWarps][2][3][32];  // xyzo, conic, rgb of the hit entries of two chunks
-  __shared__ float s_acc[kWarps][32][9];      // the chunk's warp sums ([slot][value])
-  const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
-  if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
+__global__ void __launch_bounds__(32 * kHitsWarps) raster_bwd_hits_kernel(BwdArgs a) {
+  __shared__ float4 s_raw[kHitsWarps][2][3][32];  // xyzo, conic, rgb of the hit entries of two chunks
+  __shared__ float s_acc[kHitsWarps][32][9];      // the chunk's warp sums ([slot][value])
+  const int wc = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * kHitsWarps + wc;  // (tile slot, 8x8 block)
+  const uint32_t slot4 = (uint32_t)(gw >> 2);
+  const uint32_t tile_u = a.order ? a.order[slot4] : slot4;
+  if (tile_u >= gridDim.x * (uint32_t)kHitsWarps / 4u) return;  // not a tile: a schedule that is no permutation
   const int tile = (int)tile_u;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = (int)(gw & 3);
   const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
   const int u = tx0 + (warp & 1) * 8 + (lane & 7), v = ty0 + (warp >> 1) * 8 + (lane >> 3);
   const uint2 range = a.ranges[tile];
@@ -623,8 +631,8 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_hits_kernel(BwdArgs a) 
   const uint32_t fbits = (1u << f) | (1u << (f + 2));
   const uint32_t* lv = a.vals + range.x;
   const uint8_t* hb = a.hits + range.x;
-  float4(*raw)[3][32] = s_raw[warp];
-  float(*acc)[9] = s_acc[warp];
+  float4(*raw)[3][32] = s_raw[wc];
+  float(*acc)[9] = s_acc[wc];
   // lane's entry of chunk c: its record index and whether the block can blend it
   auto meta = [&](int c, uint32_t& idx, bool& hit) {
     const int off = warp_last - 1 - 32 * c - lane;
@@ -766,7 +774,7 @@ cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const ui
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d; a.hits = hits;
   if (hits)
-    raster_bwd_hits_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
+    raster_bwd_hits_kernel<<<cam.TW * cam.TH * 4 / kHitsWarps, 32 * kHitsWarps, 0, s>>>(a);
   else
     raster_bwd_kernel<<<cam.TW * cam.TH, kBlockB, 0, s>>>(a);
   count_launches(1);

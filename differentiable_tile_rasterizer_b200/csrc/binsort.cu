@@ -388,10 +388,8 @@ __global__ void __launch_bounds__(kRadix) digit_offsets_kernel(uint32_t* hist) {
 struct PassArgs {
   const uint32_t* kin;
   const uint32_t* vin;
-  uint32_t* kout;             // next-pass keys (unused when kout64 is set)
+  uint32_t* kout;             // next-pass keys
   uint32_t* vout;
-  uint64_t* kout64;           // final pass: (tile << 32) | depth bits of the record
-  const float4* xyzo;         // records, for the depth bits of the final keys
   int64_t n_records;          // values index records [0, n_records)
   const int32_t* tiles_in;    // optional: also write tiles_out[out] = tiles_in[value]
   int32_t* tiles_out;
@@ -518,11 +516,7 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
     // (values are record indices; the bound only matters after a look-back
     // timeout, when a slot can hold a stale value)
     const bool vok = v < a.n_records;
-    if (a.kout64) {
-      a.kout64[out] = ((uint64_t)k << 32) | (vok ? __float_as_uint(a.xyzo[v].z) : kInvisibleKey);
-    } else {
-      a.kout[out] = k;
-    }
+    a.kout[out] = k;
     a.vout[out] = v;
     if (a.tiles_out) a.tiles_out[out] = vok ? a.tiles_in[v] : 0;
   }
@@ -550,16 +544,25 @@ __global__ void publish_kernel(const int64_t* total, const int32_t* status, int6
 // ---------------------------------------------------------------- ranges
 // Tiles stay empty when the sort failed (status set), so a raster call on
 // these buffers reads nothing.
-__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, const int64_t* n_dev, int64_t cap,
-                                                     const int32_t* status, int64_t TT, uint2* ranges) {
+// Also writes the final 64-bit keys, (tile << 32) | depth bits of the
+// instance's record, from the sorted tile ids and values: a streaming loop
+// hides the record gathers better than the last sort pass's scatter would.
+__global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* tk, const uint32_t* tv, const float4* xyzo,
+                                                     int64_t n_records, uint64_t* keys, const int64_t* n_dev,
+                                                     int64_t cap, const int32_t* status, int64_t TT,
+                                                     uint2* ranges) {
   if (*status != 0) return;
   const int64_t n = live_instances(n_dev, cap);
   // grid-stride: the grid is sized for a bound, the count is on the device
   for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
-    const uint64_t tile = keys[k] >> 32;
+    const uint32_t tile = tk[k];
+    const uint32_t v = tv[k];
+    // (the bound only matters after a look-back timeout, when a slot can
+    // hold a stale value)
+    keys[k] = ((uint64_t)tile << 32) | (v < n_records ? __float_as_uint(xyzo[v].z) : kInvisibleKey);
     if (tile >= (uint64_t)TT) continue;
-    const uint64_t prev = k > 0 ? (keys[k - 1] >> 32) : ~0ull;
-    const uint64_t next = k + 1 < n ? (keys[k + 1] >> 32) : ~0ull;
+    const uint32_t prev = k > 0 ? tk[k - 1] : ~0u;
+    const uint32_t next = k + 1 < n ? tk[k + 1] : ~0u;
     if (prev != tile) ranges[tile].x = (uint32_t)k;
     if (next != tile) ranges[tile].y = (uint32_t)(k + 1);
   }
@@ -567,12 +570,12 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, const
 
 // One LSD sort over `passes` 8-bit digits starting at bit 0, keys/values
 // ping-ponging between (k0, v0) and (k1, v1); the last pass writes to
-// (last_k or last_k64, last_v). n keys, or with n_dev at most n keys, their
+// (last_k, last_v). n keys, or with n_dev at most n keys, their
 // number read on the device (live_instances(n_dev, n)). Returns the kernels
 // launched, -1 on error.
 int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint32_t* v1, int64_t n,
-                const int64_t* n_dev, int passes, uint32_t* last_k, uint64_t* last_k64, uint32_t* last_v,
-                const float4* xyzo, int64_t n_records, const int32_t* tiles_in, int32_t* tiles_out, int64_t stall,
+                const int64_t* n_dev, int passes, uint32_t* last_k, uint32_t* last_v, int64_t n_records,
+                const int32_t* tiles_in, int32_t* tiles_out, int64_t stall,
                 cudaStream_t s) {
   if (cudaMemsetAsync(w.hist, 0, kMaxPasses * kRadix * sizeof(uint32_t), s) != cudaSuccess) return -1;
   const int64_t nt = sort_tiles(n);
@@ -589,9 +592,7 @@ int sort_passes(const SortWs& w, uint32_t* k0, uint32_t* v0, uint32_t* k1, uint3
     a.kin = kb[p & 1];
     a.vin = vb[p & 1];
     a.kout = last ? last_k : kb[(p + 1) & 1];
-    a.kout64 = last ? last_k64 : nullptr;
     a.vout = last ? last_v : vb[(p + 1) & 1];
-    a.xyzo = xyzo;
     a.n_records = n_records;
     a.tiles_in = tiles_in;
     a.tiles_out = last ? tiles_out : nullptr;
@@ -663,7 +664,7 @@ cudaError_t launch_depth_order(const Records& rec, int64_t n, int32_t* offsets, 
     // 4 passes over the nvis keys: dkey[0] -> [1] -> [0] -> [1] -> [0]
     // the last pass also writes tiles_touched in depth order (dtiles)
     const int k = sort_passes(w, w.dkey[0], w.dval[0], w.dkey[1], w.dval[1], n, nvis, kDepthPasses, w.dkey[0],
-                              nullptr, w.dval[0], rec.xyzo, n, rec.tiles, w.dtiles, stall_tile, s);
+                              w.dval[0], n, rec.tiles, w.dtiles, stall_tile, s);
     if (k < 0) return cudaErrorLaunchFailure;
     launched += 3 + k;
     scan_reduce_kernel<<<(unsigned)nb, kScanBlock, 0, s>>>(w.dtiles, nullptr, n, w.total + 1, w.partials);
@@ -701,14 +702,15 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
                                                          vals);
       ++launched;
     } else {
+      // the last pass leaves tile ids (the ranges kernel writes the keys)
       const int k = sort_passes(w, w.tkey[0], w.tval[0], w.tkey[1], w.tval[1], cap, w.total, plan.passes,
-                                nullptr, keys, vals, rec.xyzo, n, nullptr, nullptr, stall_tile, s);
+                                w.tkey[plan.passes & 1], vals, n, nullptr, nullptr, stall_tile, s);
       if (k < 0) return cudaErrorLaunchFailure;
       launched += k;
     }
-    ranges_kernel<<<(unsigned)std::min<int64_t>(grid_for(cap, 256), 148 * 16), 256, 0, s>>>(keys, w.total, cap,
-                                                                                          w.status, TT,
-                                                      reinterpret_cast<uint2*>(ranges));
+    const uint32_t* tiles_sorted = plan.passes == 0 ? w.tkey[0] : w.tkey[plan.passes & 1];
+    ranges_kernel<<<(unsigned)std::min<int64_t>(grid_for(cap, 256), 148 * 16), 256, 0, s>>>(
+        tiles_sorted, vals, rec.xyzo, n, keys, w.total, cap, w.status, TT, reinterpret_cast<uint2*>(ranges));
     ++launched;
   }
   count_launches(launched);

@@ -10,6 +10,14 @@
 // ascending (tile, depth, record index). At 1080p with ~6 instances per
 // Gaussian this moves ~1/4 of the bytes of sorting all key bits per instance.
 //
+// Stages: the visible records' depth keys, compacted in record order (so a
+// cull that leaves few records visible sorts few keys); 4 depth passes; a
+// scan of tiles_touched in depth order, which also records the Gaussian of
+// every 256-instance chunk's first instance; the emission, partitioned by
+// instance so that Gaussians touching thousands of tiles are shared by many
+// warps; the tile passes over 32-bit tile ids; and the ranges kernel, which
+// finds each tile's run and writes the final 64-bit keys.
+//
 // Each sort pass is one "onesweep" kernel: a CTA takes the next 4096-key tile
 // (atomic ticket, so all earlier tiles are already resident), ranks its keys
 // per digit with warp ballots, publishes its per-digit counts and finds its

@@ -308,10 +308,11 @@ GS_API int gs_preprocess_multiview(const float* means, const float* log_scales, 
  * row-major order within the record's rect, sorted stably by key (equal keys
  * keep record order), then [start, end) per tile into tile_ranges (empty tiles
  * [0, 0)). The sort is an LSD radix sort with 8-bit digits (onesweep passes
- * with decoupled look-back): the 32 depth bits are sorted once per Gaussian,
- * the instances are emitted in that order, and only the ceil(log2(TW*TH)) tile
- * bits are sorted over the instances, which gives the same order as sorting
- * all key bits of every instance.
+ * with decoupled look-back): the 32 depth bits are sorted once per visible
+ * record (tiles_touched > 0; compacted in record order, so equal depths keep
+ * record order), the instances are emitted in that order, and only the
+ * ceil(log2(TW*TH)) tile bits are sorted over the instances, which gives the
+ * same order as sorting all key bits of every instance.
  *   in           [host] struct of [device] records, n entries
  *   offsets      [device] [n] i32 out, or NULL: exclusive scan of
  *                tiles_touched in record order

@@ -26,7 +26,11 @@ constexpr int kBlock = kTile * kTile;
 // Backward CTA: 4 warps, two pixels per thread.
 constexpr int kBlockB = kBlock / 2;
 // List entries staged in shared memory per CTA-wide step: one per thread.
-constexpr int kBatchF = kBlock;
+// Forward batch: 512 entries (two staged per thread) halve the CTA barriers
+// and even out the warps' shares of a batch; the importance variant, whose
+// per-entry sums need more registers, keeps 256.
+template <bool kImp>
+constexpr int fwd_batch() { return kImp ? kBlock : 2 * kBlock; }
 constexpr int kBatchB = kBlockB;
 
 // 16-byte asynchronous global -> shared copy (L2 only), its commit and the
@@ -171,13 +175,17 @@ struct FwdArgs {
 // shared-memory sum per staged entry, one atomic per (Gaussian, tile).
 template <bool kImp>
 __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
+  constexpr int kBatchF = fwd_batch<kImp>();
+  constexpr int kStageF = kBatchF / kBlock;  // entries each thread stages per batch
   __shared__ float s_imp[kImp ? kBatchF : 1];
   __shared__ float4 s_geo[kBatchF];  // px, py, a2, b2
   __shared__ float2 s_co[kBatchF];   // c2, opacity
   __shared__ float4 s_rgb[kBatchF];
-  __shared__ float4 s_box[kBatchF];  // blend region of each staged entry
+  // blend region of each staged entry (BlendRegion without what s_geo holds
+  // and the pad, which region_hits needs only when it derives from px, py)
+  __shared__ float2 s_hxy[kBatchF];  // box half-widths
   __shared__ float4 s_q1[kBatchF];
-  __shared__ float4 s_q2[kBatchF];
+  __shared__ float2 s_q2[kBatchF];
   // per batch parity: the entries of chunk c that blended at some pixel of
   // warp w (0 for chunks the warp did not reach: its pixels had all stopped)
   __shared__ uint32_t s_wm[2][kBlock / 32][kBatchF / 32];
@@ -198,26 +206,37 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int cnt = 0, lst = 0;
   bool done = !inside;
-  // importance: the entry this thread staged last, and its flush
-  uint32_t istaged = 0;
-  bool have_staged = false;
-  if (kImp) s_imp[tid] = 0.0f;
+  // importance: the entries this thread staged last (slots tid + s kBlock),
+  // and their flush
+  uint32_t istaged[kStageF] = {};
+  bool have_staged[kStageF] = {};
+  if (kImp)
+    for (int st = 0; st < kStageF; ++st) s_imp[tid + st * kBlock] = 0.0f;
   auto flush = [&]() {
-    if (kImp && have_staged) {
-      const float w = s_imp[tid];
-      if (w != 0.0f) atomicAdd(a.importance + (a.active_idx ? a.active_idx[istaged] : (int32_t)istaged), w);
-      s_imp[tid] = 0.0f;
-      have_staged = false;
+#pragma unroll
+    for (int st = 0; st < kStageF; ++st) {
+      if (kImp && have_staged[st]) {
+        const int e = tid + st * kBlock;
+        const float w = s_imp[e];
+        const uint32_t i = istaged[st];
+        if (w != 0.0f) atomicAdd(a.importance + (a.active_idx ? a.active_idx[i] : (int32_t)i), w);
+        s_imp[e] = 0.0f;
+        have_staged[st] = false;
+      }
     }
   };
-  // hit byte of the entry this thread staged in the batch at `hbase`, from
-  // the eight warps' ballots of parity `par`
+  // hit bytes of the entries this thread staged in the batch at `hbase`,
+  // from the eight warps' ballots of parity `par`
   auto write_hits = [&](int hbase, int par) {
-    if (a.hits && hbase >= 0 && hbase + tid < n) {
-      uint32_t h = 0;
 #pragma unroll
-      for (int w = 0; w < kBlock / 32; ++w) h |= ((s_wm[par][w][tid >> 5] >> lane) & 1u) << w;
-      a.hits[range.x + hbase + tid] = (uint8_t)h;
+    for (int st = 0; st < kStageF; ++st) {
+      const int e = tid + st * kBlock;
+      if (a.hits && hbase >= 0 && hbase + e < n) {
+        uint32_t h = 0;
+#pragma unroll
+        for (int w = 0; w < kBlock / 32; ++w) h |= ((s_wm[par][w][e >> 5] >> lane) & 1u) << w;
+        a.hits[range.x + hbase + e] = (uint8_t)h;
+      }
     }
   };
   // (The forward stages with plain gathers: with five CTAs per SM the
@@ -228,32 +247,44 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
     flush();  // the previous batch's sums are complete (barrier above)
     write_hits(base - kBatchF, par ^ 1);  // and its ballots
     last_staged = base;
+    static_assert((kBlock / 32) * (kBatchF / 32) <= kBlock, "one word per thread clears the ballots");
     if (a.hits && tid < (kBlock / 32) * (kBatchF / 32)) (&s_wm[par][0][0])[tid] = 0u;
-    if (base + tid < n) {
-      const int e = tid;
-      const uint32_t i = a.vals[range.x + base + e];
-      if (kImp) {
-        istaged = i;
-        have_staged = true;
+#pragma unroll
+    for (int st = 0; st < kStageF; ++st) {
+      const int e = tid + st * kBlock;
+      if (base + e < n) {
+        const uint32_t i = a.vals[range.x + base + e];
+        if (kImp) {
+          istaged[st] = i;
+          have_staged[st] = true;
+        }
+        const float4 g = a.xyzo[i];
+        const float4 q = a.conic[i];
+        const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
+                    c2 = __fmul_rn(q.z, kHalfNegLog2e);
+        s_geo[e] = make_float4(g.x, g.y, a2, b2);
+        s_co[e] = make_float2(c2, g.w);
+        s_rgb[e] = a.rgb[i];
+        const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
+        s_hxy[e] = make_float2(r.box.z, r.box.w);
+        s_q1[e] = r.q1;
+        s_q2[e] = make_float2(r.q2.x, r.q2.y);
       }
-      const float4 g = a.xyzo[i];
-      const float4 q = a.conic[i];
-      const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
-                  c2 = __fmul_rn(q.z, kHalfNegLog2e);
-      s_geo[e] = make_float4(g.x, g.y, a2, b2);
-      s_co[e] = make_float2(c2, g.w);
-      s_rgb[e] = a.rgb[i];
-      const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
-      s_box[e] = r.box;
-      s_q1[e] = r.q1;
-      s_q2[e] = r.q2;
     }
     __syncthreads();
     const int m = min(kBatchF, n - base);
     for (int c0 = 0; c0 < m; c0 += 32) {
       if (__all_sync(0xffffffffu, done)) break;
       const int j = c0 + lane;
-      const bool rel = j < m && region_hits(s_box[j], s_q1[j], s_q2[j], wcx, wcy, 3.5f, 1.5f);
+      bool rel = false;
+      if (j < m) {
+        const float4 gj = s_geo[j];
+        const float2 hj = s_hxy[j], qj = s_q2[j];
+        // blend_region's box and q2, the pad recomputed exactly as it did
+        const float pad = 0.05f + 1e-6f * (fabsf(gj.x) + fabsf(gj.y));
+        rel = region_hits(make_float4(gj.x, gj.y, hj.x, hj.y), s_q1[j], make_float4(qj.x, qj.y, pad, 0.0f), wcx,
+                          wcy, 3.5f, 1.5f);
+      }
       unsigned msk = __ballot_sync(0xffffffffu, rel);
       unsigned blended = 0u;  // bit k - c0: entry k blended at this lane's pixel (OR-ed over the warp below)
       // Entries are taken two at a time: their alphas at this pixel run as

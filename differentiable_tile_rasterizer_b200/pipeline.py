@@ -1,7 +1,8 @@
 """The rasterizer's public Python API: one view forward and backward through
-the five C entry points (gs_cull, gs_preprocess, gs_bin_sort,
-gs_rasterize_fwd, gs_rasterize_bwd). Torch only allocates device memory and
-supplies the stream; every stage runs in libgs.so.
+the C entry points (gs_cull, gs_preprocess, gs_bin_sort(_async),
+gs_tile_order, gs_rasterize_fwd, gs_rasterize_bwd), plus the multi-view
+renderer and the quantised SH optimizer. Torch only allocates device memory
+and supplies the stream; every stage runs in libgs.so.
 """
 
 from __future__ import annotations
@@ -80,10 +81,12 @@ class Rasterizer:
     """Buffers and calls for rendering one view of N Gaussians at W x H.
 
     forward() runs cull (when a gate is on) -> preprocess -> bin_sort ->
-    tile_order -> rasterize_fwd and keeps
-    what backward() needs; backward() runs rasterize_bwd. Buffers are
+    tile_order -> rasterize_fwd and keeps what backward() needs (including
+    the forward's hit bytes); backward() runs rasterize_bwd. Buffers are
     allocated once (the instance capacity grows when gs_bin_sort reports it
-    is too small) and reused across calls.
+    is too small) and reused across calls. In deferred mode no call reads
+    the device from the host, so a whole step can be captured in a CUDA
+    graph.
     """
 
     def __init__(self, N: int, sh_degree: int, width: int, height: int, device=None,
@@ -113,9 +116,10 @@ class Rasterizer:
         # sort and given to the raster launches; None: CTA b takes tile b.
         self.schedule_tiles = True
         self.tile_order = torch.arange(max(self.TT, 1), **i32)
-        # The forward writes one byte per list entry with the pixel blocks it
-        # may blend in, and the backward walks only those (gs_rasterize_fwd's
-        # hit_bits). False: the backward tests every entry itself.
+        # The forward writes one byte per list entry with the 8x4 pixel
+        # blocks where it blended, and the backward walks only those
+        # (gs_rasterize_fwd's hit_bits). False: the backward tests every
+        # entry's blend region itself.
         self.use_hit_bits = True
         self._hits_fresh = False  # hit_bits hold the current lists' bytes
         self.grad2d = torch.empty((n, 12), **f32)

@@ -374,9 +374,21 @@ __global__ void __launch_bounds__(256) digit_hist_kernel(const uint32_t* keys, i
   if (n_dev) n = live_instances(n_dev, cap);
   for (int b = threadIdx.x; b < kMaxPasses * kRadix; b += blockDim.x) sh[b] = 0;
   __syncthreads();
-  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n; k += (int64_t)gridDim.x * blockDim.x) {
-    const uint32_t key = keys[k];
+  // eight keys per thread and step, as two 16-byte loads issued together
+  // (the key buffers are 256-byte aligned), so their latencies overlap
+  auto count = [&](uint32_t key) {
     for (int p = 0; p < passes; ++p) atomicAdd(&sh[p * kRadix + ((key >> (8 * p)) & 255u)], 1u);
+  };
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x * 8;
+  for (int64_t k = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; k < n; k += stride) {
+    if (k + 8 <= n) {
+      const uint4 a = *reinterpret_cast<const uint4*>(keys + k);
+      const uint4 b = *reinterpret_cast<const uint4*>(keys + k + 4);
+      count(a.x); count(a.y); count(a.z); count(a.w);
+      count(b.x); count(b.y); count(b.z); count(b.w);
+    } else {
+      for (int64_t j = k; j < n; ++j) count(keys[j]);
+    }
   }
   __syncthreads();
   for (int b = threadIdx.x; b < passes * kRadix; b += blockDim.x)

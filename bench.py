@@ -4,14 +4,22 @@
 Workload (default): 1M Gaussians, SH degree 3, 1920x1080, four camera poses
 per step; each pose runs the whole path through the C ABI -- preprocess,
 bin/sort, tile order, rasterize forward, rasterize backward (2-D part and
-parameter part); both cull gates are off, so no cull runs. Inputs are synthetic and resident in HBM before timing; the
-236 MB parameter set is larger than the 126 MB L2, so no flush is needed.
+parameter part); both cull gates are off, so no cull runs. Inputs are
+synthetic and resident in HBM before timing; the 236 MB parameter set is
+larger than the 126 MB L2, so no flush is needed.
+
+Timing: `value` is K replays of one CUDA graph holding a whole step (each
+pose on its own stream and buffers); per-stage times and the roofline's
+kernel duration come from a second loop of K steps launched call by call
+with CUDA events around each stage. `e2e` runs the same steps through the
+public API with pinned host buffers, copies inside the timed region.
 
 Prints one JSON line on rank 0. Under torchrun (N > 1) each rank renders its
 own batch of poses with no collective on the data path (weak scaling); the
 time is the maximum over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload 1|2|3] [--multiview] [--interleaved G]
 """
 
 from __future__ import annotations

@@ -194,9 +194,12 @@ def cpu_sample(scene, tile_stride=32, pose=0):
 
     Sample: the full preprocess and bin/sort of one pose, forward and 2-D
     backward over every `tile_stride`-th tile, and the full parameter-gradient
-    chain; the per-tile parts are scaled by (tiles / sampled tiles)."""
+    chain; only the per-tile parts are scaled by (tiles / sampled tiles) (the
+    backward's once-per-call fp64 re-projection is measured with a one-tile
+    call and counted once)."""
     import oracle
     cam = scene.cameras[pose]
+    g = scene.grad_image(pose)  # the upstream gradient is an input, not timed
     t0 = time.perf_counter()
     rec = oracle.preprocess(scene, cam)
     t1 = time.perf_counter()
@@ -206,14 +209,29 @@ def cpu_sample(scene, tile_stride=32, pose=0):
     sub = np.arange(0, TT, tile_stride, dtype=np.int32)
     oracle.raster_fwd(rec, bins, cam, scene.bg, tile_subset=sub)
     t3 = time.perf_counter()
-    g = scene.grad_image(pose)
-    oracle.backward(scene, cam, rec, bins, g, params3d=True, tile_subset=sub)
+    # The raster backward re-projects every Gaussian in fp64 once per call
+    # (its fixed part) before the per-tile work; a one-tile call measures
+    # that part, so only the per-tile remainder is scaled to the frame.
+    bwd_fixed = 0.0
+    if len(sub) < TT:
+        oracle.backward(scene, cam, rec, bins, g, params3d=False, tile_subset=sub[:1])
+        bwd_fixed = time.perf_counter() - t3
+    t3b = time.perf_counter()
+    ob = oracle.backward(scene, cam, rec, bins, g, params3d=False, tile_subset=sub)
     t4 = time.perf_counter()
+    oracle.preprocess_bwd(scene, cam, rec, ob["g2d"])  # every Gaussian, whatever the tile sample
+    t5 = time.perf_counter()
     scale = TT / len(sub)
-    frame = (t1 - t0) + (t2 - t1) + (t3 - t2) * scale + (t4 - t3) * scale
-    return {"frame_s": frame, "sample_s": t4 - t0, "tiles_sampled": int(len(sub)), "tiles": int(TT),
+    if len(sub) < TT:
+        per_tile = max(0.0, (t4 - t3b) - bwd_fixed) / (len(sub) - 1) if len(sub) > 1 else 0.0
+        bwd = bwd_fixed + per_tile * (TT - 1)
+    else:
+        bwd = t4 - t3b
+    frame = (t1 - t0) + (t2 - t1) + (t3 - t2) * scale + bwd + (t5 - t4)
+    return {"frame_s": frame, "sample_s": t5 - t0, "tiles_sampled": int(len(sub)), "tiles": int(TT),
             "parts_s": {"preprocess": t1 - t0, "bin_sort": t2 - t1, "raster_fwd_sample": t3 - t2,
-                        "backward_sample": t4 - t3}}
+                        "raster_bwd_fixed": bwd_fixed, "raster_bwd_sample": t4 - t3b,
+                        "raster_bwd_frame": bwd, "preprocess_bwd": t5 - t4}}
 
 
 def run_reference(args):
@@ -235,7 +253,8 @@ def run_reference(args):
     ms = 1000.0 * float(np.mean(frames)) * len(scene.cameras)
     value = 1000.0 * len(scene.cameras) / ms
     sample = (f"per step: preprocess + bin/sort of 1 pose in full, forward and backward on every "
-              f"{args.ref_tile_stride}th tile, parameter gradients in full; scaled to a frame")
+              f"{args.ref_tile_stride}-th tile, parameter gradients in full; the per-tile parts scaled to "
+              f"a frame (the backward's once-per-call fp64 re-projection counted once)")
     line = {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",

@@ -354,7 +354,9 @@ GS_API int gs_bin_sort_async(const gs_projected* in, int64_t n, const gs_camera*
  * CTAs that take the longest lists start first and the launch does not end on
  * a few long tiles running alone (a longest-processing-time-first schedule;
  * without it, CTA b takes tile b). The order within one length class is
- * unspecified. The raster outputs do not depend on it.
+ * unspecified. The raster outputs do not depend on it. The pages describe
+ * no launch schedule (the 4D-GS page's tiled rasterization fixes only what
+ * each tile computes); this is an execution order, not a step of the method.
  *   tile_ranges  [device] [n_tiles] (start, end) u32 pairs from gs_bin_sort
  *   order        [device] [n_tiles] u32 out: a permutation of 0 .. n_tiles - 1
  * One CTA. Asynchronous; GS_ERR_INVALID_ARGUMENT on NULL pointers with

@@ -40,8 +40,11 @@ sys.path.insert(0, ROOT)
 METRIC = "fwd+bwd frames/s @1080p, 1M Gaussians SH3; blends/s; % of HBM/FP32 roofline"
 WORKLOAD_CONFIG = 2
 
-# Algorithmic fp32 operations per unit of work ("Roofline").
-OPS_EVAL = 21          # evaluate one (pixel, Gaussian) pair: quadratic form, exp2, alpha, test
+# Algorithmic fp32 operations per unit of work, counted from the operations of
+# the arithmetic specification (an FMA is one operation); the raster kernels'
+# roofline is these counts times the device-counted pairs and blends over the
+# launch time, against 148 SMs x 128 fp32 lanes x the max SM clock.
+OPS_EVAL = 21          # evaluate one (pixel, Gaussian) pair: quadratic 7, exp2 11, alpha 2, test 1
 OPS_BLEND_FWD = 8      # blend it: weight, 3 colour FMAs, 1 - alpha, T update, T test
 OPS_BLEND_BWD = 45     # backward per blend: T recovery, 9 gradient terms, 3 colour updates, 9 sums
 FP32_LANES_PER_SM = 128

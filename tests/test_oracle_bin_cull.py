@@ -1,8 +1,12 @@
 """Pins for the oracle's cull, scan, key emission, sort and tile ranges.
 
 References: numpy sorts and cumulative sums, Python's stable sorted(), a
-float64 distance, and a linear scan for ranges.
+float64 distance, and a linear scan for ranges; the sort also on random
+record sets drawn by hypothesis (repeated depths, invisible records,
+one-tile images).
 """
+
+import types
 
 import numpy as np
 import pytest
@@ -105,3 +109,56 @@ def test_cull_against_numpy(orc):
         assert np.array_equal(out["mask"].astype(bool), keep)
         assert np.array_equal(out["active_idx"], np.nonzero(keep)[0].astype(np.int32))
         assert out["n_active"] == keep.sum()
+
+
+def _records_strategy():
+    from hypothesis import strategies as st
+
+    @st.composite
+    def records(draw):
+        W = draw(st.integers(1, 90))
+        H = draw(st.integers(1, 70))
+        TW, TH = (W + 15) // 16, (H + 15) // 16
+        n = draw(st.integers(0, 30))
+        depths = draw(st.lists(st.sampled_from([0.25, 0.5, 1.0, 1.0000001, 3.0, 7.5]), min_size=n, max_size=n))
+        xyzo = np.zeros((n, 4), np.float32)
+        rect = np.zeros((n, 4), np.uint16)
+        tiles = np.zeros(n, np.int32)
+        for i in range(n):
+            xyzo[i, 2] = depths[i]
+            if draw(st.booleans()):  # visible: a non-empty rect inside the grid
+                x0 = draw(st.integers(0, TW - 1))
+                x1 = draw(st.integers(x0 + 1, TW))
+                y0 = draw(st.integers(0, TH - 1))
+                y1 = draw(st.integers(y0 + 1, TH))
+                rect[i] = (x0, y0, x1, y1)
+                tiles[i] = (x1 - x0) * (y1 - y0)
+        cam = types.SimpleNamespace(width=W, height=H, tiles_x=TW, tiles_y=TH)
+        return {"xyzo": xyzo, "rect": rect, "tiles": tiles}, cam
+
+    return records()
+
+
+def test_bin_sort_properties_on_random_records(orc):
+    # random rects, repeated depths, invisible records and one-tile images:
+    # the sort equals Python's stable sort of the emitted keys, the ranges
+    # are the runs of each tile, and the offsets the exclusive scan
+    from hypothesis import given, settings
+
+    @settings(max_examples=80, deadline=None)
+    @given(_records_strategy())
+    def check(rc):
+        rec, cam = rc
+        b = orc.bin_sort(rec, cam)
+        assert b["rc"] == 0
+        assert np.array_equal(b["offsets"], (np.cumsum(rec["tiles"]) - rec["tiles"]).astype(np.int32))
+        keys, vals = _emit_reference(rec, cam)
+        assert b["n_instances"] == keys.size
+        assert np.array_equal(b["keys"], keys)
+        assert np.array_equal(b["vals"], vals)
+        tile_of = (keys >> np.uint64(32)).astype(np.int64)
+        for t in range(cam.tiles_x * cam.tiles_y):
+            idx = np.nonzero(tile_of == t)[0]
+            assert tuple(b["ranges"][t]) == ((idx[0], idx[-1] + 1) if idx.size else (0, 0))
+
+    check()

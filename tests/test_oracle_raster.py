@@ -143,3 +143,22 @@ def test_float64_recursion_on_sampled_pixels(orc):
         assert T == pytest.approx(f["final_T"][v, u], rel=1e-4, abs=1e-9)
         np.testing.assert_allclose(C + T * sc.bg, f["image"][:, v, u], atol=2e-5)
     assert checked > 250
+
+
+def test_tiled_equals_bruteforce_on_random_scenes(orc):
+    # scene sizes, SH degrees, scale ranges and seeds drawn by hypothesis:
+    # the tiled walk gives the brute-force composite bit for bit
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=30, deadline=None)
+    @given(st.integers(1, 160), st.integers(1, 70), st.integers(1, 50), st.integers(0, 3),
+           st.sampled_from([(-3.5, 0.3), (-2.0, 0.5), (-1.0, 0.4)]), st.integers(0, 2 ** 16))
+    def check(n, W, H, deg, log_scale, seed):
+        sc = S.random_scene(n, W, H, sh_degree=deg, seed=seed, log_scale=log_scale)
+        r = orc.render(sc)
+        bf = orc.raster_fwd_bruteforce(r["rec"], r["cam"], sc.bg)
+        for k in ("image", "final_T", "n_contrib", "last"):
+            assert np.array_equal(bf[k], r["fwd"][k]), k
+
+    check()

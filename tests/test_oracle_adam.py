@@ -45,18 +45,15 @@ def test_log1p_and_expm1_spec_against_float64():
     assert oracle.expm1_spec(0.0) == 0.0
 
 
-@pytest.mark.parametrize("bits", [8, 16])
-def test_block_code_error_bound_and_order(bits):
-    rng = np.random.default_rng(92 + bits)
-    U, N = 5, 1000  # 4 blocks, the last one ragged
-    x = rng.normal(0, 1, (U, N)).astype(np.float32) * (10.0 ** rng.uniform(-4, 2, (U, 1))).astype(np.float32)
-    x[2, 256:512] = 0.375  # a constant block
+def _check_block_codes(x, bits):
+    U, N = x.shape
+    nb = (N + 255) // 256
     codes, bounds = oracle.quant_encode(x, bits)
     Q = 2 ** bits - 1
-    assert codes.shape == (U, 1024) and bounds.shape == (U, 4, 2)
+    assert codes.shape == (U, 256 * nb) and bounds.shape == (U, nb, 2)
     xh = oracle.quant_decode(codes, bounds, N, bits)
     for u in range(U):
-        for b in range(4):
+        for b in range(nb):
             sl = slice(256 * b, min(N, 256 * b + 256))
             blk, c = x[u, sl], codes[u, sl]
             lo, hi = bounds[u, b]
@@ -71,6 +68,34 @@ def test_block_code_error_bound_and_order(bits):
             err = np.abs(xh[u, sl].astype(np.float64) - blk)
             assert err.max() <= d / (2 * Q) * (1 + 1e-3) + 4 * np.spacing(F32(max(abs(lo), abs(hi))))
     assert not codes[:, N:].any()  # padding
+
+
+@pytest.mark.parametrize("bits", [8, 16])
+def test_block_code_error_bound_and_order(bits):
+    rng = np.random.default_rng(92 + bits)
+    U, N = 5, 1000  # 4 blocks, the last one ragged
+    x = rng.normal(0, 1, (U, N)).astype(np.float32) * (10.0 ** rng.uniform(-4, 2, (U, 1))).astype(np.float32)
+    x[2, 256:512] = 0.375  # a constant block
+    _check_block_codes(x, bits)
+
+
+def test_block_codes_on_random_planes():
+    # plane counts, ragged widths, scales, offsets and constant runs drawn by
+    # hypothesis: the same bounds, extremes, order and half-step error
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=40, deadline=None)
+    @given(st.integers(1, 4), st.integers(1, 700), st.sampled_from([8, 16]), st.floats(-6, 3),
+           st.floats(-100, 100), st.integers(0, 2 ** 16), st.booleans())
+    def check(U, N, bits, log_scale, offset, seed, constant_run):
+        rng = np.random.default_rng(seed)
+        x = (rng.normal(0, 1, (U, N)) * 10.0 ** log_scale + offset).astype(np.float32)
+        if constant_run:
+            x[0, : min(N, 300)] = np.float32(offset)
+        _check_block_codes(x, bits)
+
+    check()
 
 
 def _decode_state(st, N):

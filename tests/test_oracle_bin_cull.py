@@ -162,3 +162,32 @@ def test_bin_sort_properties_on_random_records(orc):
             assert tuple(b["ranges"][t]) == ((idx[0], idx[-1] + 1) if idx.size else (0, 0))
 
     check()
+
+
+def test_cull_quantile_on_random_weights(orc):
+    # sizes, quantiles and tie-heavy non-negative weights drawn by
+    # hypothesis: tau is numpy's value of rank floor(q N), the mask keeps
+    # w >= tau, and the active list is the kept indices in order
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    cam = simple_camera()
+    cam.campos = np.array([0.5, -1.0, 2.0], np.float32)
+
+    @settings(max_examples=40, deadline=None)
+    @given(st.integers(1, 3000), st.floats(0.001, 0.999), st.integers(1, 50), st.integers(0, 2 ** 16))
+    def check(N, q, n_values, seed):
+        rng = np.random.default_rng(seed)
+        imp = rng.choice(rng.exponential(1.0, n_values).astype(np.float32), N)  # many ties
+        means = rng.uniform(-5, 5, (3, N)).astype(np.float32)
+        sc = make_scene(means, np.zeros((3, N)), np.tile([[1], [0], [0], [0]], (1, N)), np.zeros(N),
+                        np.zeros((3, N)), 0, [cam], importance=imp, lod_dist=0.0, importance_q=q)
+        out = orc.cull(sc, cam)
+        tau = np.sort(imp)[int(np.floor(np.float64(np.float32(q)) * N))]
+        assert out["tau"] == tau
+        keep = imp >= tau
+        assert np.array_equal(out["mask"].astype(bool), keep)
+        assert np.array_equal(out["active_idx"], np.nonzero(keep)[0].astype(np.int32))
+        assert out["n_active"] == keep.sum()
+
+    check()

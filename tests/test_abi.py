@@ -62,3 +62,12 @@ def test_tile_order_argument_checks_need_no_gpu():
     assert L.gs_tile_order(None, -1, None, None) == gs.GS_ERR_INVALID_ARGUMENT
     assert L.gs_tile_order(None, 10, None, None) == gs.GS_ERR_INVALID_ARGUMENT
     assert L.gs_tile_order(None, 1 << 31, None, None) == gs.GS_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++17")])
+def test_header_is_plain_c_and_cxx(lang, std):
+    # the boundary is a C ABI: the header compiles as strict C99 and as C++
+    cc = "gcc" if lang == "c" else "g++"
+    r = subprocess.run([cc, "-fsyntax-only", f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-x", lang,
+                        os.path.join(ROOT, "include", "gs.h")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr

@@ -13,20 +13,6 @@ namespace {
 
 int64_t g_stall_tile = -1;
 
-bool finite_f(float v) { return std::isfinite(v); }
-
-bool camera_ok(const gs_camera* c) {
-  if (!c) return false;
-  if (c->width < 1 || c->height < 1 || c->width > 65535 * 16 || c->height > 65535 * 16) return false;
-  for (int k = 0; k < 9; ++k)
-    if (!finite_f(c->R[k])) return false;
-  for (int k = 0; k < 3; ++k)
-    if (!finite_f(c->t[k]) || !finite_f(c->campos[k])) return false;
-  if (!finite_f(c->fx) || !finite_f(c->fy) || !finite_f(c->cx) || !finite_f(c->cy)) return false;
-  if (!finite_f(c->near_z) || c->near_z < 0.0f) return false;
-  return true;
-}
-
 bool records_ok(const gs_projected* r) {
   return r && r->xyzo && r->conic && r->rgb && r->radius && r->rect && r->tiles_touched;
 }

@@ -20,6 +20,9 @@
 //    overlaps on the GPU (different streams, or different host threads) race
 //    on it and corrupt each other's results.
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <mutex>
 
@@ -31,45 +34,77 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 32 * 1024;
 
 // The scratch itself. In host code this name is only a stand-in for the symbol,
-// not a device address: the address is obtained once per device with
-// cudaGetSymbolAddress (see scratch_for_current_device) and passed to the
-// kernels like any workspace pointer.
+// not a device address: the address is obtained with cudaGetSymbolAddress
+// (see scratch_for_current_context) and passed to the kernels like any
+// workspace pointer.
 static __device__ __align__(256) unsigned char g_cull_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
+// The address of g_cull_scratch belongs to one CUDA context: every context
+// that loads the library (the device's primary context, a context the host
+// application created itself with cuCtxCreate, or the primary context
+// re-created after cudaDeviceReset) holds its own copy of the array at its own
+// address. The address is therefore cached per context, keyed by the
+// context's unique id (cuCtxGetId), which, unlike a context handle, is never
+// reused within a process. The two driver calls are reached through the
+// runtime's entry-point query, so the library does not link libcuda itself.
+constexpr int kMaxContexts = 64;
+struct ScratchSlot {
+  unsigned long long ctx_id;
+  void* ptr;
+};
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+ScratchSlot g_slots[kMaxContexts] = {};
+int g_n_slots = 0, g_next_evict = 0;
+PFN_cuCtxGetCurrent_v4000 g_get_current = nullptr;
+PFN_cuCtxGetId_v12000 g_get_id = nullptr;
 
-// Device address of the scratch on the current device; looked up on the first
-// call made with that device current, then cached.
-cudaError_t scratch_for_current_device(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_cull_scratch);
-    if (e != cudaSuccess) return e;
-    if (p == nullptr) return cudaErrorInvalidSymbol;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+cudaError_t resolve_driver_calls() {  // under g_mu
+  if (g_get_current && g_get_id) return cudaSuccess;
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) return e != cudaSuccess ? e : cudaErrorNotSupported;
+  g_get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  f = nullptr;
+  e = cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) return e != cudaSuccess ? e : cudaErrorNotSupported;
+  g_get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
   return cudaSuccess;
 }
 
-// The same camera checks as gs_cull.
-bool camera_usable(const gs_camera* c) {
-  if (!c) return false;
-  if (c->width < 1 || c->height < 1 || c->width > 65535 * 16 || c->height > 65535 * 16) return false;
-  for (int k = 0; k < 9; ++k)
-    if (!std::isfinite(c->R[k])) return false;
-  for (int k = 0; k < 3; ++k)
-    if (!std::isfinite(c->t[k]) || !std::isfinite(c->campos[k])) return false;
-  if (!std::isfinite(c->fx) || !std::isfinite(c->fy) || !std::isfinite(c->cx) || !std::isfinite(c->cy))
-    return false;
-  return std::isfinite(c->near_z) && c->near_z >= 0.0f;
+// Device address of the scratch in the context current on this thread; looked
+// up with cudaGetSymbolAddress on the first call made in that context, then
+// cached. If no context is current yet, the lookup itself binds the current
+// device's primary context, as any runtime call would.
+cudaError_t scratch_for_current_context(void** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaError_t e = resolve_driver_calls();
+  if (e != cudaSuccess) return e;
+  CUcontext ctx = nullptr;
+  if (g_get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  void* fresh = nullptr;
+  if (ctx == nullptr) {
+    e = cudaGetSymbolAddress(&fresh, g_cull_scratch);
+    if (e != cudaSuccess) return e;
+    if (g_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+  }
+  unsigned long long id = 0;
+  if (g_get_id(ctx, &id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  for (int k = 0; k < g_n_slots; ++k)
+    if (g_slots[k].ctx_id == id) {
+      *out = g_slots[k].ptr;
+      return cudaSuccess;
+    }
+  if (fresh == nullptr) {
+    e = cudaGetSymbolAddress(&fresh, g_cull_scratch);
+    if (e != cudaSuccess) return e;
+  }
+  if (fresh == nullptr) return cudaErrorInvalidSymbol;
+  // ids of destroyed contexts never come back, so an old slot can be reused
+  const int k = g_n_slots < kMaxContexts ? g_n_slots++ : (g_next_evict++ % kMaxContexts);
+  g_slots[k] = {id, fresh};
+  *out = fresh;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -77,14 +112,14 @@ bool camera_usable(const gs_camera* c) {
 extern "C" GS_API int gs_cull_noalloc(const float* means, const float* importance, int64_t N,
                                       const gs_camera* cam, float lod_dist, float importance_q, uint8_t* mask,
                                       int32_t* active_idx, int32_t* n_active, void* stream) {
-  if (N < 0 || N > GS_CULL_NOALLOC_MAX_N || !camera_usable(cam)) return GS_ERR_INVALID_ARGUMENT;
+  if (N < 0 || N > GS_CULL_NOALLOC_MAX_N || !gs::camera_ok(cam)) return GS_ERR_INVALID_ARGUMENT;
   if (!(importance_q >= 0.0f) || !(importance_q < 1.0f) || !std::isfinite(lod_dist))
     return GS_ERR_INVALID_ARGUMENT;
   if (gs::cull_workspace_bytes(N) > kNoAllocScratchBytes) return GS_ERR_INVALID_ARGUMENT;
   if (!n_active || (N > 0 && (!means || !mask || !active_idx))) return GS_ERR_INVALID_ARGUMENT;
   if (importance_q > 0.0f && N > 0 && !importance) return GS_ERR_INVALID_ARGUMENT;
   void* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != cudaSuccess) return GS_ERR_CUDA;
+  if (scratch_for_current_context(&scratch) != cudaSuccess) return GS_ERR_CUDA;
   const cudaError_t e = gs::launch_cull(means, importance, N, gs::make_devcam(*cam), lod_dist, importance_q, mask,
                                         active_idx, n_active, scratch, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;

@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 
@@ -16,6 +17,20 @@ struct DevCam {
   float fx, fy, cx, cy, near_z;
   int width, height, TW, TH;
 };
+
+// Host-side camera validation shared by every entry point that takes a camera:
+// a positive image size whose tile grid fits the 16-bit rect fields, finite
+// pose and intrinsics, and near_z >= 0 (so depth bits sort like depths).
+inline bool camera_ok(const gs_camera* c) {
+  if (!c) return false;
+  if (c->width < 1 || c->height < 1 || c->width > 65535 * 16 || c->height > 65535 * 16) return false;
+  for (int k = 0; k < 9; ++k)
+    if (!std::isfinite(c->R[k])) return false;
+  for (int k = 0; k < 3; ++k)
+    if (!std::isfinite(c->t[k]) || !std::isfinite(c->campos[k])) return false;
+  if (!std::isfinite(c->fx) || !std::isfinite(c->fy) || !std::isfinite(c->cx) || !std::isfinite(c->cy)) return false;
+  return std::isfinite(c->near_z) && c->near_z >= 0.0f;
+}
 
 inline DevCam make_devcam(const gs_camera& c) {
   DevCam d;

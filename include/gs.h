@@ -124,9 +124,12 @@ GS_API int gs_cull(const float* means, const float* importance, int64_t N, const
  *   arguments    as for gs_cull, without workspace/workspace_bytes
  *   N            at most GS_CULL_NOALLOC_MAX_N; larger N returns
  *                GS_ERR_INVALID_ARGUMENT (use gs_cull with a workspace)
- * The first call made with a given device current looks up the array's device
- * address (cudaGetSymbolAddress) and caches it; make that first call before
- * any stream capture on the device. Every call shares the one array: each
+ * Each CUDA context that loads the library (a device's primary context, a
+ * context the host application created itself, the primary context again
+ * after cudaDeviceReset) holds its own copy of the array. The first call made
+ * in a context looks up that copy's device address (cudaGetSymbolAddress) and
+ * caches it under the context's unique id; make that first call before any
+ * stream capture in the context. Every call shares the one array: each
  * clears what must start at zero, but calls that overlap on the GPU (other
  * streams or host threads) race on it. Asynchronous otherwise. */
 #define GS_CULL_NOALLOC_MAX_N 16777216

@@ -18,3 +18,21 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Worst gradient ratios |g - g_ref| / (rtol |g_ref| + m S) of the GPU
+    parity checks, at each recorded floor m."""
+    try:
+        from tests.gpu_helpers import FLOORS, GRAD_RATIOS
+    except Exception:
+        return
+    if not GRAD_RATIOS:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "gradient parity: worst ratio per check (<= 1 passes)")
+    tr.write_line(f"{'check':60s} {'elements':>10s} {'rtol':>7s} " + " ".join(f"{'m=%g' % m:>10s}" for m in FLOORS))
+    for what, n, rtol, worst in GRAD_RATIOS:
+        tr.write_line(f"{what[:60]:60s} {n:10d} {rtol:7.0e} " + " ".join(f"{w:10.4f}" for w in worst))
+    tr.write_line("overall worst: " + ", ".join(f"m={m:g}: {max(r[3][k] for r in GRAD_RATIOS):.4f}"
+                                                for k, m in enumerate(FLOORS)))

@@ -94,9 +94,9 @@ def test_deferred_capacity_failure_leaves_tiles_empty_then_recovers():
 
 
 def test_async_lookback_timeout_reported_in_result():
-    sc = S.random_scene(3000, 256, 256, sh_degree=0, seed=42, log_scale=(-1.0, 0.3))
+    sc = S.random_scene(12000, 256, 256, sh_degree=0, seed=42, log_scale=(-1.5, 0.3))
     R = gpu_forward(sc)
-    assert R.n_instances > 3 * 4096  # several sort tiles per pass
+    assert int((R.rec["tiles"] > 0).sum()) > 4096 and R.n_instances > 3 * 4096  # several sort tiles per pass
     c = gs.camera(sc.cameras[0])
     res = torch.zeros(2, dtype=torch.int64, device="cuda")
     gs.gs_debug_set_stalled_sort_tile(1)

@@ -248,10 +248,12 @@ def test_preprocess_backward_stagewise():
 
 
 def test_sort_lookback_timeout_is_reported_and_recoverable():
-    sc = S.random_scene(3000, 256, 256, sh_degree=0, seed=42, log_scale=(-1.0, 0.3))
+    # more than one 4096-key sort tile in every radix pass, the depth passes
+    # over the visible records included
+    sc = S.random_scene(12000, 256, 256, sh_degree=0, seed=42, log_scale=(-1.5, 0.3))
     cam = sc.cameras[0]
     R = gpu_forward(sc)
-    assert R.n_instances > 3 * 4096  # several sort tiles per pass
+    assert int((R.rec["tiles"] > 0).sum()) > 4096 and R.n_instances > 3 * 4096
     c = gs.camera(cam)
     gs.gs_debug_set_stalled_sort_tile(1)
     try:

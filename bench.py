@@ -14,9 +14,10 @@ kernel duration come from a second loop of K steps launched call by call
 with CUDA events around each stage. `e2e` runs the same steps through the
 public API with pinned host buffers, copies inside the timed region.
 
-Prints one JSON line on rank 0. Under torchrun (N > 1) each rank renders its
-own batch of poses with no collective on the data path (weak scaling); the
-time is the maximum over ranks.
+Prints one JSON line on rank 0. Under torchrun (N > 1) the step is
+data-parallel training over views (weak scaling): each rank renders its own
+batch of poses, sums their parameter gradients and all-reduces the sum with
+the other ranks (NCCL) every step; the time is the maximum over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload 1|2|3] [--multiview] [--interleaved G]
@@ -95,6 +96,84 @@ def profiled_traffic(stage: str):
             if kv.get("source") == want:
                 return float(kv["bytes_per_launch"])
     return None
+
+
+def profiled_exec_ops(stage: str):
+    """Executed fp32 operations per launch of the kernel of `stage` (FFMA +
+    FADD + FMUL thread instructions, the packed FFMA2/FADD2/FMUL2 counted
+    twice) from one ncu capture recorded in the committed summary, or None
+    when it has none for the current kernel sources. Summary line format:
+    `fp32ops <kernel> ops_per_launch=<x> launches=<n> source=<hash>`."""
+    p = os.path.join(ROOT, TRAFFIC_PROFILE)
+    kernel = KERNEL_OF_STAGE.get(stage)
+    if kernel is None or not os.path.exists(p):
+        return None
+    want = raster_source_hash()
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 5 and f[0] == "fp32ops" and f[1] == kernel:
+            kv = dict(t.split("=", 1) for t in f[2:] if "=" in t)
+            if kv.get("source") == want:
+                return float(kv["ops_per_launch"])
+    return None
+
+
+def stage_work(scene, counts):
+    """Algorithmic bytes and fp32 operations per stage, summed over the
+    poses of one step, from the per-pose counts (V visible, I instances, E
+    and E_bwd evaluated pairs, B blends). Bytes are what a stage must move at
+    least: parameters and records read once, outputs written once."""
+    K = scene.K
+    N = scene.N
+    cam = scene.cameras[0]
+    P = cam.width * cam.height
+    TT = cam.tiles_x * cam.tiles_y
+    par = (11 + 3 * K) * 4  # parameter bytes per Gaussian
+    w = {k: {"bytes": 0.0, "ops": 0.0} for k in ("cull", "preprocess", "bin_sort", "raster_fwd", "raster_bwd",
+                                                 "preprocess_bwd")}
+    for c in counts:
+        V, I, E, Eb, B = c["V"], c["I"], c["E"], c["E_bwd"], c["B"]
+        A = c.get("A", N)
+        if c.get("culled"):
+            # means and weight in, two 16-bit select passes over the weights,
+            # mask out, active list out
+            w["cull"]["bytes"] += N * (16 + 2 * 4 + 1) + 4 * A
+        w["preprocess"]["bytes"] += A * (par + 64)  # active parameters in, 64 B record out
+        # record depth, rect and tile count in; 64-bit keys and values out; ranges
+        w["bin_sort"]["bytes"] += 16 * N + 12 * I + 8 * TT
+        # list entry, its 48 B record and its hit byte; image, T, counts, last out
+        w["raster_fwd"]["bytes"] += 53 * I + 24 * P
+        w["raster_fwd"]["ops"] += OPS_EVAL * E + OPS_BLEND_FWD * B
+        # the same entries; upstream gradient, T and last in; 48 B gradient rows out
+        w["raster_bwd"]["bytes"] += 53 * I + 20 * P + 48 * V
+        w["raster_bwd"]["ops"] += OPS_EVAL * Eb + OPS_BLEND_BWD * B
+        # every gradient row out (zero rows of culled and invisible
+        # Gaussians included); parameters, 2-D gradient row and colour in for
+        # the visible ones
+        w["preprocess_bwd"]["bytes"] += N * par + V * (par + 48 + 16)
+    if not any(c.get("culled") for c in counts):
+        del w["cull"]
+    return w
+
+
+def step_roofline(work, stage_ms, ms_per_step, steps, bw_gbs, peak_alu_t):
+    """Sum over stages of max(bytes / HBM bandwidth, ops / fp32 peak) for one
+    step, against the measured step time."""
+    per = {}
+    bound_ms = 0.0
+    for k, v in work.items():
+        t_mem = v["bytes"] / (bw_gbs * 1e9) * 1e3
+        t_alu = v["ops"] / (peak_alu_t * 1e12) * 1e3
+        t = max(t_mem, t_alu)
+        bound_ms += t
+        meas = stage_ms.get(k, 0.0) / max(steps, 1)
+        per[k] = {"bytes": v["bytes"], "ops": v["ops"], "bound": "alu" if t_alu > t_mem else "hbm",
+                  "roofline_ms": t, "measured_ms": meas, "frac": t / meas if meas > 0 else None}
+    return {"frac": bound_ms / ms_per_step, "roofline_ms_per_step": bound_ms, "ms_per_step": ms_per_step,
+            "stages": per,
+            "definition": "sum over stages of max(bytes / measured HBM copy bandwidth, fp32 ops / (SMs x 128 "
+                          "lanes x max clock)) for one step, over the graph-replayed step time; per stage the "
+                          "same bound over its call-by-call CUDA-event time"}
 
 
 class ClockSampler:
@@ -185,6 +264,28 @@ def _max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def flat_gradients(N: int, K: int, device):
+    """One flat float32 buffer of a whole parameter gradient and its views in
+    the library's SoA shapes (means [3][N], log_scales [3][N], quats [4][N],
+    opacity_logits [N], sh [3K][N]), so that one collective reduces all."""
+    import torch
+    flat = torch.empty((11 + 3 * K) * N, dtype=torch.float32, device=device)
+    views, o = {}, 0
+    for name, rows in (("means", 3), ("log_scales", 3), ("quats", 4), ("opacity_logits", 1), ("sh", 3 * K)):
+        v = flat[o: o + rows * N]
+        views[name] = v if name == "opacity_logits" else v.view(rows, N)
+        o += rows * N
+    return flat, views
+
+
+def reduce_gradients(flat, world: int):
+    """The data-parallel step's exchange: the sum over ranks of every rank's
+    parameter gradient (one all-reduce; NCCL between GPUs, gloo on CPU)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM)
+
+
 def _barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -243,8 +344,30 @@ def cpu_sample(scene, tile_stride=32, pose=0):
                         "raster_bwd_frame": bwd, "preprocess_bwd": t5 - t4}}
 
 
+def bench_config(scene, world: int) -> dict:
+    """The `config` of the JSON line, the same for both arms."""
+    params_mb = sum(np.asarray(a).nbytes for a in (scene.means, scene.log_scales, scene.quats,
+                                                   scene.opacity_logits, scene.sh)) / 1e6
+    lod, quant = float(scene.lod_dist), float(scene.importance_q)
+    cam = scene.cameras[0]
+    return {"workload": scene.name, "gaussians": scene.N, "sh_degree": scene.sh_degree,
+            "width": cam.width, "height": cam.height, "poses_per_step": len(scene.cameras),
+            "l2": (f"inputs larger than L2 ({params_mb:.0f} MB of parameters), no flush" if params_mb > 126
+                   else f"inputs smaller than L2 ({params_mb:.0f} MB of parameters): L2-warm, no flush"),
+            "cull": {"lod_dist": lod, "importance_q": quant} if (lod > 0 or quant > 0) else "gates off",
+            "parallelism": (f"data parallel over views: {world} ranks, each rendering its own poses; the "
+                            f"step's parameter gradients all-reduced (NCCL) every step") if world > 1
+            else "single GPU"}
+
+
 def run_reference(args):
-    """The oracle timed as it stands on this host's cores (reference arm)."""
+    """The oracle timed as it stands on this host's cores (reference arm).
+
+    A reference step is a bounded sample of the bench step: one of its poses
+    (in turn), the whole frame -- preprocess, bin/sort, forward and backward
+    on every tile (unless --ref-tile-stride samples tiles, then the per-tile
+    parts are scaled to the frame), parameter gradients. Each step is timed by
+    its own wall clock, so ms_per_step x steps is the timed region."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -252,27 +375,29 @@ def run_reference(args):
     import oracle
     from differentiable_tile_rasterizer_b200 import synthetic
     scene = synthetic.make_config(args.workload)
+    n_poses = len(scene.cameras)
     for w in range(args.warmup):
-        cpu_sample(scene, tile_stride=args.ref_tile_stride, pose=w % len(scene.cameras))
+        cpu_sample(scene, tile_stride=args.ref_tile_stride, pose=w % n_poses)
     frames = []
     t0 = time.perf_counter()
     for s in range(args.steps):
-        frames.append(cpu_sample(scene, tile_stride=args.ref_tile_stride, pose=s % len(scene.cameras))["frame_s"])
+        frames.append(cpu_sample(scene, tile_stride=args.ref_tile_stride, pose=s % n_poses)["frame_s"])
     wall = time.perf_counter() - t0
-    ms = 1000.0 * float(np.mean(frames)) * len(scene.cameras)
-    value = 1000.0 * len(scene.cameras) / ms
-    sample = (f"per step: preprocess + bin/sort of 1 pose in full, forward and backward on every "
-              f"{args.ref_tile_stride}-th tile, parameter gradients in full; the per-tile parts scaled to "
-              f"a frame (the backward's once-per-call fp64 re-projection counted once)")
+    ms = 1000.0 * float(np.mean(frames))  # one frame per reference step
+    value = 1000.0 / ms
+    tiles = "every tile" if args.ref_tile_stride == 1 else (
+        f"every {args.ref_tile_stride}-th tile, the per-tile parts scaled to a frame (the backward's "
+        f"once-per-call fp64 re-projection counted once)")
+    sample = (f"per step: one of the step's {n_poses} poses in turn, whole frame: preprocess, bin/sort, "
+              f"forward and backward on {tiles}, parameter gradients")
     line = {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "reference",
-            "config": {"workload": scene.name, "gaussians": scene.N, "sh_degree": 3, "width": 1920,
-                       "height": 1080, "poses_per_step": len(scene.cameras)},
+            "config": bench_config(scene, world),
             "cpu_baseline": {"value": value, "unit": "frames/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "wall_s": wall}
+            "frames_per_step": 1, "wall_s": wall}
     print(json.dumps(line), flush=True)
 
 
@@ -307,6 +432,12 @@ def run_ours(args):
     # chain per pose).
     Rp = [R] + [Rasterizer(scene.N, scene.sh_degree, W, H, capacity=6 * scene.N) for _ in cams[1:]]
     streams = [torch.cuda.Stream() for _ in cams]
+    # With several ranks the step is data-parallel training over views: each
+    # rank sums its poses' parameter gradients (the first pose writes, the
+    # others add, in order on one stream) and the ranks all-reduce the sum.
+    flat = acc = None
+    if world > 1:
+        flat, acc = flat_gradients(scene.N, scene.K, params.means.device)
 
     def step_streams():
         cur = torch.cuda.current_stream()
@@ -314,14 +445,21 @@ def run_ours(args):
             streams[p].wait_stream(cur)
             with torch.cuda.stream(streams[p]):
                 Rp[p].forward(params, c, bg, lod, quant)
-                Rp[p].backward(gimg[p])
+                if acc is None:
+                    Rp[p].backward(gimg[p])
+                else:
+                    Rp[p].backward_2d(gimg[p])
         for st in streams:
             cur.wait_stream(st)
+        if acc is not None:
+            for p in range(len(cams)):
+                Rp[p].backward_params(acc, accumulate=p > 0)
 
     # warm-up (also settles the instance capacities)
     for _ in range(max(args.warmup, 0)):
         step()
         step_streams()
+        reduce_gradients(flat, world)
     torch.cuda.synchronize()
     # work counts per pose (deterministic; measured outside the timed region)
     counts = []
@@ -346,6 +484,7 @@ def run_ours(args):
     launches_per_step = gs.gs_debug_kernel_launches() - l0
     slots = [r._n_pending for r in Rp]
     graph.replay()  # one more untimed step, through the graph
+    reduce_gradients(flat, world)
     torch.cuda.synchronize()
     _barrier(world)
     torch.cuda.synchronize()
@@ -354,6 +493,7 @@ def run_ours(args):
         ev0.record()
         for _ in range(args.steps):
             graph.replay()
+            reduce_gradients(flat, world)
         ev1.record()
         torch.cuda.synchronize()
     _barrier(world)
@@ -363,8 +503,6 @@ def run_ours(args):
         r.check()
     elapsed_ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
     frames = args.steps * len(poses) * world
-    params_mb = sum(t.numel() * t.element_size() for t in
-                    (params.means, params.log_scales, params.quats, params.opacity_logits, params.sh)) / 1e6
     value = 1000.0 * frames / elapsed_ms
     ms_per_step = elapsed_ms / args.steps
     del graph
@@ -402,10 +540,18 @@ def run_ours(args):
     if dom in per_kernel:
         ops_per_launch = per_kernel[dom] / len(poses)
         achieved = ops_per_launch / (avg_ms * 1e-3) / 1e12
+        exe = profiled_exec_ops(dom)
         roof = {"kernel": dom, "kernel_name": KERNEL_OF_STAGE[dom], "bound": "alu", "achieved": achieved, "peak": peak_alu, "unit": "TFLOP/s",
-                "frac": achieved / peak_alu, "traffic": profiled_traffic(dom),
+                "frac": achieved / peak_alu, "frac_spec": achieved / peak_alu,
+                "frac_executed": (exe / (avg_ms * 1e-3) / 1e12 / peak_alu) if exe else None,
+                "executed_fp32_ops_per_launch": exe,
+                "traffic": profiled_traffic(dom),
                 "peak_source": f"148 SMs x 128 fp32 lanes x {peaks['sm_max_mhz']:.0f} MHz (fp32 ops, FMA = 1)",
-                "ops_per_launch": ops_per_launch, "avg_launch_ms": avg_ms}
+                "ops_per_launch": ops_per_launch, "avg_launch_ms": avg_ms,
+                "bases": "frac_spec: the specification's operations for every evaluated pair and blend (21 E_bwd + "
+                         "45 B for the backward), some of which the kernel provably skips; frac_executed: the fp32 "
+                         "instructions one ncu capture counted for one launch (FFMA + FADD + FMUL, packed "
+                         "FFMA2/FADD2/FMUL2 twice), over the same launch time"}
     else:
         K = scene.K
         nbytes = (11 + 3 * K) * 4 * scene.N + 64 * scene.N if dom == "preprocess" else \
@@ -418,23 +564,23 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": scene.name, "gaussians": scene.N, "sh_degree": scene.sh_degree,
-                       "width": W, "height": H, "poses_per_step": len(poses),
-                       "l2": (f"inputs larger than L2 ({params_mb:.0f} MB of parameters), no flush" if params_mb > 126
-                              else f"inputs smaller than L2 ({params_mb:.0f} MB of parameters): L2-warm, no flush"),
-                       "cull": {"lod_dist": lod, "importance_q": quant} if (lod > 0 or quant > 0) else "gates off",
-                       "parallelism": f"{world} independent replicas" if world > 1 else "single GPU"},
+            "config": bench_config(scene, world),
             "blends_per_s": 1000.0 * B * args.steps * world / elapsed_ms,
             "evaluated_pairs_per_s": 1000.0 * E * args.steps * world / elapsed_ms,
             "work_per_step": {"V": sum(c["V"] for c in counts), "I": sum(c["I"] for c in counts),
                               "E": E, "E_bwd": Eb, "B": B},
             "stages_ms_per_step": {k: v / args.steps for k, v in stage_ms.items()},
             "timing": {"value": "one CUDA graph per step, replayed K times: all launches of the 4 poses, each "
-                                "pose on its own stream and buffers (4 independent chains)",
+                                "pose on its own stream and buffers (4 independent chains)" +
+                                ("; with several ranks the graph also sums the poses' parameter gradients and "
+                                 "each replay is followed by their all-reduce" if world > 1 else ""),
                        "stages": "a second loop of K steps launched call by call, CUDA events around each "
                                  "stage (the roofline's launch duration)",
                        "stage_loop_ms_per_step": stage_loop_ms},
-            "roofline": roof, "gpu_launches": int(launches), "gpu_launches_per_step": int(launches_per_step),
+            "roofline": roof,
+            "step_roofline": step_roofline(stage_work(scene, counts), stage_ms, ms_per_step, args.steps,
+                                           peaks["hbm_gbs"], peak_alu),
+            "gpu_launches": int(launches), "gpu_launches_per_step": int(launches_per_step),
             "clocks": clocks}
 
     # ---- the importance pass: the forward that also sums alpha*T per Gaussian
@@ -673,7 +819,7 @@ def e2e(args, scene, R, gimg, cams, bg, world):
     dev = [GaussianParams.from_scene(scene) for _ in range(2)]
     dg = [[torch.empty_like(g) for g in gimg] for _ in range(2)]
     img = [[torch.empty_like(R.image) for _ in cams] for _ in range(2)]
-    acc = [{k: torch.empty_like(v) for k, v in R.grads.items()} for _ in range(2)]
+    flats, acc = zip(*[flat_gradients(scene.N, scene.K, R.dev) for _ in range(2)])
     out_img = [torch.empty_like(R.image, device="cpu").pin_memory() for _ in cams]
     out_grads = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in R.grads.items()}
     h2d = sum(t.numel() * t.element_size() for t in host.values()) + sum(
@@ -709,6 +855,7 @@ def e2e(args, scene, R, gimg, cams, bg, world):
             img[b][p].copy_(R.image)
             for k, v in R.grads.items():
                 acc[b][k].add_(v)
+        reduce_gradients(flats[b], world)
         ev_comp[b].record(comp)
         with torch.cuda.stream(down):
             down.wait_event(ev_comp[b])
@@ -783,8 +930,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--ref-tile-stride", type=int, default=32,
-                    help="reference arm: sample every n-th tile per step")
+    ap.add_argument("--ref-tile-stride", type=int, default=1,
+                    help="reference arm: sample every n-th tile per step (1: whole frames)")
     ap.add_argument("--no-importance", action="store_true", help="skip timing the importance pass")
     ap.add_argument("--no-adam", action="store_true", help="skip timing the quantised SH Adam step")
     ap.add_argument("--interleaved", type=int, default=0,

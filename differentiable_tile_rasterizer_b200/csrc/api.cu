@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 
+#include "checked.cuh"
 #include "gs.h"
 #include "gs_internal.cuh"
 
@@ -58,6 +59,21 @@ GS_API const char* gs_status_string(int status) {
 GS_API void gs_debug_set_stalled_sort_tile(int64_t tile) { g_stall_tile = tile < 0 ? -1 : tile; }
 
 GS_API int64_t gs_debug_kernel_launches(void) { return kernel_launches(); }
+
+GS_API int gs_debug_is_checked_build(void) {
+#ifdef GS_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+GS_API uint32_t gs_debug_checked_status(void) {
+  const uint32_t s[3] = {checked_status_raster(), checked_status_binsort(), checked_status_preprocess()};
+  for (uint32_t v : s)
+    if (v) return v;
+  return 0;
+}
 
 GS_API int gs_cull(const float* means, const float* importance, int64_t N, const gs_camera* cam,
                    float lod_dist, float importance_q, uint8_t* mask, int32_t* active_idx,
@@ -183,6 +199,7 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals, const 
                             int32_t* n_contrib, int32_t* last, uint8_t* hit_bits, void* stream) {
   if (!records_ok(in) || !camera_ok(cam) || !tile_ranges || !bg || !image || !final_T || !n_contrib || !last)
     return GS_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(hit_bits) & 3u) return GS_ERR_INVALID_ARGUMENT;  // word atomics
   const float b[3] = {bg[0], bg[1], bg[2]};
   return cuda_status(launch_raster_fwd(to_records(in), vals, tile_ranges, make_devcam(*cam), b, image, final_T,
                                        n_contrib, last, nullptr, nullptr, tile_order, hit_bits,
@@ -265,12 +282,18 @@ GS_API int gs_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* v
 
 GS_API int64_t gs_route_ctas(int64_t n) { return n < 0 ? 0 : route_ctas(n); }
 
-GS_API int gs_route_count(const gs_projected* rec, int64_t n, int n_ranks, int tiles_y, uint32_t* mask,
-                          uint32_t* cta_counts, int64_t* totals, void* stream) {
+GS_API int gs_route_count(const gs_projected* rec, int64_t n, int n_ranks, int tiles_y, const int32_t* band_starts,
+                          uint32_t* mask, uint32_t* cta_counts, int64_t* totals, int64_t* dst_offsets, void* stream) {
   if (!records_ok(rec) || n < 0 || n >= (int64_t(1) << 31) || n_ranks < 1 || n_ranks > GS_MAX_RANKS ||
       tiles_y < 1 || !totals || (n > 0 && (!mask || !cta_counts)))
     return GS_ERR_INVALID_ARGUMENT;
-  return cuda_status(launch_route_count(to_records(rec), n, n_ranks, tiles_y, mask, cta_counts, totals,
+  BandStarts b;
+  for (int q = 0; q <= n_ranks; ++q) {
+    b.row[q] = band_starts ? band_starts[q] : (int32_t)(((int64_t)q * tiles_y) / n_ranks);
+    if (q > 0 && b.row[q] < b.row[q - 1]) return GS_ERR_INVALID_ARGUMENT;
+  }
+  if (b.row[0] != 0 || b.row[n_ranks] != tiles_y) return GS_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_route_count(to_records(rec), n, n_ranks, b, mask, cta_counts, totals, dst_offsets,
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -322,7 +345,26 @@ GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const 
   Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};
   Grads g{d_means, d_log_scales, d_quats, d_opacity_logits, d_sh};
   return cuda_status(launch_preprocess_bwd(p, mask, make_devcam(*cam), to_records(in),
-                                           reinterpret_cast<const float4*>(grad2d), g,
+                                           reinterpret_cast<const float4*>(grad2d), g, false,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+GS_API int gs_preprocess_bwd_accumulate(const float* means, const float* log_scales, const float* quats,
+                                        const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                                        const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
+                                        const gs_projected* in, const float* grad2d, float* d_means,
+                                        float* d_log_scales, float* d_quats, float* d_opacity_logits, float* d_sh,
+                                        void* stream) {
+  if (sh_degree < 0) return GS_ERR_INVALID_ARGUMENT;
+  if (sh_degree > 3) return GS_ERR_UNSUPPORTED;
+  if (!params_ok(means, log_scales, quats, opacity_logits, sh, N) || !camera_ok(cam) || !records_ok(in))
+    return GS_ERR_INVALID_ARGUMENT;
+  if (N > 0 && (!grad2d || !d_means || !d_log_scales || !d_quats || !d_opacity_logits || !d_sh))
+    return GS_ERR_INVALID_ARGUMENT;
+  Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};
+  Grads g{d_means, d_log_scales, d_quats, d_opacity_logits, d_sh};
+  return cuda_status(launch_preprocess_bwd(p, nullptr, make_devcam(*cam), to_records(in),
+                                           reinterpret_cast<const float4*>(grad2d), g, true,
                                            static_cast<cudaStream_t>(stream)));
 }
 
@@ -354,7 +396,7 @@ GS_API int gs_rasterize_bwd(const float* means, const float* log_scales, const f
   }
   Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, active_idx, n_active};
   Grads g{d_means, d_log_scales, d_quats, d_opacity_logits, d_sh};
-  return cuda_status(launch_preprocess_bwd(p, mask, dc, rec, reinterpret_cast<const float4*>(grad2d), g, s));
+  return cuda_status(launch_preprocess_bwd(p, mask, dc, rec, reinterpret_cast<const float4*>(grad2d), g, false, s));
 }
 
 }  // extern "C"

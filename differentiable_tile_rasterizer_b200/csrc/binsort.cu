@@ -27,6 +27,7 @@
 // GS_ERR_DEVICE_TIMEOUT in the status word and carries on without hanging.
 // A single histogram kernel per sort builds the digit counts of all passes.
 
+#include "checked.cuh"
 #include "gs_internal.cuh"
 #include "scan_util.cuh"
 
@@ -41,8 +42,8 @@ constexpr int kScanTile = kScanBlock * kScanItems;
 constexpr int kVisTile = 1024;  // records per CTA of the visible-record compaction
 constexpr int kVisRows = kVisTile / kScanBlock;
 constexpr int kEmitChunk = 256;  // instances per warp of the emission
-constexpr int kSortBlock = 256;
-constexpr int kSortItems = 16;
+constexpr int kSortBlock = 512;
+constexpr int kSortItems = 8;
 constexpr int kSortTile = kSortBlock * kSortItems;  // 4096
 constexpr int kSortWarps = kSortBlock / 32;
 constexpr int kRadix = 256;
@@ -424,10 +425,15 @@ struct PassArgs {
   int64_t stall_tile;
 };
 
-__global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
+// 512 threads of 8 keys each, two CTAs per SM (64 registers): twice the
+// resident warps of 256 threads of 16 keys, for the same 4096-key tile and
+// look-back. A warp's count of one digit is at most 256 and a digit's
+// exclusive offset inside the tile below 4096, so the per-warp counts are
+// 16-bit (the CTA's shared memory stays under the 48 KB static limit).
+__global__ void __launch_bounds__(kSortBlock, 2) onesweep_kernel(PassArgs a) {
   __shared__ uint32_t s_keys[kSortTile];
   __shared__ uint32_t s_vals[kSortTile];
-  __shared__ uint32_t s_whist[kSortWarps][kRadix];
+  __shared__ uint16_t s_whist[kSortWarps][kRadix];
   __shared__ uint32_t s_dstart[kRadix];
   __shared__ uint32_t s_gbase[kRadix];
   __shared__ uint32_t s_scan[kSortWarps + 1];
@@ -468,29 +474,34 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
       const uint32_t bb = __ballot_sync(0xffffffffu, (d >> b) & 1u);
       peers &= ((d >> b) & 1u) ? bb : ~bb;
     }
-    const uint32_t pre = d < kRadix ? s_whist[warp][d] : 0u;
+    const uint32_t pre = d < kRadix ? (uint32_t)s_whist[warp][d] : 0u;
     __syncwarp();
-    if (d < kRadix && lane == 31 - __clz(peers)) s_whist[warp][d] = pre + __popc(peers);
+    if (d < kRadix && lane == 31 - __clz(peers)) s_whist[warp][d] = (uint16_t)(pre + __popc(peers));
     __syncwarp();
     rank[j] = pre + __popc(peers & lt);
   }
   __syncthreads();
-  // Per digit (thread d): exclusive offsets of the warps, block count.
+  // Per digit (thread d < kRadix): exclusive offsets of the warps, block count.
   const int d = tid;
+  const bool owner = d < kRadix;
   uint32_t cnt = 0;
+  if (owner) {
 #pragma unroll
-  for (int w = 0; w < kSortWarps; ++w) {
-    const uint32_t c = s_whist[w][d];
-    s_whist[w][d] = cnt;
-    cnt += c;
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t c = s_whist[w][d];
+      s_whist[w][d] = (uint16_t)cnt;
+      cnt += c;
+    }
   }
   uint32_t blk_total;
-  s_dstart[d] = block_exclusive_scan<uint32_t, kSortBlock>(cnt, blk_total, s_scan);
+  const uint32_t dstart = block_exclusive_scan<uint32_t, kSortBlock>(cnt, blk_total, s_scan);
+  if (owner) s_dstart[d] = dstart;
   // Decoupled look-back for digit d.
   const bool stall = tile == a.stall_tile;
   uint32_t* row = a.lookback + (size_t)tile * kRadix;
   uint32_t excl = 0;
-  if (tile == 0) {
+  if (!owner) {
+  } else if (tile == 0) {
     if (!stall) st_relaxed(row + d, kFlagInc | cnt);
   } else {
     if (!stall) st_relaxed(row + d, kFlagAgg | cnt);
@@ -513,14 +524,14 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
     }
     if (!stall) st_relaxed(row + d, kFlagInc | ((excl + cnt) & kValMask));
   }
-  s_gbase[d] = a.digit_off[d] + excl;
+  if (owner) s_gbase[d] = a.digit_off[d] + excl;
   __syncthreads();
   // Scatter into shared memory in digit order.
 #pragma unroll
   for (int j = 0; j < kSortItems; ++j) {
     const uint32_t dj = dig[j];
     if (dj < kRadix) {
-      const uint32_t pos = s_dstart[dj] + s_whist[warp][dj] + rank[j];
+      const uint32_t pos = s_dstart[dj] + (uint32_t)s_whist[warp][dj] + rank[j];
       s_keys[pos] = key[j];
       s_vals[pos] = val[j];
     }
@@ -536,6 +547,7 @@ __global__ void __launch_bounds__(kSortBlock) onesweep_kernel(PassArgs a) {
     // (values are record indices; the bound only matters after a look-back
     // timeout, when a slot can hold a stale value)
     const bool vok = v < a.n_records;
+    if (!check(out < (uint64_t)n, kCheckSortSlot)) continue;
     a.kout[out] = k;
     a.vout[out] = v;
     if (a.tiles_out) a.tiles_out[out] = vok ? a.tiles_in[v] : 0;
@@ -579,7 +591,8 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* tk, const u
     const uint32_t v = tv[k];
     // (the bound only matters after a look-back timeout, when a slot can
     // hold a stale value)
-    keys[k] = ((uint64_t)tile << 32) | (v < n_records ? __float_as_uint(xyzo[v].z) : kInvisibleKey);
+    keys[k] = ((uint64_t)tile << 32) |
+              (check(v < n_records, kCheckRecordIndex) ? __float_as_uint(xyzo[v].z) : kInvisibleKey);
     if (tile >= (uint64_t)TT) continue;
     const uint32_t prev = k > 0 ? tk[k - 1] : ~0u;
     const uint32_t next = k + 1 < n ? tk[k + 1] : ~0u;
@@ -736,5 +749,7 @@ cudaError_t launch_emit_sort_ranges(const Records& rec, int64_t n, const DevCam&
   count_launches(launched);
   return cudaGetLastError();
 }
+
+uint32_t checked_status_binsort() { return take_checked_status(); }
 
 }  // namespace gs

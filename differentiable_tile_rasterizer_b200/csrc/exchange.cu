@@ -4,8 +4,10 @@
 // each projected Gaussian to the GPUs that own the screen tiles it touches).
 //
 // Rank r of G owns Gaussians g = r, r + G, r + 2G, ... (local record l is
-// global Gaussian l G + r) and the tile rows [band(r), band(r + 1)),
-// band(q) = floor(q TH / G). Kernels here, per rank:
+// global Gaussian l G + r) and the tile rows [band(r), band(r + 1)) of a
+// partition of the TH tile rows into G bands in rank order: by default
+// band(q) = floor(q TH / G), or bounds the caller chose (for instance from
+// the measured work per tile row). Kernels here, per rank:
 //   route     which bands each visible local record reaches, and its slot in
 //             the send buffer of each (records stay in local, hence global,
 //             order within a destination);
@@ -31,21 +33,19 @@ namespace {
 
 constexpr int kRouteBlock = 256;
 
-__device__ __forceinline__ int band_start(int q, int G, int TH) { return (int)(((int64_t)q * TH) / G); }
-
 // Mask of the bands that the rect rows [y0, y1) reach (bit q).
-__device__ __forceinline__ uint32_t band_mask(int y0, int y1, int G, int TH) {
+__device__ __forceinline__ uint32_t band_mask(int y0, int y1, int G, const BandStarts& b) {
   uint32_t m = 0;
   for (int q = 0; q < G; ++q)
-    if (y0 < band_start(q + 1, G, TH) && y1 > band_start(q, G, TH)) m |= 1u << q;
+    if (y0 < b.row[q + 1] && y1 > b.row[q]) m |= 1u << q;
   return m;
 }
 
 // Per record: its band mask; per CTA: the count of records for every band
 // (cta_counts [n_ctas][G]).
 __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const ushort4* rect, const int32_t* tiles,
-                                                                  int64_t n, int G, int TH, uint32_t* mask,
-                                                                  uint32_t* cta_counts) {
+                                                                  int64_t n, int G, BandStarts bands,
+                                                                  uint32_t* mask, uint32_t* cta_counts) {
   __shared__ uint32_t s_cnt[kMaxRanks];
   if (threadIdx.x < kMaxRanks) s_cnt[threadIdx.x] = 0;
   __syncthreads();
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const ushort4*
   uint32_t m = 0;
   if (i < n && tiles[i] > 0) {
     const ushort4 r = rect[i];
-    m = band_mask(r.y, r.w, G, TH);
+    m = band_mask(r.y, r.w, G, bands);
   }
   if (i < n) mask[i] = m;
   for (int q = 0; q < G; ++q) {
@@ -65,17 +65,30 @@ __global__ void __launch_bounds__(kRouteBlock) route_count_kernel(const ushort4*
 }
 
 // Exclusive scan of cta_counts over CTAs for every band (one thread per
-// band, sequential: G <= 32 bands and a few thousand CTAs), and the totals.
-__global__ void route_scan_kernel(uint32_t* cta_counts, int64_t n_ctas, int G, int64_t* totals) {
+// band, sequential: G <= 32 bands and a few thousand CTAs), the totals, and
+// (dst_off non-null) their exclusive scan: each destination's first slot in
+// the send buffer, so the pack needs no host round trip.
+__global__ void route_scan_kernel(uint32_t* cta_counts, int64_t n_ctas, int G, int64_t* totals,
+                                  int64_t* dst_off) {
   const int q = threadIdx.x;
-  if (q >= G) return;
   int64_t run = 0;
-  for (int64_t c = 0; c < n_ctas; ++c) {
-    const uint32_t v = cta_counts[c * G + q];
-    cta_counts[c * G + q] = (uint32_t)run;
-    run += v;
+  if (q < G) {
+    for (int64_t c = 0; c < n_ctas; ++c) {
+      const uint32_t v = cta_counts[c * G + q];
+      cta_counts[c * G + q] = (uint32_t)run;
+      run += v;
+    }
+    totals[q] = run;
   }
-  totals[q] = run;
+  if (dst_off) {
+    int64_t x = q < G ? run : 0;  // inclusive warp scan of the totals
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (q >= o) x += y;
+    }
+    if (q < G) dst_off[q] = x - run;
+  }
 }
 
 // Writes record i to slot dst_off[q] + (its rank among the records for band
@@ -177,11 +190,12 @@ __global__ void __launch_bounds__(256) return_grad_kernel(const float4* ret, con
 
 int64_t route_ctas(int64_t n) { return (n + kRouteBlock - 1) / kRouteBlock; }
 
-cudaError_t launch_route_count(const Records& rec, int64_t n, int G, int TH, uint32_t* mask, uint32_t* cta_counts,
-                               int64_t* totals, cudaStream_t s) {
+cudaError_t launch_route_count(const Records& rec, int64_t n, int G, const BandStarts& bands, uint32_t* mask,
+                               uint32_t* cta_counts, int64_t* totals, int64_t* dst_off, cudaStream_t s) {
   const int64_t nc = route_ctas(n);
-  if (nc > 0) route_count_kernel<<<(unsigned)nc, kRouteBlock, 0, s>>>(rec.rect, rec.tiles, n, G, TH, mask, cta_counts);
-  route_scan_kernel<<<1, 32, 0, s>>>(cta_counts, nc, G, totals);
+  if (nc > 0)
+    route_count_kernel<<<(unsigned)nc, kRouteBlock, 0, s>>>(rec.rect, rec.tiles, n, G, bands, mask, cta_counts);
+  route_scan_kernel<<<1, 32, 0, s>>>(cta_counts, nc, G, totals, dst_off);
   count_launches(nc > 0 ? 2 : 1);
   return cudaGetLastError();
 }

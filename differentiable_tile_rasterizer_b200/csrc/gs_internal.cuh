@@ -82,9 +82,11 @@ int64_t kernel_launches();
 // preprocess.cu
 cudaError_t launch_preprocess(const Params& p, const DevCam& cam, const Records& out,
                               cudaStream_t s);
+// accumulate: add the visible records' chains to the gradient rows and touch
+// nothing else; otherwise overwrite every row (zero for culled and invisible).
 cudaError_t launch_preprocess_bwd(const Params& p, const uint8_t* mask, const DevCam& cam,
                                   const Records& in, const float4* grad2d, const Grads& g,
-                                  cudaStream_t s);
+                                  bool accumulate, cudaStream_t s);
 
 // cull.cu
 size_t cull_workspace_bytes(int64_t N);
@@ -128,9 +130,13 @@ struct WireRecord {   // 64 bytes on the wire
   uint2 pad;
 };
 static_assert(sizeof(WireRecord) == 64, "wire record layout");
+// First tile row of every rank's band (row[G] = tile rows), by value.
+struct BandStarts {
+  int32_t row[kMaxRanks + 1];
+};
 int64_t route_ctas(int64_t n);
-cudaError_t launch_route_count(const Records& rec, int64_t n, int G, int TH, uint32_t* mask, uint32_t* cta_counts,
-                               int64_t* totals, cudaStream_t s);
+cudaError_t launch_route_count(const Records& rec, int64_t n, int G, const BandStarts& bands, uint32_t* mask,
+                               uint32_t* cta_counts, int64_t* totals, int64_t* dst_off, cudaStream_t s);
 cudaError_t launch_route_pack(const Records& rec, const uint32_t* mask, int64_t n, int G, int rank,
                               const uint32_t* cta_offsets, const int64_t* dst_off, WireRecord* send,
                               int32_t* src_idx, cudaStream_t s);

@@ -9,6 +9,7 @@
 // Forward arithmetic follows the fixed fp32 specification step by step (the
 // step numbers match the CPU oracle's comments); the backward is plain fp32.
 
+#include "checked.cuh"
 #include "gs_device.cuh"
 #include "gs_internal.cuh"
 
@@ -237,7 +238,10 @@ __global__ void __launch_bounds__(256) preprocess_kernel(Params p, DevCam cam, R
   const int64_t na = p.n_active ? (int64_t)*p.n_active : p.N;
   Proj o;
   o.visible = false;
-  if (i < na) project<K>(PlaneSource{p, p.active_idx ? (int64_t)p.active_idx[i] : i}, cam, o);
+  if (i < na) {
+    const int64_t g = p.active_idx ? (int64_t)p.active_idx[i] : i;
+    if (check(g >= 0 && g < p.N, kCheckRecordIndex)) project<K>(PlaneSource{p, g}, cam, o);
+  }
   write_record(o, out, i);
 }
 
@@ -302,7 +306,23 @@ __device__ __forceinline__ void zero_grads(const Grads& gr, int64_t N, int K, in
   for (int k = 0; k < 3 * K; ++k) gr.d_sh[(int64_t)k * N + g] = 0.0f;
 }
 
-template <int K>
+// How the kernel writes the gradient rows.
+enum GradMode {
+  kWriteAll = 0,    // every row: the chain for visible records, zeros for culled and invisible ones
+  kPreZeroed = 1,   // the rows were zeroed by a memset first (a cull mask is given, so most rows are
+                    // zero and the memset writes them at copy bandwidth): visible records only
+  kAccumulate = 2,  // visible records' chains added to the rows; nothing else touched
+};
+
+template <int kMode>
+__device__ __forceinline__ void put_grad(float* p, float v) {
+  if (kMode == kAccumulate)
+    *p += v;
+  else
+    *p = v;
+}
+
+template <int K, int kMode>
 __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uint8_t* mask, DevCam cam,
                                                              Records rec, const float4* grad2d,
                                                              Grads gr) {
@@ -310,12 +330,13 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
   const int64_t N = p.N;
   if (i >= N) return;
   // Gaussian i culled by the active-set mask: its gradient is zero.
-  if (mask && mask[i] == 0) zero_grads(gr, N, K, i);
+  if (kMode == kWriteAll && mask && mask[i] == 0) zero_grads(gr, N, K, i);
   const int64_t na = p.n_active ? (int64_t)*p.n_active : N;
   if (i >= na) return;
   const int64_t g = p.active_idx ? (int64_t)p.active_idx[i] : i;
+  if (!check(g >= 0 && g < N, kCheckRecordIndex)) return;
   if (rec.tiles[i] <= 0) {
-    zero_grads(gr, N, K, g);
+    if (kMode == kWriteAll) zero_grads(gr, N, K, g);
     return;
   }
   const float4 g0 = grad2d[3 * i], g1 = grad2d[3 * i + 1], g2 = grad2d[3 * i + 2];
@@ -370,7 +391,7 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
   const float gpx = g0.x, gpy = g0.y, gop = g0.z, gA = g1.x, gB = g1.y, gC = g1.z;
   float g_mu[3], g_t[3];
   // opacity
-  gr.d_logits[g] = gop * op * (1.0f - op);
+  put_grad<kMode>(&gr.d_logits[g], gop * op * (1.0f - op));
   // colour
   const float dv[3] = {mu[0] - cam.campos[0], mu[1] - cam.campos[1], mu[2] - cam.campos[2]};
   const float nd = sqrtf(fmaf(dv[2], dv[2], fmaf(dv[1], dv[1], dv[0] * dv[0])));
@@ -390,7 +411,7 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
 #pragma unroll
       for (int ch = 0; ch < 3; ++ch) {
         const int64_t plane = (int64_t)(3 * k + ch) * N + g;
-        gr.d_sh[plane] = gv[ch] * Y[k];
+        put_grad<kMode>(&gr.d_sh[plane], gv[ch] * Y[k]);
         gY = fmaf(gv[ch], p.sh[plane], gY);
       }
 #pragma unroll
@@ -439,7 +460,7 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
       gs = fmaf(gM[3 * a + b], Rq[3 * a + b], gs);
       gR[3 * a + b] = gM[3 * a + b] * s[b];
     }
-    gr.d_log_scales[b * N + g] = gs * s[b];
+    put_grad<kMode>(&gr.d_log_scales[b * N + g], gs * s[b]);
   }
   const float gw = 2.f * (-z * gR[1] + y * gR[2] + z * gR[3] - x * gR[5] - y * gR[6] + x * gR[7]);
   const float gx = 2.f * (y * gR[1] + z * gR[2] + y * gR[3] - 2.f * x * gR[4] - w * gR[5] + z * gR[6] +
@@ -449,10 +470,10 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
   const float gz = 2.f * (-2.f * z * gR[0] - w * gR[1] + x * gR[2] + w * gR[3] - 2.f * z * gR[4] + y * gR[5] +
                           x * gR[6] + y * gR[7]);
   const float qdot = gw * w + gx * x + gy * y + gz * z;
-  gr.d_quats[g] = (gw - qdot * w) * inq;
-  gr.d_quats[N + g] = (gx - qdot * x) * inq;
-  gr.d_quats[2 * N + g] = (gy - qdot * y) * inq;
-  gr.d_quats[3 * N + g] = (gz - qdot * z) * inq;
+  put_grad<kMode>(&gr.d_quats[g], (gw - qdot * w) * inq);
+  put_grad<kMode>(&gr.d_quats[N + g], (gx - qdot * x) * inq);
+  put_grad<kMode>(&gr.d_quats[2 * N + g], (gy - qdot * y) * inq);
+  put_grad<kMode>(&gr.d_quats[3 * N + g], (gz - qdot * z) * inq);
   float gJ00 = 0.f, gJ02 = 0.f, gJ11 = 0.f, gJ12 = 0.f;
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
@@ -466,7 +487,7 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
   g_t[2] += -(fx * gJ00 + fy * gJ11) * itz2 + 2.f * (fx * t[0] * gJ02 + fy * t[1] * gJ12) * itz2 * itz;
 #pragma unroll
   for (int m = 0; m < 3; ++m)
-    gr.d_means[m * N + g] = g_mu[m] + g_t[0] * W[m] + g_t[1] * W[3 + m] + g_t[2] * W[6 + m];
+    put_grad<kMode>(&gr.d_means[m * N + g], g_mu[m] + g_t[0] * W[m] + g_t[1] * W[3 + m] + g_t[2] * W[6 + m]);
 }
 
 }  // namespace
@@ -497,19 +518,44 @@ cudaError_t launch_preprocess_multiview(const Params& p, const MultiViewArgs& mv
   return cudaGetLastError();
 }
 
-cudaError_t launch_preprocess_bwd(const Params& p, const uint8_t* mask, const DevCam& cam,
-                                  const Records& in, const float4* grad2d, const Grads& g,
-                                  cudaStream_t s) {
-  if (p.N == 0) return cudaSuccess;
+namespace {
+template <int kMode>
+void launch_chain(const Params& p, const uint8_t* mask, const DevCam& cam, const Records& in,
+                  const float4* grad2d, const Grads& g, cudaStream_t s) {
   const unsigned grid = grid_for(p.N, 256);
   switch (p.sh_degree) {
-    case 0: preprocess_bwd_kernel<1><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
-    case 1: preprocess_bwd_kernel<4><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
-    case 2: preprocess_bwd_kernel<9><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
-    default: preprocess_bwd_kernel<16><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
+    case 0: preprocess_bwd_kernel<1, kMode><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
+    case 1: preprocess_bwd_kernel<4, kMode><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
+    case 2: preprocess_bwd_kernel<9, kMode><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
+    default: preprocess_bwd_kernel<16, kMode><<<grid, 256, 0, s>>>(p, mask, cam, in, grad2d, g); break;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_preprocess_bwd(const Params& p, const uint8_t* mask, const DevCam& cam,
+                                  const Records& in, const float4* grad2d, const Grads& g,
+                                  bool accumulate, cudaStream_t s) {
+  if (p.N == 0) return cudaSuccess;
+  const int K = (p.sh_degree + 1) * (p.sh_degree + 1);
+  if (accumulate) {
+    launch_chain<kAccumulate>(p, mask, cam, in, grad2d, g, s);
+  } else if (mask) {  // most rows are culled: zero everything at copy bandwidth first
+    const size_t row = (size_t)p.N * sizeof(float);
+    const size_t planes[5] = {3, 3, 4, 1, (size_t)3 * K};
+    float* dst[5] = {g.d_means, g.d_log_scales, g.d_quats, g.d_logits, g.d_sh};
+    for (int k = 0; k < 5; ++k) {
+      const cudaError_t e = cudaMemsetAsync(dst[k], 0, planes[k] * row, s);
+      if (e != cudaSuccess) return e;
+    }
+    launch_chain<kPreZeroed>(p, mask, cam, in, grad2d, g, s);
+  } else {
+    launch_chain<kWriteAll>(p, mask, cam, in, grad2d, g, s);
   }
   count_launches(1);
   return cudaGetLastError();
 }
+
+uint32_t checked_status_preprocess() { return take_checked_status(); }
 
 }  // namespace gs

@@ -15,6 +15,7 @@
 // backward recomputes alpha with the same operations, so its skip decisions
 // match the forward's exactly, and recovers T by division.
 
+#include "checked.cuh"
 #include "gs_device.cuh"
 #include "gs_internal.cuh"
 
@@ -41,6 +42,8 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+// cp.async groups: wait until at most one (the newest) is still in flight.
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // Pixel of thread `tid` in the tile: warp w covers the 8x4 block at
 // ((w & 1) * 8, (w >> 1) * 4).
@@ -70,6 +73,17 @@ __device__ __forceinline__ void tile_pixel(int tid, int& du, int& dv) {
 // m01 / m11, pad, 0). An empty box (negative half-widths) if the Gaussian
 // can never blend, an unbounded one if (M - sl I) is not safely positive
 // definite.
+// The region's square roots and quotients use the hardware approximations
+// (sqrt.approx, div.approx: a few ulp, ~1e-6 relative at most) instead of
+// correctly rounded ones: the box is widened by 2% and the threshold by 1%,
+// four orders of magnitude more than those errors, and the minimum of the
+// quadratic form moves only to second order with the edge point the ratios
+// give, so the region stays conservative.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float r;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 struct BlendRegion {
   float4 box;
   float4 q1;
@@ -88,14 +102,15 @@ __device__ __forceinline__ BlendRegion blend_region(float px, float py, float a2
   if (!(m00 > 0.0f) || !(m11 > 0.0f) || !(det > 1e-3f * (m00 * m11)))
     return BlendRegion{make_float4(px, py, kInf, kInf), make_float4(1.f, 0.f, 1.f, kInf), none};
   const float pad = 0.05f + 1e-6f * (fabsf(px) + fabsf(py));
-  const float hx = sqrtf(rho2 * m11 / det) * 1.02f + pad;
-  const float hy = sqrtf(rho2 * m00 / det) * 1.02f + pad;
+  const float idet = __fdividef(rho2, det);
+  const float hx = sqrt_approx(idet * m11) * 1.02f + pad;
+  const float hy = sqrt_approx(idet * m00) * 1.02f + pad;
   const float half_tr = 0.5f * (m00 + m11);
-  const float disc = sqrtf(0.25f * (m00 - m11) * (m00 - m11) + m01 * m01);
+  const float disc = sqrt_approx(0.25f * (m00 - m11) * (m00 - m11) + m01 * m01);
   const float lmin = half_tr - disc;
   const float thr = lmin > 0.01f * (half_tr + disc) ? rho2 * 1.01f : kInf;
   return BlendRegion{make_float4(px, py, hx, hy), make_float4(m00, m01, m11, thr),
-                     make_float4(m01 / m00, m01 / m11, pad, 0.f)};
+                     make_float4(__fdividef(m01, m00), __fdividef(m01, m11), pad, 0.f)};
 }
 
 // Can the Gaussian blend at a pixel centre of the warp block with centre
@@ -202,7 +217,7 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   // centre of this warp's 8x4 block of pixel centres
   const float wcx = block_cx(tx0, warp), wcy = block_cy(ty0, warp);
   const uint2 range = a.ranges[tile];
-  const int n = (int)(range.y - range.x);
+  const int n = check(range.y >= range.x, kCheckTileRange) ? (int)(range.y - range.x) : 0;
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int cnt = 0, lst = 0;
   bool done = !inside;
@@ -353,6 +368,167 @@ __global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
   }
 }
 
+// Zeroes the hit bytes of every tile's list entries ([range.x, range.y) of
+// each tile, one CTA per tile) before a forward whose warps OR their bits in.
+__global__ void __launch_bounds__(256) zero_hits_kernel(const uint2* ranges, uint8_t* hits) {
+  const uint2 r = ranges[blockIdx.x];
+  for (uint32_t k = r.x + threadIdx.x; k < r.y; k += 256) hits[k] = 0;
+}
+
+// Forward with one warp per CTA and no CTA barrier: warp w of a tile (CTA
+// 4 slot + w) owns the 8x8 pixel block at ((w & 1) * 8, (w >> 1) * 8), lane l
+// its pixels (l & 7, l >> 3) and (l & 7, (l >> 3) + 4), both run as packed
+// fp32 pairs (each half rounded as the scalar operation, so every pixel's
+// values are those of the specification). The warp walks its tile's list
+// front to back in chunks of 32 entries (lane l: entry 32 c + l): the
+// entries' records arrive by cp.async in the warp's own double-buffered
+// slots, one chunk ahead, and their indices two chunks ahead. Each lane tests
+// its entry's blend region against the warp's block; the warp then blends the
+// entries that can reach it, in list order. A warp leaves as soon as its 64
+// pixels have stopped, independently of the tile's other blocks.
+// Hit bytes: bit f (pixel rows 0-3 of the block, the 8x4 block f of the
+// eight-warp layout) and bit f + 2 (rows 4-7), f = (w & 1) | (w >> 1) << 2,
+// are OR-ed into the entry's byte with one word atomic per 4 entries; the
+// bytes are zeroed first (zero_hits_kernel).
+// kFwdWarps independent warps per CTA (blocks of the same tile, sharing
+// nothing): more resident warps than one-warp CTAs allow (32 per SM), within
+// the register bound below.
+constexpr int kFwdWarps = 2;
+static_assert(4 % kFwdWarps == 0, "a tile's four blocks split evenly over the CTAs");
+__global__ void __launch_bounds__(32 * kFwdWarps, 18) raster_fwd_warp_kernel(FwdArgs a) {
+  __shared__ float4 s_raw_all[kFwdWarps][2][3][32];  // per warp: xyzo, conic, rgb of two chunks of entries
+  const int lane = threadIdx.x & 31;
+  float4(*s_raw)[3][32] = s_raw_all[threadIdx.x >> 5];
+  const int64_t gw = (int64_t)blockIdx.x * kFwdWarps + (threadIdx.x >> 5);  // (tile slot, 8x8 block)
+  const uint32_t slot4 = (uint32_t)(gw >> 2);
+  const int warp = (int)(gw & 3);
+  const uint32_t tile_u = a.order ? a.order[slot4] : slot4;
+  if (tile_u >= gridDim.x * (uint32_t)kFwdWarps / 4u) return;  // not a tile: a schedule that is no permutation
+  const int tile = (int)tile_u;
+  const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
+  const int u = tx0 + (warp & 1) * 8 + (lane & 7), v0 = ty0 + (warp >> 1) * 8 + (lane >> 3);
+  const bool in0 = u < a.W && v0 < a.H, in1 = u < a.W && v0 + 4 < a.H;
+  const float xc = __fadd_rn((float)u, 0.5f);
+  const float2 yc = make_float2(__fadd_rn((float)v0, 0.5f), __fadd_rn((float)(v0 + 4), 0.5f));
+  const float bcx = (float)(tx0 + (warp & 1) * 8) + 4.0f, bcy = (float)(ty0 + (warp >> 1) * 8) + 4.0f;
+  const uint2 range = a.ranges[tile];
+  const int n = check(range.y >= range.x, kCheckTileRange) ? (int)(range.y - range.x) : 0;
+  const int f = (warp & 1) | ((warp >> 1) << 2);
+  float2 T = make_float2(1.0f, 1.0f), C0 = make_float2(0.f, 0.f), C1 = C0, C2 = C0;
+  int cnt0 = 0, cnt1 = 0, lst0 = 0, lst1 = 0;
+  bool done0 = !in0, done1 = !in1;
+  const uint32_t* lv = a.vals + range.x;
+  auto meta = [&](int c) { return 32 * c + lane < n ? lv[32 * c + lane] : 0u; };
+  auto fetch = [&](int buf, int c, uint32_t idx) {
+    if (32 * c + lane < n) {
+      cp_async16(&s_raw[buf][0][lane], a.xyzo + idx);
+      cp_async16(&s_raw[buf][1][lane], a.conic + idx);
+      cp_async16(&s_raw[buf][2][lane], a.rgb + idx);
+    }
+    cp_async_commit();
+  };
+  const int nchunks = (n + 31) >> 5;
+  uint32_t i_cur = meta(0);
+  fetch(0, 0, i_cur);
+  uint32_t i_nxt = meta(1);
+  for (int c = 0; c < nchunks; ++c) {
+    if (__all_sync(0xffffffffu, done0 && done1)) break;
+    const int buf = c & 1;
+    fetch(buf ^ 1, c + 1, i_nxt);  // chunk c + 1 in flight (its buffer was released after chunk c - 1)
+    i_cur = i_nxt;
+    i_nxt = meta(c + 2);
+    cp_async_wait_1();  // this lane's copies of chunk c have landed
+    __syncwarp();       // and every lane's
+    const int j = 32 * c + lane;
+    bool rel = false;
+    if (j < n) {
+      const float4 g = s_raw[buf][0][lane];
+      const float4 q = s_raw[buf][1][lane];
+      const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
+                  c2 = __fmul_rn(q.z, kHalfNegLog2e);
+      const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
+      rel = region_hits(r.box, r.q1, r.q2, bcx, bcy, 3.5f, 3.5f);
+      s_raw[buf][1][lane] = make_float4(a2, b2, c2, 0.0f);  // the scaled conic, once per entry
+    }
+    unsigned msk = __ballot_sync(0xffffffffu, rel);
+    __syncwarp();                 // the scaled conics are visible to every lane
+    uint32_t bl0 = 0u, bl1 = 0u;  // bit k: entry 32 c + k blended at this lane's pixel 0 / 1
+    while (msk) {
+      const int k = __ffs(msk) - 1;
+      msk &= msk - 1;
+      const float4 g = s_raw[buf][0][k];
+      const float4 q = s_raw[buf][1][k];
+      const float a2 = q.x, b2 = q.y, c2 = q.z;
+      const float dx = __fsub_rn(g.x, xc);
+      const float2 dy = sub2(splat2(g.y), yc);
+      const float2 qv = fma2(splat2(b2), dy, splat2(__fmul_rn(a2, dx)));
+      float2 p2 = mul2(splat2(dx), qv);
+      p2 = fma2(mul2(splat2(c2), dy), dy, p2);
+      const float2 e = exp2_raster2(p2);
+      const float2 va = mul2(splat2(g.w), e);
+      const float al0 = fminf(va.x, kAlphaMax), al1 = fminf(va.y, kAlphaMax);
+      // a pixel that skips the entry or has stopped blends with alpha 0, which
+      // leaves its colour, T and counts exactly as they were
+      const bool b0 = !done0 && al0 >= kAlphaMin, b1 = !done1 && al1 >= kAlphaMin;
+      if (!__any_sync(0xffffffffu, b0 || b1)) continue;
+      const float4 col = s_raw[buf][2][k];
+      const float2 ab = make_float2(b0 ? al0 : 0.0f, b1 ? al1 : 0.0f);
+      const float2 wgt = mul2(ab, T);
+      C0 = fma2(wgt, splat2(col.x), C0);
+      C1 = fma2(wgt, splat2(col.y), C1);
+      C2 = fma2(wgt, splat2(col.z), C2);
+      T = mul2(T, sub2(splat2(1.0f), ab));
+      done0 = done0 || T.x < kTMin;
+      done1 = done1 || T.y < kTMin;
+      bl0 |= (b0 ? 1u : 0u) << k;
+      bl1 |= (b1 ? 1u : 0u) << k;
+    }
+    // contributor counts and last blends of the chunk, from its blend masks
+    cnt0 += __popc(bl0);
+    cnt1 += __popc(bl1);
+    if (bl0) lst0 = 32 * c + (32 - __clz(bl0));
+    if (bl1) lst1 = 32 * c + (32 - __clz(bl1));
+    if (a.hits) {
+      // lane k: the byte bits of entry 32 c + k; one atomic OR per 4 entries
+      const uint32_t h0 = __reduce_or_sync(0xffffffffu, bl0), h1 = __reduce_or_sync(0xffffffffu, bl1);
+      const uint32_t e = range.x + (uint32_t)j;  // global entry index
+      uint32_t byte = (((h0 >> lane) & 1u) << f) | (((h1 >> lane) & 1u) << (f + 2));
+      if (j >= n) byte = 0u;
+      uint32_t word = byte << (8 * (e & 3u));
+#pragma unroll
+      for (int d = 1; d < 4; ++d) {  // the following lanes of the same 4-entry word
+        const uint32_t o = __shfl_down_sync(0xffffffffu, word, d);
+        const uint32_t oe = __shfl_down_sync(0xffffffffu, e, d);
+        if (lane + d < 32 && (oe >> 2) == (e >> 2)) word |= o;
+      }
+      const bool leads = lane == 0 || (e & 3u) == 0u;
+      if (leads && word != 0u && j < n)
+        atomicOr(reinterpret_cast<unsigned int*>(a.hits + (e & ~3u)), word);
+    }
+    __syncwarp();  // every lane is done with buffer buf before it is refilled
+  }
+  cp_async_wait_all();  // no copy outlives the CTA
+  const size_t P = (size_t)a.W * a.H;
+  if (in0) {
+    const size_t pix = (size_t)v0 * a.W + u;
+    a.image[pix] = __fmaf_rn(T.x, a.bg0, C0.x);
+    a.image[P + pix] = __fmaf_rn(T.x, a.bg1, C1.x);
+    a.image[2 * P + pix] = __fmaf_rn(T.x, a.bg2, C2.x);
+    a.final_T[pix] = T.x;
+    a.n_contrib[pix] = cnt0;
+    a.last[pix] = lst0;
+  }
+  if (in1) {
+    const size_t pix = (size_t)(v0 + 4) * a.W + u;
+    a.image[pix] = __fmaf_rn(T.y, a.bg0, C0.y);
+    a.image[P + pix] = __fmaf_rn(T.y, a.bg1, C1.y);
+    a.image[2 * P + pix] = __fmaf_rn(T.y, a.bg2, C2.y);
+    a.final_T[pix] = T.y;
+    a.n_contrib[pix] = cnt1;
+    a.last[pix] = lst1;
+  }
+}
+
 struct BwdArgs {
   const float4* xyzo;
   const float4* conic;
@@ -367,6 +543,7 @@ struct BwdArgs {
   const float* dL_dimage;
   float4* grad2d;  // [n][3]
   const uint8_t* hits;  // [entries] from the forward, or null
+  int64_t n_records;    // records (bound of the list values)
 };
 
 // Where the multi-value butterfly below leaves its results: lane `lane` ends
@@ -495,7 +672,10 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
   // of the next batch are copied into s_raw while this one is processed and
   // the indices of the batch after it are loaded into a register.
   const uint32_t* lv = a.vals + range.x;
-  auto index_of = [&](int d) { return n - 1 - d - tid >= 0 ? lv[n - 1 - d - tid] : 0u; };
+  auto index_of = [&](int d) {
+    const uint32_t i = n - 1 - d - tid >= 0 ? lv[n - 1 - d - tid] : 0u;
+    return check(i < (uint64_t)a.n_records, kCheckRecordIndex) ? i : 0u;
+  };
   auto fetch = [&](int d, uint32_t i) {
     if (n - 1 - d - tid >= 0) {
       cp_async16(&s_raw[0][tid], a.xyzo + i);
@@ -628,8 +808,6 @@ __global__ void __launch_bounds__(kBlockB, 8) raster_bwd_kernel(BwdArgs a) {
 constexpr int kHitsWarps = 1;
 static_assert(4 % kHitsWarps == 0, "a tile's four blocks split evenly over the CTAs");
 
-// cp.async groups: wait until at most one (the newest) is still in flight.
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
 // Backward with the forward's hit bytes: warp w (the 8x8 block of forward
 // warps f and f + 2, f = (w & 1) | (w >> 1) << 2) walks its own list
@@ -670,7 +848,7 @@ __global__ void __launch_bounds__(32 * kHitsWarps) raster_bwd_hits_kernel(BwdArg
     const bool in = off >= 0;
     const uint32_t b = in ? (uint32_t)hb[off] : 0u;
     idx = in ? lv[off] : 0u;
-    hit = (b & fbits) != 0u;
+    hit = (b & fbits) != 0u && check(idx < (uint64_t)a.n_records, kCheckRecordIndex);
   };
   auto fetch = [&](int buf, uint32_t idx, bool hit) {
     if (hit) {
@@ -784,11 +962,18 @@ cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const ui
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.image = image; a.final_T = final_T; a.n_contrib = n_contrib; a.last = last;
   a.importance = importance; a.active_idx = active_idx; a.hits = hits;
-  if (importance)
-    raster_fwd_kernel<true><<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
-  else
-    raster_fwd_kernel<false><<<cam.TW * cam.TH, kBlock, 0, s>>>(a);
-  count_launches(1);
+  const int TT = cam.TW * cam.TH;
+  int launched = 1;
+  if (importance) {
+    raster_fwd_kernel<true><<<TT, kBlock, 0, s>>>(a);
+  } else {
+    if (hits) {
+      zero_hits_kernel<<<TT, 256, 0, s>>>(a.ranges, hits);
+      ++launched;
+    }
+    raster_fwd_warp_kernel<<<TT * 4 / kFwdWarps, 32 * kFwdWarps, 0, s>>>(a);
+  }
+  count_launches(launched);
   return cudaGetLastError();
 }
 
@@ -804,6 +989,7 @@ cudaError_t launch_raster_bwd(const Records& rec, const uint32_t* vals, const ui
   a.W = cam.width; a.H = cam.height; a.TW = cam.TW;
   a.bg0 = bg[0]; a.bg1 = bg[1]; a.bg2 = bg[2];
   a.final_T = final_T; a.last = last; a.dL_dimage = dL_dimage; a.grad2d = grad2d; a.hits = hits;
+  a.n_records = n_records;
   if (hits)
     raster_bwd_hits_kernel<<<cam.TW * cam.TH * 4 / kHitsWarps, 32 * kHitsWarps, 0, s>>>(a);
   else
@@ -818,5 +1004,7 @@ cudaError_t launch_tile_order(const uint32_t* ranges, int64_t TT, uint32_t* orde
   count_launches(1);
   return cudaGetLastError();
 }
+
+uint32_t checked_status_raster() { return take_checked_status(); }
 
 }  // namespace gs

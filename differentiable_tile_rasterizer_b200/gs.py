@@ -28,7 +28,9 @@ EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_pr
             "gs_quant_decode", "gs_adam_sh_quant", "gs_route_ctas", "gs_route_count", "gs_route_pack",
             "gs_merge_received", "gs_unmerge_grad2d", "gs_return_grad2d",
             "gs_rasterize_fwd", "gs_rasterize_fwd_importance", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
-            "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_cull_noalloc"]
+            "gs_preprocess_bwd_accumulate",
+            "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_debug_is_checked_build",
+            "gs_debug_checked_status", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
 GS_MAX_VIEWS = 16
 GS_WIRE_RECORD_BYTES = 64
@@ -69,18 +71,21 @@ PPROJ = ctypes.POINTER(GsProjected)
 
 
 def lib_path() -> str:
-    return _build.LIB
+    """libgs.so, or its checked build (device-side bounds checks) when the
+    environment sets GS_CHECKED=1."""
+    return _build.LIB_CHECKED if os.environ.get("GS_CHECKED") == "1" else _build.LIB
 
 
 def load(build_if_missing: bool = True) -> ctypes.CDLL:
     """Load libgs.so (building it first if it is absent and nvcc is available)."""
     global _LIB
     if _LIB is None:
-        if not os.path.exists(_build.LIB):
+        path = lib_path()
+        if not os.path.exists(path):
             if not build_if_missing:
-                raise OSError(f"libgs.so not built: {_build.LIB}")
-            _build.build()
-        L = ctypes.CDLL(_build.LIB)
+                raise OSError(f"library not built: {path}")
+            _build.build(checked=path == _build.LIB_CHECKED)
+        L = ctypes.CDLL(path)
         L.gs_version.restype = ctypes.c_int
         L.gs_status_string.restype = ctypes.c_char_p
         L.gs_status_string.argtypes = [ctypes.c_int]
@@ -93,7 +98,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_adam_sh_quant.argtypes = [P, I64, I64, P, P, P, P, P, P, ctypes.POINTER(GsAdamConfig), P]
         L.gs_route_ctas.argtypes = [I64]
         L.gs_route_ctas.restype = ctypes.c_int64
-        L.gs_route_count.argtypes = [PPROJ, I64, ctypes.c_int, ctypes.c_int, P, P, P, P]
+        L.gs_route_count.argtypes = [PPROJ, I64, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P]
         L.gs_route_pack.argtypes = [PPROJ, P, I64, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
         L.gs_merge_received.argtypes = [P, P, ctypes.c_int, I64, ctypes.c_int, ctypes.c_int, PPROJ, P, P]
         L.gs_unmerge_grad2d.argtypes = [P, P, I64, P, P]
@@ -108,17 +113,23 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_preprocess_bwd.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, P, PCAM, PPROJ, P,
                                         P, P, P, P, P, P]
         L.gs_rasterize_bwd_2d.argtypes = [PPROJ, I64, P, P, P, P, PCAM, P, P, P, P, P, P]
+        L.gs_preprocess_bwd_accumulate.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, PCAM, PPROJ, P,
+                                                   P, P, P, P, P, P]
         L.gs_cull_noalloc.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P]
         L.gs_cull_noalloc.restype = ctypes.c_int
         L.gs_debug_kernel_launches.restype = ctypes.c_int64
         L.gs_debug_kernel_launches.argtypes = []
         L.gs_debug_set_stalled_sort_tile.argtypes = [I64]
         L.gs_debug_set_stalled_sort_tile.restype = None
+        L.gs_debug_is_checked_build.restype = ctypes.c_int
+        L.gs_debug_is_checked_build.argtypes = []
+        L.gs_debug_checked_status.restype = ctypes.c_uint32
+        L.gs_debug_checked_status.argtypes = []
         for name in ["gs_cull", "gs_preprocess", "gs_preprocess_multiview", "gs_bin_sort", "gs_accumulate_grad2d_norm",
                      "gs_quant_encode", "gs_quant_decode", "gs_adam_sh_quant", "gs_route_count", "gs_route_pack",
                      "gs_merge_received", "gs_unmerge_grad2d", "gs_return_grad2d", "gs_bin_sort_async", "gs_rasterize_fwd",
                      "gs_rasterize_fwd_importance",
-                     "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd"]:
+                     "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd", "gs_preprocess_bwd_accumulate"]:
             getattr(L, name).restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -228,9 +239,15 @@ def gs_adam_sh_quant(grad, U, N, pc, pb, mc, mb, vc, vb, lr, beta1, beta2, eps, 
         _stream(stream)))
 
 
-def gs_route_count(rec: GsProjected, n, n_ranks, tiles_y, mask, cta_counts, totals, stream=None):
-    _check("gs_route_count", load().gs_route_count(ctypes.byref(rec), int(n), int(n_ranks), int(tiles_y), _p(mask),
-                                                   _p(cta_counts), _p(totals), _stream(stream)))
+def gs_route_count(rec: GsProjected, n, n_ranks, tiles_y, mask, cta_counts, totals, band_starts=None,
+                   dst_offsets=None, stream=None):
+    """band_starts: host sequence of n_ranks + 1 tile rows (None: equal bands)."""
+    bs = None
+    if band_starts is not None:
+        bs = (ctypes.c_int32 * len(band_starts))(*[int(v) for v in band_starts])
+    _check("gs_route_count", load().gs_route_count(ctypes.byref(rec), int(n), int(n_ranks), int(tiles_y),
+                                                   bs, _p(mask), _p(cta_counts), _p(totals), _p(dst_offsets),
+                                                   _stream(stream)))
 
 
 def gs_route_pack(rec: GsProjected, mask, n, n_ranks, rank, cta_offsets, dst_offsets, send, src_idx, stream=None):
@@ -347,5 +364,23 @@ def gs_preprocess_bwd(means, log_scales, quats, opacity_logits, sh, sh_degree, N
         _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
 
 
+def gs_preprocess_bwd_accumulate(means, log_scales, quats, opacity_logits, sh, sh_degree, N, active_idx, n_active,
+                                 cam: GsCamera, rec: GsProjected, grad2d, d_means, d_log_scales, d_quats,
+                                 d_opacity_logits, d_sh, stream=None):
+    _check("gs_preprocess_bwd_accumulate", load().gs_preprocess_bwd_accumulate(
+        _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
+        _p(active_idx), _p(n_active), ctypes.byref(cam), ctypes.byref(rec), _p(grad2d),
+        _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
+
+
 def gs_debug_set_stalled_sort_tile(tile: int):
     load().gs_debug_set_stalled_sort_tile(int(tile))
+
+
+def gs_debug_is_checked_build() -> bool:
+    return bool(load().gs_debug_is_checked_build())
+
+
+def gs_debug_checked_status() -> int:
+    """First failed device-side check since the last call (0: none)."""
+    return int(load().gs_debug_checked_status())

@@ -14,8 +14,9 @@ is a libgs call; this module only sizes buffers and moves them between the
 calls.
 """
 
-from typing import List, Optional
+from typing import List, Optional, Sequence
 
+import numpy as np
 import torch
 
 from . import gs
@@ -25,8 +26,47 @@ WIRE = gs.GS_WIRE_RECORD_BYTES
 
 
 def band_rows(rank: int, world: int, tiles_y: int):
-    """Tile rows [lo, hi) owned by `rank`."""
+    """Tile rows [lo, hi) owned by `rank` with equal bands."""
     return rank * tiles_y // world, (rank + 1) * tiles_y // world
+
+
+def equal_bands(world: int, tiles_y: int) -> List[int]:
+    """First tile row of every rank's band, and tiles_y: equal row counts."""
+    return [q * tiles_y // world for q in range(world + 1)]
+
+
+def balance_bands(row_cost: Sequence[float], world: int) -> List[int]:
+    """Band starts (world + 1 values, 0 .. len(row_cost)) of contiguous row
+    bands in rank order whose largest summed cost is the least any such
+    partition reaches: a binary search over that largest cost, each candidate
+    checked by filling rows greedily. The cost of a row is the work its
+    tiles take (for instance the list entries of its tiles in a previous
+    view). With no cost at all the bands are equal."""
+    cost = np.asarray(row_cost, dtype=np.float64)
+    TH = int(cost.size)
+    if world <= 1 or TH == 0 or not (cost.sum() > 0):
+        return equal_bands(world, TH)
+
+    def cuts(limit):
+        starts, acc = [0], 0.0
+        for r, c in enumerate(cost):
+            if acc + c > limit and acc > 0:
+                starts.append(r)
+                acc = 0.0
+            acc += c
+        return starts
+
+    lo, hi = float(cost.max()), float(cost.sum())
+    for _ in range(60):
+        mid = 0.5 * (lo + hi)
+        if len(cuts(mid)) <= world:
+            hi = mid
+        else:
+            lo = mid
+    starts = cuts(hi)
+    while len(starts) < world:  # fewer bands were needed: split the last rows off as empty bands
+        starts.append(TH)
+    return starts + [TH]
 
 
 def local_params(params: GaussianParams, rank: int, world: int) -> GaussianParams:
@@ -39,13 +79,13 @@ def local_params(params: GaussianParams, rank: int, world: int) -> GaussianParam
 
 class InterleavedRank:
     def __init__(self, n_local: int, sh_degree: int, width: int, height: int, rank: int, world: int,
-                 device=None, recv_capacity: Optional[int] = None):
+                 device=None, recv_capacity: Optional[int] = None, band_starts: Optional[Sequence[int]] = None):
         if not 1 <= world <= gs.GS_MAX_RANKS or not 0 <= rank < world:
             raise ValueError("bad rank / world")
         self.rank, self.world = rank, world
         self.dev = torch.device(device or "cuda")
         self.local = Rasterizer(n_local, sh_degree, width, height, device=self.dev)
-        self.row_lo, self.row_hi = band_rows(rank, world, self.local.TH)
+        self.set_bands(band_starts if band_starts is not None else equal_bands(world, self.local.TH))
         self.sh_degree, self.W, self.H = sh_degree, width, height
         self._band_cap = 0
         self.band: Optional[Rasterizer] = None
@@ -54,6 +94,25 @@ class InterleavedRank:
         self.mask = torch.empty(max(n_local, 1), dtype=torch.int32, device=self.dev)
         self.cta_counts = torch.empty(nc * world, dtype=torch.int32, device=self.dev)
         self.totals = torch.empty(world, dtype=torch.int64, device=self.dev)
+        self.dst_off = torch.empty(world, dtype=torch.int64, device=self.dev)
+
+    def set_bands(self, band_starts: Sequence[int]):
+        """The tile rows every rank owns (the same list on every rank)."""
+        b = [int(v) for v in band_starts]
+        if len(b) != self.world + 1 or b[0] != 0 or b[-1] != self.local.TH or any(
+                x > y for x, y in zip(b, b[1:])):
+            raise ValueError("band starts must rise from 0 to the tile rows, one band per rank")
+        self.bands = b
+        self.row_lo, self.row_hi = b[self.rank], b[self.rank + 1]
+
+    def band_row_costs(self) -> np.ndarray:
+        """List entries per tile row of this rank's band in the last render
+        (zero for the other rows): the work measure balance_bands takes."""
+        B = self.band
+        lens = (B.ranges[:, 1] - B.ranges[:, 0]).to(torch.int64).cpu().numpy().reshape(B.TH, B.TW)
+        out = np.zeros(B.TH, np.float64)
+        out[self.row_lo:self.row_hi] = lens[self.row_lo:self.row_hi].sum(axis=1)
+        return out
 
     def _ensure_band(self, n: int):
         if n <= self._band_cap:
@@ -63,27 +122,36 @@ class InterleavedRank:
         self._band_cap = cap
 
     # ---------------------------------------------------------------- forward
-    def project_and_pack(self, params: GaussianParams, cam, lod_dist=0.0):
-        """Preprocess the local Gaussians and pack the wire records for every
-        rank. Returns (send bytes [sum counts * 64] uint8, counts per rank)."""
+    def project(self, params: GaussianParams, cam):
+        """Preprocess the local Gaussians and route them to the bands: the
+        records per destination (self.totals) and their first slots in the
+        send buffer (self.dst_off) stay on the device."""
         c = cam if isinstance(cam, gs.GsCamera) else gs.camera(cam)
         L = self.local
         L.params, L.cam = params, c
         L.culled = False
         L.preprocess(params, c)
-        n = L.N
-        gs.gs_route_count(L._proj, n, self.world, L.TH, self.mask, self.cta_counts, self.totals)
-        counts = [int(v) for v in self.totals.cpu().tolist()]
-        offs = [0]
-        for v in counts:
-            offs.append(offs[-1] + v)
-        self.sent = offs[-1]
-        dst = torch.tensor(offs[:-1], dtype=torch.int64, device=self.dev)
+        gs.gs_route_count(L._proj, L.N, self.world, L.TH, self.mask, self.cta_counts, self.totals,
+                          band_starts=self.bands, dst_offsets=self.dst_off)
+
+    def pack(self, counts: List[int]) -> torch.Tensor:
+        """The wire records for every rank, given this rank's send counts (the
+        host copy of self.totals). Returns send bytes [sum counts * 64]."""
+        L = self.local
+        self.sent = int(sum(counts))
         send = torch.empty(max(self.sent, 1) * WIRE, dtype=torch.uint8, device=self.dev)
         self.src_idx = torch.empty(max(self.sent, 1), dtype=torch.int32, device=self.dev)
-        gs.gs_route_pack(L._proj, self.mask, n, self.world, self.rank, self.cta_counts, dst, send, self.src_idx)
-        self.send_counts = counts
-        return send[: self.sent * WIRE], counts
+        gs.gs_route_pack(L._proj, self.mask, L.N, self.world, self.rank, self.cta_counts, self.dst_off, send,
+                         self.src_idx)
+        self.send_counts = [int(v) for v in counts]
+        return send[: self.sent * WIRE]
+
+    def project_and_pack(self, params: GaussianParams, cam, lod_dist=0.0):
+        """project() and pack() with one host read of the counts. Returns
+        (send bytes [sum counts * 64] uint8, counts per rank)."""
+        self.project(params, cam)
+        counts = [int(v) for v in self.totals.cpu().tolist()]
+        return self.pack(counts), counts
 
     def receive_and_render(self, recv: torch.Tensor, recv_counts: List[int], cam, bg=(0.0, 0.0, 0.0)):
         """Merge the received records (one segment per source rank, in rank
@@ -134,31 +202,58 @@ class InterleavedRank:
 
 class DistExchange:
     """The two all-to-alls over a torch.distributed group: counts, then the
-    payload (wire records forward, gradient rows backward)."""
+    payload (wire records forward, gradient rows backward).
 
-    def __init__(self, group=None):
+    host_staging: the collectives run on host copies of the tensors (a gloo
+    group, whose all-to-all takes CPU tensors) and the results are copied back
+    to the device; otherwise they run on the device tensors (NCCL)."""
+
+    def __init__(self, group=None, host_staging: bool = False):
         import torch.distributed as dist
-        self.dist, self.group = dist, group
+        self.dist, self.group, self.host = dist, group, bool(host_staging)
 
     def counts(self, send_counts: List[int], device) -> List[int]:
-        s = torch.tensor(send_counts, dtype=torch.int64, device=device)
+        s = torch.tensor(send_counts, dtype=torch.int64, device="cpu" if self.host else device)
         r = torch.empty_like(s)
         self.dist.all_to_all_single(r, s, group=self.group)
         return [int(v) for v in r.cpu().tolist()]
 
+    def counts_from_device(self, totals: torch.Tensor):
+        """(send counts, receive counts) from this rank's device totals, with
+        a single host read: the counts are exchanged before they are read."""
+        s = totals.cpu() if self.host else totals
+        r = torch.empty_like(s)
+        self.dist.all_to_all_single(r, s, group=self.group)
+        both = torch.cat([s, r]).cpu().tolist()
+        n = len(both) // 2
+        return [int(v) for v in both[:n]], [int(v) for v in both[n:]]
+
+    def row_costs(self, local: np.ndarray) -> np.ndarray:
+        """The sum over ranks of their band row costs (each rank fills its rows)."""
+        t = torch.from_numpy(np.ascontiguousarray(local, np.float64))
+        if not self.host:
+            t = t.cuda()
+        self.dist.all_reduce(t, group=self.group)
+        return t.cpu().numpy()
+
     def payload(self, send: torch.Tensor, send_rows: List[int], recv_rows: List[int], row_elems: int):
-        out = torch.empty((sum(recv_rows) * row_elems,), dtype=send.dtype, device=send.device)
-        self.dist.all_to_all_single(out, send.reshape(-1), output_split_sizes=[r * row_elems for r in recv_rows],
+        src = send.reshape(-1)
+        dev = src.device
+        if self.host:
+            src = src.cpu()
+        out = torch.empty((sum(recv_rows) * row_elems,), dtype=src.dtype, device=src.device)
+        self.dist.all_to_all_single(out, src, output_split_sizes=[r * row_elems for r in recv_rows],
                                     input_split_sizes=[r * row_elems for r in send_rows], group=self.group)
-        return out
+        return out.to(dev) if self.host else out
 
 
 def render_distributed(rank_state: InterleavedRank, ex: DistExchange, params: GaussianParams, cam, bg,
                        dL_dimage: Optional[torch.Tensor] = None):
     """One view on this rank of a group: forward (and backward when dL_dimage
     is given). Returns (band image, local parameter gradients or None)."""
-    send, counts = rank_state.project_and_pack(params, cam)
-    recv_counts = ex.counts(counts, send.device)
+    rank_state.project(params, cam)
+    counts, recv_counts = ex.counts_from_device(rank_state.totals)  # the view's one host round trip
+    send = rank_state.pack(counts)
     recv = ex.payload(send, counts, recv_counts, WIRE)
     img = rank_state.receive_and_render(recv, recv_counts, cam, bg)
     if dL_dimage is None:

@@ -49,27 +49,27 @@ class GaussianParams:
         return {k: f(getattr(scene, k)) for k in ("means", "log_scales", "quats", "opacity_logits", "sh")}
 
 
-class _NoTimer:
+class _Stage:
+    """One stage of a view: an NVTX range named gs.<stage> (visible to
+    profilers that record NVTX) and, when a store is given, CUDA events
+    around the stage's launches."""
+
+    def __init__(self, name, store=None):
+        self.name, self.store = name, store
+
     def __enter__(self):
+        torch.cuda.nvtx.range_push("gs." + self.name)
+        if self.store is not None:
+            self.start = torch.cuda.Event(enable_timing=True)
+            self.end = torch.cuda.Event(enable_timing=True)
+            self.start.record()
         return self
 
     def __exit__(self, *a):
-        return False
-
-
-class _StageTimer:
-    def __init__(self, store):
-        self.store = store
-
-    def __enter__(self):
-        self.start = torch.cuda.Event(enable_timing=True)
-        self.end = torch.cuda.Event(enable_timing=True)
-        self.start.record()
-        return self
-
-    def __exit__(self, *a):
-        self.end.record()
-        self.store.append((self.start, self.end))
+        if self.store is not None:
+            self.end.record()
+            self.store.append((self.start, self.end))
+        torch.cuda.nvtx.range_pop()
         return False
 
 
@@ -152,9 +152,7 @@ class Rasterizer:
 
     def _timed(self, stage):
         ev = self.stage_events
-        if ev is None:
-            return _NoTimer()
-        return _StageTimer(ev.setdefault(stage, []))
+        return _Stage(stage, None if ev is None else ev.setdefault(stage, []))
 
     def _ensure_capacity(self, cap: int):
         if cap <= self.capacity:
@@ -162,7 +160,7 @@ class Rasterizer:
         cap = int(cap)
         self.keys = torch.empty(max(cap, 1), dtype=torch.int64, device=self.dev)
         self.vals = torch.empty(max(cap, 1), dtype=torch.int32, device=self.dev)
-        self.hit_bits = torch.empty(max(cap, 1), dtype=torch.uint8, device=self.dev)
+        self.hit_bits = torch.empty((max(cap, 1) + 3) // 4 * 4, dtype=torch.uint8, device=self.dev)
         probe = gs.GsCamera()
         probe.width, probe.height = self.W, self.H
         self.sort_ws = _u8(gs.gs_bin_sort_workspace(self.N, probe, cap), self.dev)
@@ -298,18 +296,36 @@ class Rasterizer:
         self.raster_fwd(c, self.bg)
         return self.image
 
-    def backward(self, dL_dimage: torch.Tensor) -> dict:
+    def backward(self, dL_dimage: torch.Tensor, accumulate_into: Optional[dict] = None) -> dict:
+        """Gradients of the last forward's view. Into self.grads (overwritten)
+        or, with accumulate_into (a dict of parameter-shaped float32 tensors,
+        zeroed by the caller before the first view), added to those: the
+        gradient of a loss summed over views. Accumulating calls on the same
+        tensors must run in order on one stream."""
         p, c = self.params, self.cam
         act = self.active_idx if self.culled else None
         na = self.n_active if self.culled else None
         mask = self.mask if self.culled else None
         g = self.grads
+        if accumulate_into is not None:
+            a = accumulate_into
+            with self._timed("raster_bwd"):
+                gs.gs_rasterize_bwd_2d(self._proj, self.N, self.vals, self.ranges, c, self.bg, self.final_T,
+                                       self.last, dL_dimage, self.grad2d, tile_order=self._order(),
+                                       hit_bits=self._hits_in())
+            with self._timed("preprocess_bwd"):
+                gs.gs_preprocess_bwd_accumulate(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh,
+                                                p.sh_degree, self.N, act, na, c, self._proj, self.grad2d,
+                                                a["means"], a["log_scales"], a["quats"], a["opacity_logits"],
+                                                a["sh"])
+            return a
         if self.stage_events is None:
-            gs.gs_rasterize_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
-                                self.N, act, na, mask, c, self._proj, self.vals, self.ranges, self.bg,
-                                self.final_T, self.last, dL_dimage, self.grad2d, g["means"],
-                                g["log_scales"], g["quats"], g["opacity_logits"], g["sh"],
-                                tile_order=self._order(), hit_bits=self._hits_in())
+            with _Stage("backward"):
+                gs.gs_rasterize_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
+                                    self.N, act, na, mask, c, self._proj, self.vals, self.ranges, self.bg,
+                                    self.final_T, self.last, dL_dimage, self.grad2d, g["means"],
+                                    g["log_scales"], g["quats"], g["opacity_logits"], g["sh"],
+                                    tile_order=self._order(), hit_bits=self._hits_in())
             return g
         # the same two parts as separate calls, so each can be timed
         with self._timed("raster_bwd"):
@@ -322,9 +338,36 @@ class Rasterizer:
                                  g["log_scales"], g["quats"], g["opacity_logits"], g["sh"])
         return g
 
+    def backward_2d(self, dL_dimage: torch.Tensor):
+        """Part 1 of backward(): the per-record 2-D gradients (self.grad2d)."""
+        with self._timed("raster_bwd"):
+            gs.gs_rasterize_bwd_2d(self._proj, self.N, self.vals, self.ranges, self.cam, self.bg, self.final_T,
+                                   self.last, dL_dimage, self.grad2d, tile_order=self._order(),
+                                   hit_bits=self._hits_in())
+
+    def backward_params(self, into: dict, accumulate: bool):
+        """Part 2 of backward(): parameter gradients from self.grad2d, written
+        into `into` (a dict of parameter-shaped float32 tensors), or added to
+        it when accumulate is set."""
+        p, c = self.params, self.cam
+        act = self.active_idx if self.culled else None
+        na = self.n_active if self.culled else None
+        with self._timed("preprocess_bwd"):
+            if accumulate:
+                gs.gs_preprocess_bwd_accumulate(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh,
+                                                p.sh_degree, self.N, act, na, c, self._proj, self.grad2d,
+                                                into["means"], into["log_scales"], into["quats"],
+                                                into["opacity_logits"], into["sh"])
+            else:
+                gs.gs_preprocess_bwd(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
+                                     self.N, act, na, self.mask if self.culled else None, c, self._proj,
+                                     self.grad2d, into["means"], into["log_scales"], into["quats"],
+                                     into["opacity_logits"], into["sh"])
+
     def work_counts(self) -> dict:
         """Per-view work of the last forward (device reductions, then one sync):
-        visible Gaussians V, instances I, forward-evaluated pairs E (pairs of a
+        active Gaussians A (N without a cull), visible Gaussians V, instances
+        I, forward-evaluated pairs E (pairs of a
         pixel and an entry of its tile's list up to the pixel's stop), backward
         pairs E_bwd (entries before each pixel's last blend) and blends B."""
         H, W = self.H, self.W
@@ -336,9 +379,11 @@ class Rasterizer:
         last = self.last.to(torch.int64)
         stopped = self.final_T < 1e-4
         E = torch.where(stopped, last, plen).sum()
+        A = self.n_active[0].to(torch.int64) if self.culled else torch.tensor(self.N, device=self.dev)
         out = torch.stack([(self.rec["tiles"] > 0).sum().to(torch.int64), E, last.sum(),
-                           self.n_contrib.to(torch.int64).sum()]).cpu().tolist()
-        return {"V": out[0], "I": self.n_instances, "E": out[1], "E_bwd": out[2], "B": out[3]}
+                           self.n_contrib.to(torch.int64).sum(), A]).cpu().tolist()
+        return {"V": out[0], "I": self.n_instances, "E": out[1], "E_bwd": out[2], "B": out[3], "A": out[4],
+                "culled": self.culled}
 
     def records_numpy(self) -> dict:
         r = {k: v.cpu().numpy() for k, v in self.rec.items()}
@@ -371,9 +416,7 @@ class MultiViewRenderer:
 
     def _timed(self, stage):
         ev = self.stage_events
-        if ev is None:
-            return _NoTimer()
-        return _StageTimer(ev.setdefault(stage, []))
+        return _Stage(stage, None if ev is None else ev.setdefault(stage, []))
 
     def forward(self, params: GaussianParams, bg=(0.0, 0.0, 0.0)) -> list:
         bg = tuple(float(b) for b in bg)

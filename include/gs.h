@@ -245,14 +245,22 @@ GS_API int gs_adam_sh_quant(const float* grad, int64_t U, int64_t N, uint16_t* v
  * is gs_route_ctas(n) * n_ranks). */
 GS_API int64_t gs_route_ctas(int64_t n);
 
-/* Which ranks each visible record (tiles_touched > 0) goes to.
+/* Which ranks each visible record (tiles_touched > 0) goes to: rank q owns
+ * the tile rows [band_starts[q], band_starts[q + 1]).
+ *   band_starts [host] [n_ranks + 1] i32: non-decreasing, from 0 to tiles_y
+ *               (else GS_ERR_INVALID_ARGUMENT); NULL: equal bands,
+ *               band_starts[q] = floor(q tiles_y / n_ranks)
  *   mask        [device] [n] u32 out: bit q = sent to rank q
  *   cta_counts  [device] [gs_route_ctas(n)][n_ranks] u32 out: per-CTA
  *               exclusive offsets within each destination
  *   totals      [device] [n_ranks] i64 out: records for each destination
+ *   dst_offsets [device] [n_ranks] i64 out, or NULL: the exclusive scan of
+ *               totals (each destination's first slot in gs_route_pack's
+ *               send buffer), so that the pack needs no host round trip
  * Asynchronous. */
-GS_API int gs_route_count(const gs_projected* rec, int64_t n, int n_ranks, int tiles_y, uint32_t* mask,
-                          uint32_t* cta_counts, int64_t* totals, void* stream);
+GS_API int gs_route_count(const gs_projected* rec, int64_t n, int n_ranks, int tiles_y, const int32_t* band_starts,
+                          uint32_t* mask, uint32_t* cta_counts, int64_t* totals, int64_t* dst_offsets,
+                          void* stream);
 
 /* Packs the records for every destination into send (wire records,
  * destination-major, each destination's records in ascending index);
@@ -379,14 +387,15 @@ GS_API int gs_tile_order(const uint32_t* tile_ranges, int64_t n_tiles, uint32_t*
  *   final_T      [device] [H][W] out
  *   n_contrib    [device] [H][W] i32 out: blended Gaussians
  *   last         [device] [H][W] i32 out: 1 + list offset of the last blend
- *   hit_bits     [device] [n_instances] u8 out, or NULL: one byte per sorted
- *                list entry (indexed as vals); bit f set when the entry
- *                blended at some pixel of the 8x4 block f of its tile (block
- *                f at column (f & 1) * 8, row (f >> 1) * 4), clear otherwise.
- *                The backward's input of the same name. Written at least for
- *                every entry up to each tile's last blend; entries after the
- *                point where all of a tile's pixels stopped may be left as
- *                they were.
+ *   hit_bits     [device] [n_instances rounded up to a multiple of 4] u8
+ *                out, or NULL: one byte per sorted list entry (indexed as
+ *                vals); bit f set when the entry blended at some pixel of the
+ *                8x4 block f of its tile (block f at column (f & 1) * 8, row
+ *                (f >> 1) * 4), clear otherwise. Every entry of every tile's
+ *                list is written. The bits are OR-ed in with 32-bit atomics,
+ *                so the pointer must be 4-byte aligned (else
+ *                GS_ERR_INVALID_ARGUMENT). The backward's input of the same
+ *                name.
  * Asynchronous. */
 GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
                             const uint32_t* tile_ranges, const uint32_t* tile_order,
@@ -466,9 +475,38 @@ GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const 
                              const float* grad2d, float* d_means, float* d_log_scales,
                              float* d_quats, float* d_opacity_logits, float* d_sh, void* stream);
 
+/* gs_preprocess_bwd that adds instead of overwriting: each visible record's
+ * parameter gradient is added to its Gaussian's rows of d_* (read-modify-
+ * write); rows of culled Gaussians and invisible records are not touched.
+ * The gradient of a loss summed over several views is the sum of the views'
+ * gradients, so a multi-view training step calls this once per view on
+ * gradients it zeroed once (the problem statement's matching backward pass,
+ * applied per view). Same arguments as gs_preprocess_bwd without the mask;
+ * active_idx / n_active select the records as there. Calls that add into the
+ * same rows must not overlap on the GPU (they would race); order them on one
+ * stream. Asynchronous. */
+GS_API int gs_preprocess_bwd_accumulate(const float* means, const float* log_scales, const float* quats,
+                                        const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                                        const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,
+                                        const gs_projected* in, const float* grad2d, float* d_means,
+                                        float* d_log_scales, float* d_quats, float* d_opacity_logits, float* d_sh,
+                                        void* stream);
+
 /* Number of kernels this library has launched in the process so far (all
  * devices, all streams). Host-side counter, for accounting in benchmarks. */
 GS_API int64_t gs_debug_kernel_launches(void);
+
+/* 1 in the checked build of the library (compiled with GS_CHECKED), else 0.
+ * The checked build bounds-checks record and list gathers on the device: a
+ * failed check records a code and skips the access instead of trapping. */
+GS_API int gs_debug_is_checked_build(void);
+
+/* The first failed device-side check since the last call (1: a list value or
+ * active index past the record count, 2: a radix-sort scatter destination
+ * past the key count, 3: a tile range that runs backwards), 0 if none,
+ * 0xffffffff if the status could not be read; the status is cleared. Always
+ * 0 in the unchecked build. Synchronous. */
+GS_API uint32_t gs_debug_checked_status(void);
 
 /* Fault-injection hook for tests of the bounded look-back wait: while set to
  * k >= 0, tile k of every radix-sort pass never publishes its counts, so its

@@ -36,3 +36,26 @@ def pytest_terminal_summary(terminalreporter):
         tr.write_line(f"{what[:60]:60s} {n:10d} {rtol:7.0e} " + " ".join(f"{w:10.4f}" for w in worst))
     tr.write_line("overall worst: " + ", ".join(f"m={m:g}: {max(r[3][k] for r in GRAD_RATIOS):.4f}"
                                                 for k, m in enumerate(FLOORS)))
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Under GS_CHECKED=1 (the bounds-checked library) a session that ran GPU
+    tests fails if any device-side check fired."""
+    if os.environ.get("GS_CHECKED") != "1":
+        return
+    try:
+        import torch
+        if not torch.cuda.is_available():
+            return
+        from differentiable_tile_rasterizer_b200 import gs
+        if gs._LIB is None:
+            return
+        assert gs.gs_debug_is_checked_build(), "GS_CHECKED=1 but the unchecked library is loaded"
+        st = gs.gs_debug_checked_status()
+    except Exception as e:  # report, do not mask the tests' own status
+        print(f"\nchecked build: status not read ({e})")
+        session.exitstatus = 1
+        return
+    print(f"\nchecked build: device-side check status {st}")
+    if st != 0:
+        session.exitstatus = 1

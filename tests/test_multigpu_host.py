@@ -35,3 +35,40 @@ def test_local_params_interleave_by_index(N, G):
             assert local.is_contiguous()
             back[..., r::G] = local.numpy()
         np.testing.assert_array_equal(back, full, err_msg=name)
+
+
+def _best_max_band(cost, world):
+    """Least largest band sum over every contiguous partition (brute force)."""
+    import itertools
+    TH = len(cost)
+    best = None
+    for cuts in itertools.combinations_with_replacement(range(TH + 1), world - 1):
+        starts = [0, *cuts, TH]
+        m = max(sum(cost[a:b]) for a, b in zip(starts, starts[1:]))
+        best = m if best is None else min(best, m)
+    return best
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_balanced_bands_reach_the_least_largest_band(seed):
+    from differentiable_tile_rasterizer_b200.multigpu import balance_bands
+    rng = np.random.default_rng(seed)
+    TH = int(rng.integers(1, 9))
+    world = int(rng.integers(1, 5))
+    cost = [int(c) for c in rng.integers(0, 50, TH) * (rng.random(TH) < 0.8)]
+    starts = balance_bands(cost, world)
+    assert len(starts) == world + 1 and starts[0] == 0 and starts[-1] == TH
+    assert all(a <= b for a, b in zip(starts, starts[1:]))
+    if sum(cost) > 0:
+        got = max(sum(cost[a:b]) for a, b in zip(starts, starts[1:]))
+        assert got == _best_max_band(cost, world)
+
+
+def test_balanced_bands_follow_the_work():
+    from differentiable_tile_rasterizer_b200.multigpu import balance_bands, equal_bands
+    assert balance_bands([0.0] * 68, 8) == equal_bands(8, 68)
+    cost = [1.0] * 60 + [100.0] * 8  # the work sits in the last rows
+    starts = balance_bands(cost, 4)
+    assert starts[1] > 40 and starts[-1] == 68
+    sums = [sum(cost[a:b]) for a, b in zip(starts, starts[1:])]
+    assert max(sums) < 0.5 * sum(cost)

@@ -84,6 +84,14 @@ def _exchange_main(rank, world, port, out):
         send = torch.stack(rows).reshape(-1)
         recv_counts = ex.counts(counts, "cpu")
         recv = ex.payload(send, counts, recv_counts, 3).reshape(-1, 3)
+        # the single-read form: the counts exchanged before they are read
+        s2, r2 = DistExchange(host_staging=True).counts_from_device(torch.tensor(counts, dtype=torch.int64))
+        assert s2 == counts and r2 == recv_counts
+        # band row costs: every rank fills its own rows, all get the sum
+        import numpy as np
+        local = np.zeros(5)
+        local[rank] = rank + 1.0
+        assert DistExchange(host_staging=True).row_costs(local).tolist() == [1.0, 2.0, 3.0, 0.0, 0.0]
         out.put((rank, recv_counts, recv.tolist()))
     finally:
         dist.destroy_process_group()
@@ -106,3 +114,45 @@ def test_exchange_counts_and_payload_with_gloo():
         # segments in source order, rows in send order
         want = [[s, dst, k] for s in range(world) for k in range((s + 1) * (dst + 1))]
         assert rows == want
+
+
+def _reduce_main(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        N, K = 5, 16
+        flat, views = bench.flat_gradients(N, K, "cpu")
+        flat.copy_(torch.arange(flat.numel(), dtype=torch.float32) * (rank + 1))
+        views["sh"][2, 3] += 100.0 * rank  # writes through the views land in the flat buffer
+        bench.reduce_gradients(flat, world)
+        out.put((rank, flat.tolist(), {k: list(v.shape) for k, v in views.items()}))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gradient_all_reduce_of_the_data_parallel_step_with_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_reduce_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = {r: (flat, shapes) for r, flat, shapes in (q.get(timeout=10) for _ in range(world))}
+    N, K = 5, 16
+    n = (11 + 3 * K) * N
+    want = [float(i * 3) for i in range(n)]  # rank 0 contributes i, rank 1 contributes 2 i
+    want[3 * N + 3 * N + 4 * N + N + 2 * N + 3] += 100.0
+    for r in range(world):
+        flat, shapes = res[r]
+        assert flat == want
+        assert shapes == {"means": [3, N], "log_scales": [3, N], "quats": [4, N], "opacity_logits": [N],
+                          "sh": [3 * K, N]}

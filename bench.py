@@ -67,7 +67,7 @@ RASTER_SOURCES = ("differentiable_tile_rasterizer_b200/csrc/raster.cu",
 TRAFFIC_PROFILE = "profiles/raster_kernels_1m_1080p_sh3.md"
 # the kernel each timed raster stage launches (the backward walks the
 # forward's hit bytes)
-KERNEL_OF_STAGE = {"raster_fwd": "raster_fwd_kernel", "raster_bwd": "raster_bwd_hits_kernel"}
+KERNEL_OF_STAGE = {"raster_fwd": "raster_fwd_warp_kernel", "raster_bwd": "raster_bwd_hits_kernel"}
 
 
 def raster_source_hash() -> str:
@@ -683,7 +683,8 @@ def interleaved(args, G):
     direction (the exchanges themselves do not run here)."""
     import torch
     from differentiable_tile_rasterizer_b200 import synthetic
-    from differentiable_tile_rasterizer_b200.multigpu import WIRE, InterleavedRank, emulate, local_params
+    from differentiable_tile_rasterizer_b200.multigpu import (WIRE, InterleavedRank, balance_bands, emulate,
+                                                             local_params)
     from differentiable_tile_rasterizer_b200.pipeline import GaussianParams
     scene = synthetic.make_config(WORKLOAD_CONFIG)
     cam = scene.cameras[0]
@@ -695,6 +696,26 @@ def interleaved(args, G):
     for _ in range(2):  # warm-up, sizes the receive buffers
         emulate(ranks, parts, cam, bg, g)
     torch.cuda.synchronize()
+    result = {"equal_bands": _interleaved_timed(ranks, parts, cam, bg, g, G)}
+    # the bands rebalanced by the measured list entries per tile row
+    cost = sum(r.band_row_costs() for r in ranks)
+    bands = balance_bands(cost, G)
+    for r in ranks:
+        r.set_bands(bands)
+    for _ in range(2):
+        emulate(ranks, parts, cam, bg, g)
+    torch.cuda.synchronize()
+    result["balanced_bands"] = _interleaved_timed(ranks, parts, cam, bg, g, G)
+    result["balanced_bands"]["band_starts"] = bands
+    return {"workload": "1m_1920x1080_sh3_pose0", "ranks": G, "emulated_on_one_gpu": True,
+            "modelled": "a G-GPU step modelled as the slowest emulated rank's phases plus both exchanges at the "
+                        "measured 770 GB/s per direction; not a measurement on G GPUs", **result}
+
+
+def _interleaved_timed(ranks, parts, cam, bg, g, G):
+    """Per-rank phase times of the emulated ranks and the modelled G-GPU step."""
+    import torch
+    from differentiable_tile_rasterizer_b200.multigpu import WIRE
     ev = lambda: torch.cuda.Event(enable_timing=True)
     reps = 5
     t = {k: [0.0] * G for k in ("project_pack", "merge_sort_raster", "raster_bwd", "return_preprocess_bwd")}
@@ -747,8 +768,7 @@ def interleaved(args, G):
     link = 770e9
     xchg_ms = 1e3 * (fwd_bytes + bwd_bytes) / link
     step_ms = max(per_rank) + xchg_ms
-    return {"workload": "1m_1920x1080_sh3_pose0", "ranks": G, "emulated_on_one_gpu": True,
-            "ms_per_rank": per_rank, "phase_ms_per_rank": t, "records_sent": sent, "records_received": recvd,
+    return {"ms_per_rank": per_rank, "phase_ms_per_rank": t, "records_sent": sent, "records_received": recvd,
             "exchange_bytes_max_rank": {"forward": fwd_bytes, "backward": bwd_bytes},
             "modelled": {"exchange_ms_at_770GBps": xchg_ms, "step_ms": step_ms, "frames_per_s": 1e3 / step_ms,
                          "load_balance_max_over_mean": max(per_rank) / (sum(per_rank) / G)}}

@@ -53,6 +53,7 @@ constexpr uint32_t kValMask = (1u << 30) - 1u;
 constexpr uint32_t kFlagAgg = 1u << 30;
 constexpr uint32_t kFlagInc = 2u << 30;
 constexpr uint32_t kSpinLimit = 1u << 20;
+constexpr int kLookAhead = 4;  // look-back words read per poll
 constexpr uint32_t kInvisibleKey = 0xffffffffu;
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -505,22 +506,41 @@ __global__ void __launch_bounds__(kSortBlock, 2) onesweep_kernel(PassArgs a) {
     if (!stall) st_relaxed(row + d, kFlagInc | cnt);
   } else {
     if (!stall) st_relaxed(row + d, kFlagAgg | cnt);
+    // kLookAhead predecessor words per poll, in flight together; they are
+    // taken in order as before: aggregates are added, the first inclusive
+    // prefix (or tile 0) ends the walk, and the first word not yet published
+    // is polled again, from where the walk stopped.
     int64_t k = tile - 1;
     uint32_t spins = 0;
     while (true) {
-      const uint32_t s = ld_relaxed(a.lookback + (size_t)k * kRadix + d);
-      const uint32_t flag = s & ~kValMask;
-      if (flag == 0u) {
+      uint32_t w[kLookAhead];
+#pragma unroll
+      for (int i = 0; i < kLookAhead; ++i)
+        w[i] = k - i >= 0 ? ld_relaxed(a.lookback + (size_t)(k - i) * kRadix + d) : 0u;
+      int i = 0;
+      bool stop = false, pending = false;
+#pragma unroll
+      for (; i < kLookAhead; ++i) {
+        const uint32_t flag = w[i] & ~kValMask;
+        if (flag == 0u) {
+          pending = true;
+          break;
+        }
+        excl += w[i] & kValMask;
+        if (flag == kFlagInc || k - i == 0) {
+          stop = true;
+          break;
+        }
+      }
+      if (stop) break;
+      k -= i;  // past the aggregates taken; at the unpublished word if pending
+      if (pending) {
         if (++spins > kSpinLimit) {
           atomicExch(a.status, (int32_t)GS_ERR_DEVICE_TIMEOUT);
           break;
         }
         __nanosleep(64);
-        continue;
       }
-      excl += s & kValMask;
-      if (flag == kFlagInc || k == 0) break;
-      --k;
     }
     if (!stall) st_relaxed(row + d, kFlagInc | ((excl + cnt) & kValMask));
   }

@@ -177,26 +177,57 @@ def step_roofline(work, stage_ms, ms_per_step, steps, bw_gbs, peak_alu_t):
 
 
 class ClockSampler:
-    """nvidia-smi clock and throttle samples during the timed region."""
+    """SM clock and throttle-reason samples during the timed region: read
+    through NVML every 5 ms from a thread (read-only queries), else through
+    nvidia-smi every 50 ms."""
 
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
     QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_s: float = 0.005):
         self.dev = device_index
+        self.interval = interval_s
         self.proc = None
+        self.thread = None
+        self.stop = threading.Event()
+        self.samples = []  # (sm MHz, max sm MHz, set of reason names)
         self.lines = []
+        self.source = None
+
+    def _uuid(self):
+        import torch
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
 
     def __enter__(self):
         try:
-            import torch
-            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self._uuid())
+            mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop.is_set():
+                    sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    bits = int(pynvml.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    self.samples.append((sm, mx, {n for n, b in self.REASONS if bits & b}))
+                    self.stop.wait(self.interval)
+
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.source = "nvml, every 5 ms"
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", sel, f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", "-i", self._uuid(), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
                  "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi, every 50 ms"
             self.thread.start()
         except Exception:
             self.proc = None
@@ -207,33 +238,33 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        elif self.thread is not None:
+            self.thread.join(timeout=5)
         return False
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        samples = list(self.samples)
+        names = [n for n, _ in self.REASONS]
         for l in self.lines:
             f = [x.strip() for x in l.split(",")]
             if len(f) < 8:
                 continue
             try:
-                sm.append(float(f[0]))
-                mx.append(float(f[1]))
+                samples.append((float(f[0]), float(f[1]), {n for n, v in zip(names, f[4:8]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for n, v in zip(names, f[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": float(np.median([x[0] for x in samples])), "sm_max_mhz": max(x[1] for x in samples),
+                "reasons": sorted(set().union(*[x[2] for x in samples])), "samples": len(samples),
+                "source": self.source}
 
 
 def _dist_setup():

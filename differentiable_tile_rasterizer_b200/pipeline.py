@@ -403,15 +403,26 @@ class MultiViewRenderer:
     parameters projects every Gaussian into all views
     (gs_preprocess_multiview), then each view runs its bin/sort and raster
     forward on its own buffers (a Rasterizer per view). No cull: every
-    Gaussian is projected into every view."""
+    Gaussian is projected into every view.
 
-    def __init__(self, N: int, sh_degree: int, cams, device=None, capacity: Optional[int] = None):
+    The views' bin/sorts and raster forwards run on n_streams streams (view
+    v on stream v mod n_streams), forked from and joined to the caller's
+    stream, so that one view's latency-bound sort kernels overlap another
+    view's compositing. With deferred mode on (set_deferred) no call waits
+    on the host; otherwise each bin/sort waits for its own stream only.
+    While stage timing is on (stage_events not None) the views run one after
+    another on one stream, so that each stage's events bracket its own work."""
+
+    def __init__(self, N: int, sh_degree: int, cams, device=None, capacity: Optional[int] = None,
+                 n_streams: int = 4):
         self.cams = [c if isinstance(c, gs.GsCamera) else gs.camera(c) for c in cams]
         if not 0 < len(self.cams) <= gs.GS_MAX_VIEWS:
             raise ValueError(f"1 .. {gs.GS_MAX_VIEWS} views per pass")
         self.N, self.sh_degree = int(N), int(sh_degree)
         self.views = [Rasterizer(N, sh_degree, c.width, c.height, device=device, capacity=capacity)
                       for c in self.cams]
+        d = torch.device(device or "cuda")
+        self.streams = [torch.cuda.Stream(device=d) for _ in range(min(max(int(n_streams), 1), len(self.cams)))]
         self.stage_events = None
 
     def _timed(self, stage):
@@ -424,13 +435,20 @@ class MultiViewRenderer:
             gs.gs_preprocess_multiview(params.means, params.log_scales, params.quats, params.opacity_logits,
                                        params.sh, params.sh_degree, self.N, self.cams,
                                        [R._proj for R in self.views])
-        for R, c in zip(self.views, self.cams):
+        cur = torch.cuda.current_stream()
+        streams = self.streams if self.stage_events is None else self.streams[:1]
+        for st in streams:
+            st.wait_stream(cur)
+        for v, (R, c) in enumerate(zip(self.views, self.cams)):
             R.params, R.cam, R.bg, R.culled = params, c, bg, False
-            with self._timed("bin_sort"):
-                R._bin_sort(c)
-            with self._timed("raster_fwd"):
-                gs.gs_rasterize_fwd(R._proj, R.vals, R.ranges, c, bg, R.image, R.final_T, R.n_contrib, R.last,
-                                    tile_order=R._order(), hit_bits=R._hits())
+            with torch.cuda.stream(streams[v % len(streams)]):
+                with self._timed("bin_sort"):
+                    R._bin_sort(c)
+                with self._timed("raster_fwd"):
+                    gs.gs_rasterize_fwd(R._proj, R.vals, R.ranges, c, bg, R.image, R.final_T, R.n_contrib,
+                                        R.last, tile_order=R._order(), hit_bits=R._hits())
+        for st in streams:
+            cur.wait_stream(st)
         return [R.image for R in self.views]
 
     def set_deferred(self, on: bool):

@@ -1,13 +1,14 @@
 // Tile compositing: forward (front to back) and backward (back to front).
 //
-// One CTA per 16x16 tile, one thread per pixel; each warp owns an 8x4 pixel
-// block so that its lanes sit close together in the image. The tile's sorted
-// list is walked in batches of 256 records, one per thread, that the CTA
-// stages in shared memory, after which every thread reads them as
-// shared-memory broadcasts. In the backward the gathers are
-// software-pipelined: a batch's records arrive by cp.async while the
-// previous batch is processed. The forward CTA leaves the walk as soon as
-// all its pixels have stopped.
+// A 16x16 tile is four 8x8 pixel blocks, each the work of one warp, whose
+// lanes hold two pixels (the same column, rows r and r + 4) run as packed
+// fp32 pairs. The forward's warps, and the backward's when the forward's hit
+// bytes are given, walk the tile's sorted list independently, with the
+// entries' records gathered by cp.async into the warp's own shared-memory
+// slots one chunk ahead; no CTA barrier stands between them. The backward
+// without hit bytes stages batches of records for the tile's four warps in
+// shared memory. The forward's warps leave the walk as soon as their pixels
+// have stopped.
 //
 // The per-pair arithmetic is the fixed fp32 specification: the conic is
 // scaled by -log2(e)/2 (and -log2(e) for the cross term) when it is staged,
@@ -26,12 +27,8 @@ constexpr int kTile = 16;
 constexpr int kBlock = kTile * kTile;
 // Backward CTA: 4 warps, two pixels per thread.
 constexpr int kBlockB = kBlock / 2;
-// List entries staged in shared memory per CTA-wide step: one per thread.
-// Forward batch: 512 entries (two staged per thread) halve the CTA barriers
-// and even out the warps' shares of a batch; the importance variant, whose
-// per-entry sums need more registers, keeps 256.
-template <bool kImp>
-constexpr int fwd_batch() { return kImp ? kBlock : 2 * kBlock; }
+// List entries staged in shared memory per CTA-wide step of the backward
+// without hit bytes: one per thread.
 constexpr int kBatchB = kBlockB;
 
 // 16-byte asynchronous global -> shared copy (L2 only), its commit and the
@@ -45,13 +42,6 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // cp.async groups: wait until at most one (the newest) is still in flight.
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
 
-// Pixel of thread `tid` in the tile: warp w covers the 8x4 block at
-// ((w & 1) * 8, (w >> 1) * 4).
-__device__ __forceinline__ void tile_pixel(int tid, int& du, int& dv) {
-  const int w = tid >> 5, l = tid & 31;
-  du = (w & 1) * 8 + (l & 7);
-  dv = (w >> 1) * 4 + (l >> 3);
-}
 
 // Conservative screen box of the pixel centres at which the fp32 pair
 // arithmetic can give alpha >= 1/255 (a warp whose pixels all lie outside
@@ -134,10 +124,6 @@ __device__ __forceinline__ bool region_hits(const float4 b, const float4 q1, con
   return best <= q1.w;
 }
 
-// Centre of the 8x4 block of pixel centres of forward warp w in the tile at
-// (tx0, ty0).
-__device__ __forceinline__ float block_cx(int tx0, int w) { return (float)(tx0 + (w & 1) * 8) + 4.0f; }
-__device__ __forceinline__ float block_cy(int ty0, int w) { return (float)(ty0 + (w >> 1) * 4) + 2.0f; }
 
 // Tiles in descending order of log2 of their list length: a launch that takes
 // its CTAs' tiles in this order starts the longest lists first, so few long
@@ -185,189 +171,6 @@ struct FwdArgs {
   uint8_t* hits;               // [entries] or null: bit w = the entry blended in warp w's block
 };
 
-// kImp also accumulates each Gaussian's importance weight (the sum over the
-// view's pixels of its blend weights alpha * T): a warp sum per step, a
-// shared-memory sum per staged entry, one atomic per (Gaussian, tile).
-template <bool kImp>
-__global__ void __launch_bounds__(kBlock, 5) raster_fwd_kernel(FwdArgs a) {
-  constexpr int kBatchF = fwd_batch<kImp>();
-  constexpr int kStageF = kBatchF / kBlock;  // entries each thread stages per batch
-  __shared__ float s_imp[kImp ? kBatchF : 1];
-  __shared__ float4 s_geo[kBatchF];  // px, py, a2, b2
-  __shared__ float2 s_co[kBatchF];   // c2, opacity
-  __shared__ float4 s_rgb[kBatchF];
-  // blend region of each staged entry (BlendRegion without what s_geo holds
-  // and the pad, which region_hits needs only when it derives from px, py)
-  __shared__ float2 s_hxy[kBatchF];  // box half-widths
-  __shared__ float4 s_q1[kBatchF];
-  __shared__ float2 s_q2[kBatchF];
-  // per batch parity: the entries of chunk c that blended at some pixel of
-  // warp w (0 for chunks the warp did not reach: its pixels had all stopped)
-  __shared__ uint32_t s_wm[2][kBlock / 32][kBatchF / 32];
-  const uint32_t tile_u = a.order ? a.order[blockIdx.x] : blockIdx.x;
-  if (tile_u >= gridDim.x) return;  // not a tile: a schedule that is no permutation
-  const int tile = (int)tile_u;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int du, dv;
-  tile_pixel(tid, du, dv);
-  const int tx0 = (tile % a.TW) * kTile, ty0 = (tile / a.TW) * kTile;
-  const int u = tx0 + du, v = ty0 + dv;
-  const bool inside = u < a.W && v < a.H;
-  const float xc = __fadd_rn((float)u, 0.5f), yc = __fadd_rn((float)v, 0.5f);
-  // centre of this warp's 8x4 block of pixel centres
-  const float wcx = block_cx(tx0, warp), wcy = block_cy(ty0, warp);
-  const uint2 range = a.ranges[tile];
-  const int n = check(range.y >= range.x, kCheckTileRange) ? (int)(range.y - range.x) : 0;
-  float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
-  int cnt = 0, lst = 0;
-  bool done = !inside;
-  // importance: the entries this thread staged last (slots tid + s kBlock),
-  // and their flush
-  uint32_t istaged[kStageF] = {};
-  bool have_staged[kStageF] = {};
-  if (kImp)
-    for (int st = 0; st < kStageF; ++st) s_imp[tid + st * kBlock] = 0.0f;
-  auto flush = [&]() {
-#pragma unroll
-    for (int st = 0; st < kStageF; ++st) {
-      if (kImp && have_staged[st]) {
-        const int e = tid + st * kBlock;
-        const float w = s_imp[e];
-        const uint32_t i = istaged[st];
-        if (w != 0.0f) atomicAdd(a.importance + (a.active_idx ? a.active_idx[i] : (int32_t)i), w);
-        s_imp[e] = 0.0f;
-        have_staged[st] = false;
-      }
-    }
-  };
-  // hit bytes of the entries this thread staged in the batch at `hbase`,
-  // from the eight warps' ballots of parity `par`
-  auto write_hits = [&](int hbase, int par) {
-#pragma unroll
-    for (int st = 0; st < kStageF; ++st) {
-      const int e = tid + st * kBlock;
-      if (a.hits && hbase >= 0 && hbase + e < n) {
-        uint32_t h = 0;
-#pragma unroll
-        for (int w = 0; w < kBlock / 32; ++w) h |= ((s_wm[par][w][e >> 5] >> lane) & 1u) << w;
-        a.hits[range.x + hbase + e] = (uint8_t)h;
-      }
-    }
-  };
-  // (The forward stages with plain gathers: with five CTAs per SM the
-  // others cover a staging CTA's latency.)
-  int par = 0, last_staged = -1;
-  for (int base = 0; base < n; base += kBatchF, par ^= 1) {
-    if (__syncthreads_count(done) == kBlock) break;
-    flush();  // the previous batch's sums are complete (barrier above)
-    write_hits(base - kBatchF, par ^ 1);  // and its ballots
-    last_staged = base;
-    static_assert((kBlock / 32) * (kBatchF / 32) <= kBlock, "one word per thread clears the ballots");
-    if (a.hits && tid < (kBlock / 32) * (kBatchF / 32)) (&s_wm[par][0][0])[tid] = 0u;
-#pragma unroll
-    for (int st = 0; st < kStageF; ++st) {
-      const int e = tid + st * kBlock;
-      if (base + e < n) {
-        const uint32_t i = a.vals[range.x + base + e];
-        if (kImp) {
-          istaged[st] = i;
-          have_staged[st] = true;
-        }
-        const float4 g = a.xyzo[i];
-        const float4 q = a.conic[i];
-        const float a2 = __fmul_rn(q.x, kHalfNegLog2e), b2 = __fmul_rn(q.y, kNegLog2e),
-                    c2 = __fmul_rn(q.z, kHalfNegLog2e);
-        s_geo[e] = make_float4(g.x, g.y, a2, b2);
-        s_co[e] = make_float2(c2, g.w);
-        s_rgb[e] = a.rgb[i];
-        const BlendRegion r = blend_region(g.x, g.y, a2, b2, c2, g.w);
-        s_hxy[e] = make_float2(r.box.z, r.box.w);
-        s_q1[e] = r.q1;
-        s_q2[e] = make_float2(r.q2.x, r.q2.y);
-      }
-    }
-    __syncthreads();
-    const int m = min(kBatchF, n - base);
-    for (int c0 = 0; c0 < m; c0 += 32) {
-      if (__all_sync(0xffffffffu, done)) break;
-      const int j = c0 + lane;
-      bool rel = false;
-      if (j < m) {
-        const float4 gj = s_geo[j];
-        const float2 hj = s_hxy[j], qj = s_q2[j];
-        // blend_region's box and q2, the pad recomputed exactly as it did
-        const float pad = 0.05f + 1e-6f * (fabsf(gj.x) + fabsf(gj.y));
-        rel = region_hits(make_float4(gj.x, gj.y, hj.x, hj.y), s_q1[j], make_float4(qj.x, qj.y, pad, 0.0f), wcx,
-                          wcy, 3.5f, 1.5f);
-      }
-      unsigned msk = __ballot_sync(0xffffffffu, rel);
-      unsigned blended = 0u;  // bit k - c0: entry k blended at this lane's pixel (OR-ed over the warp below)
-      // Entries are taken two at a time: their alphas at this pixel run as
-      // one packed pair (each half rounded as the scalar operation), then
-      // they blend in list order. Branch-free blend: a lane that skips an
-      // entry (alpha < 1/255) or has already stopped blends with alpha 0,
-      // which leaves C, T and the counts exactly as they were (colours are
-      // finite), so the warp never diverges.
-      auto blend_one = [&](int k, float alpha) {
-        const float4 c = s_rgb[k];
-        const bool blend = !done && alpha >= kAlphaMin;
-        const float ab = blend ? alpha : 0.0f;
-        const float wgt = __fmul_rn(ab, T);
-        C0 = __fmaf_rn(wgt, c.x, C0);
-        C1 = __fmaf_rn(wgt, c.y, C1);
-        C2 = __fmaf_rn(wgt, c.z, C2);
-        T = __fmul_rn(T, __fsub_rn(1.0f, ab));
-        cnt += blend ? 1 : 0;
-        lst = blend ? base + k + 1 : lst;
-        done = done || T < kTMin;
-        blended |= (blend ? 1u : 0u) << (k - c0);
-        if (kImp && __any_sync(0xffffffffu, blend)) {
-          float ws = wgt;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
-          if (lane == 0 && ws != 0.0f) atomicAdd(&s_imp[k], ws);
-        }
-      };
-      while (msk) {
-        const int k1 = c0 + __ffs(msk) - 1;
-        msk &= msk - 1;
-        const bool has2 = msk != 0;  // the same for the whole warp
-        const int k2 = has2 ? c0 + __ffs(msk) - 1 : k1;
-        msk &= msk - 1;
-        const float4 g1 = s_geo[k1], g2 = s_geo[k2];
-        const float2 co1 = s_co[k1], co2 = s_co[k2];
-        const float2 dx = sub2(make_float2(g1.x, g2.x), splat2(xc));
-        const float2 dy = sub2(make_float2(g1.y, g2.y), splat2(yc));
-        const float2 qv = fma2(make_float2(g1.w, g2.w), dy, mul2(make_float2(g1.z, g2.z), dx));
-        float2 p2 = mul2(dx, qv);
-        p2 = fma2(mul2(make_float2(co1.x, co2.x), dy), dy, p2);
-        const float2 e = exp2_raster2(p2);
-        const float2 va = mul2(make_float2(co1.y, co2.y), e);
-        blend_one(k1, fminf(va.x, kAlphaMax));
-        if (has2) blend_one(k2, fminf(va.y, kAlphaMax));
-      }
-      if (a.hits) {
-        blended = __reduce_or_sync(0xffffffffu, blended);
-        if (lane == 0) s_wm[par][warp][c0 >> 5] = blended;
-      }
-    }
-  }
-  if (kImp || a.hits) {
-    __syncthreads();
-    flush();
-    write_hits(last_staged, (last_staged / kBatchF) & 1);  // the last staged batch
-  }
-  if (inside) {
-    const size_t P = (size_t)a.W * a.H, pix = (size_t)v * a.W + u;
-    a.image[pix] = __fmaf_rn(T, a.bg0, C0);
-    a.image[P + pix] = __fmaf_rn(T, a.bg1, C1);
-    a.image[2 * P + pix] = __fmaf_rn(T, a.bg2, C2);
-    a.final_T[pix] = T;
-    a.n_contrib[pix] = cnt;
-    a.last[pix] = lst;
-  }
-}
-
 // Zeroes the hit bytes of every tile's list entries ([range.x, range.y) of
 // each tile, one CTA per tile) before a forward whose warps OR their bits in.
 __global__ void __launch_bounds__(256) zero_hits_kernel(const uint2* ranges, uint8_t* hits) {
@@ -375,8 +178,8 @@ __global__ void __launch_bounds__(256) zero_hits_kernel(const uint2* ranges, uin
   for (uint32_t k = r.x + threadIdx.x; k < r.y; k += 256) hits[k] = 0;
 }
 
-// Forward with one warp per CTA and no CTA barrier: warp w of a tile (CTA
-// 4 slot + w) owns the 8x8 pixel block at ((w & 1) * 8, (w >> 1) * 8), lane l
+// Forward with independent warps and no CTA barrier: warp w of a tile (warp
+// 4 slot + w of the grid) owns the 8x8 pixel block at ((w & 1) * 8, (w >> 1) * 8), lane l
 // its pixels (l & 7, l >> 3) and (l & 7, (l >> 3) + 4), both run as packed
 // fp32 pairs (each half rounded as the scalar operation, so every pixel's
 // values are those of the specification). The warp walks its tile's list
@@ -393,12 +196,20 @@ __global__ void __launch_bounds__(256) zero_hits_kernel(const uint2* ranges, uin
 // kFwdWarps independent warps per CTA (blocks of the same tile, sharing
 // nothing): more resident warps than one-warp CTAs allow (32 per SM), within
 // the register bound below.
+// kImp also adds each Gaussian's importance weight (the sum over the view's
+// pixels of its blend weights alpha * T): per blended entry the warp sums its
+// 64 pixels' weights (the lane's pair, then a 5-level butterfly) into the
+// entry's slot, and after the chunk each lane adds its entry's slot to the
+// Gaussian's total with one atomic: one atomic per (Gaussian, 8x8 block).
 constexpr int kFwdWarps = 2;
 static_assert(4 % kFwdWarps == 0, "a tile's four blocks split evenly over the CTAs");
+template <bool kImp>
 __global__ void __launch_bounds__(32 * kFwdWarps, 18) raster_fwd_warp_kernel(FwdArgs a) {
   __shared__ float4 s_raw_all[kFwdWarps][2][3][32];  // per warp: xyzo, conic, rgb of two chunks of entries
+  __shared__ float s_imp_all[kImp ? kFwdWarps : 1][32];  // per warp: the chunk's importance sums
   const int lane = threadIdx.x & 31;
   float4(*s_raw)[3][32] = s_raw_all[threadIdx.x >> 5];
+  float* s_imp = s_imp_all[kImp ? threadIdx.x >> 5 : 0];
   const int64_t gw = (int64_t)blockIdx.x * kFwdWarps + (threadIdx.x >> 5);  // (tile slot, 8x8 block)
   const uint32_t slot4 = (uint32_t)(gw >> 2);
   const int warp = (int)(gw & 3);
@@ -435,6 +246,7 @@ __global__ void __launch_bounds__(32 * kFwdWarps, 18) raster_fwd_warp_kernel(Fwd
     if (__all_sync(0xffffffffu, done0 && done1)) break;
     const int buf = c & 1;
     fetch(buf ^ 1, c + 1, i_nxt);  // chunk c + 1 in flight (its buffer was released after chunk c - 1)
+    const uint32_t i_this = i_cur;  // this lane's entry of chunk c
     i_cur = i_nxt;
     i_nxt = meta(c + 2);
     cp_async_wait_1();  // this lane's copies of chunk c have landed
@@ -453,6 +265,7 @@ __global__ void __launch_bounds__(32 * kFwdWarps, 18) raster_fwd_warp_kernel(Fwd
     unsigned msk = __ballot_sync(0xffffffffu, rel);
     __syncwarp();                 // the scaled conics are visible to every lane
     uint32_t bl0 = 0u, bl1 = 0u;  // bit k: entry 32 c + k blended at this lane's pixel 0 / 1
+    uint32_t imp_msk = 0u;        // kImp: bit k: entry 32 c + k has a sum in its slot
     while (msk) {
       const int k = __ffs(msk) - 1;
       msk &= msk - 1;
@@ -474,6 +287,13 @@ __global__ void __launch_bounds__(32 * kFwdWarps, 18) raster_fwd_warp_kernel(Fwd
       const float4 col = s_raw[buf][2][k];
       const float2 ab = make_float2(b0 ? al0 : 0.0f, b1 ? al1 : 0.0f);
       const float2 wgt = mul2(ab, T);
+      if (kImp) {
+        float ws = wgt.x + wgt.y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ws += __shfl_xor_sync(0xffffffffu, ws, o);
+        if (lane == 0) s_imp[k] = ws;
+        imp_msk |= 1u << k;
+      }
       C0 = fma2(wgt, splat2(col.x), C0);
       C1 = fma2(wgt, splat2(col.y), C1);
       C2 = fma2(wgt, splat2(col.z), C2);
@@ -482,6 +302,13 @@ __global__ void __launch_bounds__(32 * kFwdWarps, 18) raster_fwd_warp_kernel(Fwd
       done1 = done1 || T.y < kTMin;
       bl0 |= (b0 ? 1u : 0u) << k;
       bl1 |= (b1 ? 1u : 0u) << k;
+    }
+    if (kImp) {
+      __syncwarp();  // lane 0's sums are visible
+      if ((imp_msk >> lane) & 1u) {
+        const float w = s_imp[lane];
+        if (w != 0.0f) atomicAdd(a.importance + (a.active_idx ? a.active_idx[i_this] : (int32_t)i_this), w);
+      }
     }
     // contributor counts and last blends of the chunk, from its blend masks
     cnt0 += __popc(bl0);
@@ -964,15 +791,14 @@ cudaError_t launch_raster_fwd(const Records& rec, const uint32_t* vals, const ui
   a.importance = importance; a.active_idx = active_idx; a.hits = hits;
   const int TT = cam.TW * cam.TH;
   int launched = 1;
-  if (importance) {
-    raster_fwd_kernel<true><<<TT, kBlock, 0, s>>>(a);
-  } else {
-    if (hits) {
-      zero_hits_kernel<<<TT, 256, 0, s>>>(a.ranges, hits);
-      ++launched;
-    }
-    raster_fwd_warp_kernel<<<TT * 4 / kFwdWarps, 32 * kFwdWarps, 0, s>>>(a);
+  if (hits) {
+    zero_hits_kernel<<<TT, 256, 0, s>>>(a.ranges, hits);
+    ++launched;
   }
+  if (importance)
+    raster_fwd_warp_kernel<true><<<TT * 4 / kFwdWarps, 32 * kFwdWarps, 0, s>>>(a);
+  else
+    raster_fwd_warp_kernel<false><<<TT * 4 / kFwdWarps, 32 * kFwdWarps, 0, s>>>(a);
   count_launches(launched);
   return cudaGetLastError();
 }

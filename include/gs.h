@@ -416,8 +416,8 @@ GS_API int gs_rasterize_fwd(const gs_projected* in, const uint32_t* vals,
  *                (from gs_cull; NULL: record i is Gaussian i)
  *   importance   [device] [N] f32 in/out: this view's weights are ADDED, so
  *                zero it once and call once per view to sum over views
- * The sums are fp32 atomics in an unspecified order (a warp sum, a CTA sum,
- * then one atomic per (Gaussian, tile)). Asynchronous. */
+ * The sums are fp32 atomics in an unspecified order (a warp sum over an 8x8
+ * pixel block, then one atomic per (Gaussian, block)). Asynchronous. */
 GS_API int gs_rasterize_fwd_importance(const gs_projected* in, const uint32_t* vals,
                                        const uint32_t* tile_ranges, const uint32_t* tile_order,
                                        const gs_camera* cam, const float* bg,

@@ -88,7 +88,7 @@ def test_1m_1080p_sh3_importance_pass_pose0():
     rec = oracle.preprocess(sc, cam)
     bins = oracle.bin_sort(rec, cam)
     ref = oracle.importance(rec, bins, cam, sc.N)
-    bound = (16.0 + rec["tiles"]) * 2.0 ** -23 * ref + 1e-30
+    bound = (6.0 + 4.0 * rec["tiles"]) * 2.0 ** -23 * ref + 1e-30
     bad = np.abs(got - ref) > bound
     assert not bad.any(), (bad.sum(), got[bad][:3], ref[bad][:3])
     assert ref.sum() > 1e5

@@ -591,6 +591,9 @@ def run_ours(args):
         roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None, "avg_launch_ms": avg_ms}
     roof["peak_kind"] = peaks["source"]
+    if roof["bound"] == "alu" and clocks.get("sm_mhz"):
+        # the same against the SM clock sampled while the step ran
+        roof["frac_at_sampled_clock"] = achieved / (148 * FP32_LANES_PER_SM * clocks["sm_mhz"] * 1e6 / 1e12)
 
     line = {"metric": METRIC, "value": value, "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

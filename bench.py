@@ -2,22 +2,28 @@
 """Benchmark: forward + backward frames/s of the tile rasterizer.
 
 Workload (default): 1M Gaussians, SH degree 3, 1920x1080, four camera poses
-per step; each pose runs the whole path through the C ABI -- preprocess,
-bin/sort, tile order, rasterize forward, rasterize backward (2-D part and
-parameter part); both cull gates are off, so no cull runs. Inputs are
-synthetic and resident in HBM before timing; the 236 MB parameter set is
-larger than the 126 MB L2, so no flush is needed.
+per step: the forward and backward of all four poses and the parameter
+gradient of the loss summed over them, through the C ABI. Both cull gates
+are off, so the step is one multi-view pass: one read of the parameters
+projects every pose (gs_preprocess_multiview); each pose's bin/sort, tile
+order, raster forward and raster backward (2-D part) run on its own stream
+and buffers; one more read of the parameters chains the poses' 2-D
+gradients to the summed parameter gradient (gs_preprocess_bwd_multiview).
+A workload with a cull (or a single pose) runs each pose as a chain of its
+own: cull, preprocess, bin/sort, raster forward and backward, parameter
+part. Inputs are synthetic and resident in HBM before timing; the 236 MB
+parameter set is larger than the 126 MB L2, so no flush is needed.
 
-Timing: `value` is K replays of one CUDA graph holding a whole step (each
-pose on its own stream and buffers); per-stage times and the roofline's
-kernel duration come from a second loop of K steps launched call by call
-with CUDA events around each stage. `e2e` runs the same steps through the
-public API with pinned host buffers, copies inside the timed region.
+Timing: `value` is K replays of one CUDA graph holding a whole step;
+per-stage times and the roofline's kernel duration come from a second loop
+of K steps launched call by call with CUDA events around each stage (the
+poses one after another on one stream). `e2e` runs the same steps through
+the public API with pinned host buffers, copies inside the timed region.
 
 Prints one JSON line on rank 0. Under torchrun (N > 1) the step is
 data-parallel training over views (weak scaling): each rank renders its own
-batch of poses, sums their parameter gradients and all-reduces the sum with
-the other ranks (NCCL) every step; the time is the maximum over ranks.
+batch of poses and all-reduces its summed parameter gradient with the other
+ranks (NCCL) every step; the time is the maximum over ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload 1|2|3] [--multiview] [--interleaved G]
@@ -118,11 +124,12 @@ def profiled_exec_ops(stage: str):
     return None
 
 
-def stage_work(scene, counts):
+def stage_work(scene, counts, multiview=False):
     """Algorithmic bytes and fp32 operations per stage, summed over the
     poses of one step, from the per-pose counts (V visible, I instances, E
     and E_bwd evaluated pairs, B blends). Bytes are what a stage must move at
-    least: parameters and records read once, outputs written once."""
+    least: parameters and records read once, outputs written once. With
+    `multiview` the per-Gaussian stages are the one-pass multi-view ones."""
     K = scene.K
     N = scene.N
     cam = scene.cameras[0]
@@ -153,6 +160,15 @@ def stage_work(scene, counts):
         w["preprocess_bwd"]["bytes"] += N * par + V * (par + 48 + 16)
     if not any(c.get("culled") for c in counts):
         del w["cull"]
+    if multiview:
+        del w["preprocess"], w["preprocess_bwd"]
+        # parameters in once, a 64 B record out per pose
+        w["preprocess_multiview"] = {"bytes": N * (par + 64 * len(counts)), "ops": 0.0}
+        # parameters in and every gradient row out once; per pose the tile
+        # count of every record and the 2-D gradient row and colour of the
+        # visible ones
+        w["preprocess_bwd_multiview"] = {"bytes": 2 * N * par + sum(4 * N + 64 * c["V"] for c in counts),
+                                         "ops": 0.0}
     return w
 
 
@@ -295,20 +311,6 @@ def _max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
-def flat_gradients(N: int, K: int, device):
-    """One flat float32 buffer of a whole parameter gradient and its views in
-    the library's SoA shapes (means [3][N], log_scales [3][N], quats [4][N],
-    opacity_logits [N], sh [3K][N]), so that one collective reduces all."""
-    import torch
-    flat = torch.empty((11 + 3 * K) * N, dtype=torch.float32, device=device)
-    views, o = {}, 0
-    for name, rows in (("means", 3), ("log_scales", 3), ("quats", 4), ("opacity_logits", 1), ("sh", 3 * K)):
-        v = flat[o: o + rows * N]
-        views[name] = v if name == "opacity_logits" else v.view(rows, N)
-        o += rows * N
-    return flat, views
-
-
 def reduce_gradients(flat, world: int):
     """The data-parallel step's exchange: the sum over ranks of every rank's
     parameter gradient (one all-reduce; NCCL between GPUs, gloo on CPU)."""
@@ -436,7 +438,8 @@ def run_reference(args):
 def run_ours(args):
     import torch
     from differentiable_tile_rasterizer_b200 import gs, synthetic
-    from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, Rasterizer
+    from differentiable_tile_rasterizer_b200.pipeline import (GaussianParams, MultiViewRenderer, Rasterizer,
+                                                              flat_gradient_buffers)
 
     world, rank, local = _dist_setup()
     gs.load(build_if_missing=False)
@@ -452,68 +455,91 @@ def run_ours(args):
     R = Rasterizer(scene.N, scene.sh_degree, W, H, capacity=6 * scene.N)
     bg = tuple(float(b) for b in scene.bg)
 
-    def step():
-        for p, c in enumerate(cams):
-            R.forward(params, c, bg, lod, quant)
-            R.backward(gimg[p])
+    use_mv = lod <= 0 and quant <= 0 and 1 < len(poses) <= gs.GS_MAX_VIEWS
+    mv = None
+    flat = None
+    if use_mv:
+        # one multi-view pass per step (module docstring); its summed
+        # parameter gradient is one flat buffer, all-reduced as one
+        mv = MultiViewRenderer(scene.N, scene.sh_degree, cams, capacity=6 * scene.N, n_streams=len(cams))
+        flat = mv.grads_flat
 
-    # The poses of a step are independent: each gets its own buffers and
-    # stream, so that one pose's latency-bound bin/sort kernels share the
-    # GPU with another pose's raster kernels (the captured graph holds one
-    # chain per pose).
-    Rp = [R] + [Rasterizer(scene.N, scene.sh_degree, W, H, capacity=6 * scene.N) for _ in cams[1:]]
-    streams = [torch.cuda.Stream() for _ in cams]
-    # With several ranks the step is data-parallel training over views: each
-    # rank sums its poses' parameter gradients (the first pose writes, the
-    # others add, in order on one stream) and the ranks all-reduce the sum.
-    flat = acc = None
-    if world > 1:
-        flat, acc = flat_gradients(scene.N, scene.K, params.means.device)
+        def step():
+            mv.forward(params, bg)
+            mv.backward(gimg)
 
-    def step_streams():
-        cur = torch.cuda.current_stream()
-        for p, c in enumerate(cams):
-            streams[p].wait_stream(cur)
-            with torch.cuda.stream(streams[p]):
-                Rp[p].forward(params, c, bg, lod, quant)
-                if acc is None:
-                    Rp[p].backward(gimg[p])
-                else:
-                    Rp[p].backward_2d(gimg[p])
-        for st in streams:
-            cur.wait_stream(st)
-        if acc is not None:
-            for p in range(len(cams)):
-                Rp[p].backward_params(acc, accumulate=p > 0)
+        step_graphed = step
+        renderers = mv.views
+        timed = mv
+    else:
+        def step():
+            for p, c in enumerate(cams):
+                R.forward(params, c, bg, lod, quant)
+                R.backward(gimg[p])
+
+        # The poses of a step are independent: each gets its own buffers and
+        # stream, so that one pose's latency-bound bin/sort kernels share the
+        # GPU with another pose's raster kernels (the captured graph holds one
+        # chain per pose). With several ranks each rank sums its poses'
+        # parameter gradients (the first pose writes, the others add, in
+        # order on one stream) and the ranks all-reduce the sum.
+        Rp = [R] + [Rasterizer(scene.N, scene.sh_degree, W, H, capacity=6 * scene.N) for _ in cams[1:]]
+        streams = [torch.cuda.Stream() for _ in cams]
+        acc = None
+        if world > 1:
+            flat, acc = flat_gradient_buffers(scene.N, scene.sh_degree, params.means.device)
+
+        def step_graphed():
+            cur = torch.cuda.current_stream()
+            for p, c in enumerate(cams):
+                streams[p].wait_stream(cur)
+                with torch.cuda.stream(streams[p]):
+                    Rp[p].forward(params, c, bg, lod, quant)
+                    if acc is None:
+                        Rp[p].backward(gimg[p])
+                    else:
+                        Rp[p].backward_2d(gimg[p])
+            for st in streams:
+                cur.wait_stream(st)
+            if acc is not None:
+                for p in range(len(cams)):
+                    Rp[p].backward_params(acc, accumulate=p > 0)
+
+        renderers = Rp
+        timed = R
 
     # warm-up (also settles the instance capacities)
     for _ in range(max(args.warmup, 0)):
         step()
-        step_streams()
+        step_graphed()
         reduce_gradients(flat, world)
     torch.cuda.synchronize()
     # work counts per pose (deterministic; measured outside the timed region)
     counts = []
-    for p, c in enumerate(cams):
-        R.forward(params, c, bg, lod, quant)
-        counts.append(R.work_counts())
+    if use_mv:
+        mv.forward(params, bg)
+        counts = [v.work_counts() for v in mv.views]
+    else:
+        for p, c in enumerate(cams):
+            R.forward(params, c, bg, lod, quant)
+            counts.append(R.work_counts())
     torch.cuda.synchronize()
 
     # ---- timed region: whole steps, device-resident inputs. The bin/sort
     # results (instance counts, statuses) stay on the device (deferred mode),
     # so a whole step has no host round trip and is captured once as a CUDA
-    # graph (every launch and memset of the 4 poses), then replayed K times.
+    # graph (every launch and memset of the step), then replayed K times.
     # The slots of the last replay are checked after the region
     # (Rasterizer.check raises on any failure).
-    for r in Rp:
+    for r in renderers:
         r.deferred = True
         r.check()
     graph = torch.cuda.CUDAGraph()
     l0 = gs.gs_debug_kernel_launches()
     with torch.cuda.graph(graph):
-        step_streams()
+        step_graphed()
     launches_per_step = gs.gs_debug_kernel_launches() - l0
-    slots = [r._n_pending for r in Rp]
+    slots = [r._n_pending for r in renderers]
     graph.replay()  # one more untimed step, through the graph
     reduce_gradients(flat, world)
     torch.cuda.synchronize()
@@ -529,7 +555,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     _barrier(world)
     launches = launches_per_step * args.steps
-    for r, k in zip(Rp, slots):
+    for r, k in zip(renderers, slots):
         r._n_pending = k
         r.check()
     elapsed_ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
@@ -541,7 +567,7 @@ def run_ours(args):
     # ---- the same steps launched one call at a time, with CUDA events
     # around every stage: the per-stage times and the dominant kernel's
     # launch duration for the roofline
-    R.stage_events = {}
+    timed.stage_events = {}
     _barrier(world)
     torch.cuda.synchronize()
     es0, es1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -551,11 +577,12 @@ def run_ours(args):
     es1.record()
     torch.cuda.synchronize()
     _barrier(world)
-    R.check()
+    for r in ([R] if not use_mv else mv.views):
+        r.check()
     stage_loop_ms = _max_over_ranks(es0.elapsed_time(es1), world) / args.steps
-    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in R.stage_events.items()}
-    stage_n = {k: len(v) for k, v in R.stage_events.items()}
-    R.stage_events = None
+    stage_ms = {k: sum(a.elapsed_time(b) for a, b in v) for k, v in timed.stage_events.items()}
+    stage_n = {k: len(v) for k, v in timed.stage_events.items()}
+    timed.stage_events = None
 
     # ---- roofline of the dominant kernel
     peaks = _peaks()
@@ -565,7 +592,8 @@ def run_ours(args):
     Eb = sum(c["E_bwd"] for c in counts)
     per_kernel = {"raster_fwd": OPS_EVAL * E + OPS_BLEND_FWD * B,
                   "raster_bwd": OPS_EVAL * Eb + OPS_BLEND_BWD * B}
-    dom = max(("raster_fwd", "raster_bwd", "preprocess", "preprocess_bwd"), key=lambda k: stage_ms.get(k, 0.0))
+    work = stage_work(scene, counts, multiview=use_mv)
+    dom = max((k for k in work if k != "bin_sort"), key=lambda k: stage_ms.get(k, 0.0))
     avg_ms = stage_ms[dom] / max(stage_n[dom], 1)
     peak_alu = 148 * FP32_LANES_PER_SM * peaks["sm_max_mhz"] * 1e6 / 1e12  # T fp32 op/s
     if dom in per_kernel:
@@ -584,9 +612,8 @@ def run_ours(args):
                          "instructions one ncu capture counted for one launch (FFMA + FADD + FMUL, packed "
                          "FFMA2/FADD2/FMUL2 twice), over the same launch time"}
     else:
-        K = scene.K
-        nbytes = (11 + 3 * K) * 4 * scene.N + 64 * scene.N if dom == "preprocess" else \
-            ((11 + 3 * K) * 4 * 2 + 48 + 64) * scene.N
+        # an HBM-bound per-Gaussian stage: its algorithmic bytes per launch
+        nbytes = work[dom]["bytes"] / max(stage_n[dom] / max(args.steps, 1), 1)
         achieved = nbytes / (avg_ms * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None, "avg_launch_ms": avg_ms}
@@ -604,16 +631,21 @@ def run_ours(args):
             "work_per_step": {"V": sum(c["V"] for c in counts), "I": sum(c["I"] for c in counts),
                               "E": E, "E_bwd": Eb, "B": B},
             "stages_ms_per_step": {k: v / args.steps for k, v in stage_ms.items()},
-            "timing": {"value": "one CUDA graph per step, replayed K times: all launches of the 4 poses, each "
-                                "pose on its own stream and buffers (4 independent chains)" +
-                                ("; with several ranks the graph also sums the poses' parameter gradients and "
-                                 "each replay is followed by their all-reduce" if world > 1 else ""),
-                       "stages": "a second loop of K steps launched call by call, CUDA events around each "
-                                 "stage (the roofline's launch duration)",
+            "timing": {"value": ("one CUDA graph per step, replayed K times: one multi-view preprocess of the "
+                                 f"{len(poses)} poses, then each pose's bin/sort, raster forward and raster "
+                                 "backward on its own stream and buffers, then one multi-view preprocess "
+                                 "backward giving the parameter gradient summed over the poses" if use_mv else
+                                 f"one CUDA graph per step, replayed K times: all launches of the {len(poses)} "
+                                 "poses, each pose on its own stream and buffers (independent chains)" +
+                                 ("; with several ranks the graph also sums the poses' parameter gradients"
+                                  if world > 1 else "")) +
+                                ("; each replay is followed by the all-reduce of the summed gradient"
+                                 if world > 1 else ""),
+                       "stages": "a second loop of K steps launched call by call, the poses one after another "
+                                 "on one stream, CUDA events around each stage (the roofline's launch duration)",
                        "stage_loop_ms_per_step": stage_loop_ms},
             "roofline": roof,
-            "step_roofline": step_roofline(stage_work(scene, counts), stage_ms, ms_per_step, args.steps,
-                                           peaks["hbm_gbs"], peak_alu),
+            "step_roofline": step_roofline(work, stage_ms, ms_per_step, args.steps, peaks["hbm_gbs"], peak_alu),
             "gpu_launches": int(launches), "gpu_launches_per_step": int(launches_per_step),
             "clocks": clocks}
 
@@ -624,7 +656,7 @@ def run_ours(args):
                                                   peak_alu, fwd_ms)
 
     if not args.no_adam:
-        line["adam_sh_quant"] = adam_pass(R, params, peaks)
+        line["adam_sh_quant"] = adam_pass(R, params, peaks, (mv.grads if use_mv else R.grads)["sh"])
 
     if args.multiview and world == 1:
         line["multiview"] = multiview(args, peaks)
@@ -633,7 +665,7 @@ def run_ours(args):
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
-        line["e2e"] = e2e(args, scene, R, gimg, cams, bg, world)
+        line["e2e"] = e2e(args, scene, R, mv, gimg, cams, bg, world)
     if rank == 0 and world == 1 and not args.no_cpu:
         import oracle
         # one whole bench step on the host: every pose, every tile (unless a
@@ -681,14 +713,13 @@ def importance_pass(R, params, cams, bg, ops_per_view, peak_alu, fwd_ms, reps=10
             "views": len(cams), "reps": reps}
 
 
-def adam_pass(R, params, peaks, reps=20):
+def adam_pass(R, params, peaks, d_sh, reps=20):
     """The fused quantised-SH Adam step (gs_adam_sh_quant) on the bench model:
-    45 unit planes x 1M Gaussians, with the last backward's gradients."""
+    45 unit planes x 1M Gaussians, with the step's SH gradient d_sh."""
     import torch
     from differentiable_tile_rasterizer_b200.pipeline import QuantizedSHAdam
     opt = QuantizedSHAdam(R.N, R.sh_degree, lr=1e-3)
     opt.load(params.sh)
-    d_sh = R.grads["sh"]
     for _ in range(3):
         opt.step(d_sh)
     torch.cuda.synchronize()
@@ -871,21 +902,24 @@ def multiview(args, peaks):
                                     "bytes": "(11 + 3K) x 4 read + 64 per view written, per Gaussian"}}
 
 
-def e2e(args, scene, R, gimg, cams, bg, world):
+def e2e(args, scene, R, mv, gimg, cams, bg, world):
     """Same metric with pinned host buffers, through the public API: every step
     copies the parameters and the 4 upstream image gradients in, and the 4
     images and the step's parameter gradients (summed over its poses, the
     optimizer's input) out. Copies run on their own streams, one per
     direction, and the device inputs and outputs are double-buffered, so a
-    step's uploads overlap the previous step's compute and read-back."""
+    step's uploads overlap the previous step's compute and read-back. The
+    step is the bench's: the multi-view pass (mv) when it has one, else a
+    chain per pose."""
     import torch
-    from differentiable_tile_rasterizer_b200.pipeline import GaussianParams
+    from differentiable_tile_rasterizer_b200.pipeline import GaussianParams, flat_gradient_buffers
     host = GaussianParams.empty_like_host(scene)
     host_g = [g.cpu().pin_memory() for g in gimg]
     dev = [GaussianParams.from_scene(scene) for _ in range(2)]
     dg = [[torch.empty_like(g) for g in gimg] for _ in range(2)]
     img = [[torch.empty_like(R.image) for _ in cams] for _ in range(2)]
-    flats, acc = zip(*[flat_gradients(scene.N, scene.K, R.dev) for _ in range(2)])
+    flats, acc = zip(*[flat_gradient_buffers(scene.N, scene.sh_degree, R.dev) for _ in range(2)])
+    checked = mv.views if mv is not None else [R]  # their deferred bin/sort results are read after a loop
     out_img = [torch.empty_like(R.image, device="cpu").pin_memory() for _ in cams]
     out_grads = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in R.grads.items()}
     h2d = sum(t.numel() * t.element_size() for t in host.values()) + sum(
@@ -913,14 +947,20 @@ def e2e(args, scene, R, gimg, cams, bg, world):
             ev_in[b].record(up)
         comp.wait_event(ev_in[b])
         comp.wait_event(ev_out[b])  # step s - 2's outputs in buffer b have been read back
-        for v in acc[b].values():
-            v.zero_()
-        for p, c in enumerate(cams):
-            R.forward(dev[b], c, bg)
-            R.backward(dg[b][p])
-            img[b][p].copy_(R.image)
-            for k, v in R.grads.items():
-                acc[b][k].add_(v)
+        if mv is not None:
+            mv.forward(dev[b], bg)
+            mv.backward(dg[b], into=acc[b])
+            for p, r in enumerate(mv.views):
+                img[b][p].copy_(r.image)
+        else:
+            for v in acc[b].values():
+                v.zero_()
+            for p, c in enumerate(cams):
+                R.forward(dev[b], c, bg)
+                R.backward(dg[b][p])
+                img[b][p].copy_(R.image)
+                for k, v in R.grads.items():
+                    acc[b][k].add_(v)
         reduce_gradients(flats[b], world)
         ev_comp[b].record(comp)
         with torch.cuda.stream(down):
@@ -934,7 +974,8 @@ def e2e(args, scene, R, gimg, cams, bg, world):
     for s in range(max(1, args.warmup)):
         step(s)
     torch.cuda.synchronize()
-    R.check()
+    for r in checked:
+        r.check()
     _barrier(world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(comp)
@@ -943,7 +984,8 @@ def e2e(args, scene, R, gimg, cams, bg, world):
     comp.wait_stream(down)  # the timed region ends after the last read-back
     ev1.record(comp)
     torch.cuda.synchronize()
-    R.check()
+    for r in checked:
+        r.check()
     ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
 
     # the bound: the same copies with no compute, each direction alone and

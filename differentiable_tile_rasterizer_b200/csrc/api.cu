@@ -349,6 +349,29 @@ GS_API int gs_preprocess_bwd(const float* means, const float* log_scales, const 
                                            static_cast<cudaStream_t>(stream)));
 }
 
+GS_API int gs_preprocess_bwd_multiview(const float* means, const float* log_scales, const float* quats,
+                                       const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                                       const gs_camera* cams, int n_views, const gs_projected* ins,
+                                       const float* const* grad2ds, float* d_means, float* d_log_scales,
+                                       float* d_quats, float* d_opacity_logits, float* d_sh, void* stream) {
+  if (sh_degree < 0 || n_views < 1 || n_views > GS_MAX_VIEWS || !cams || !ins || !grad2ds)
+    return GS_ERR_INVALID_ARGUMENT;
+  if (sh_degree > 3) return GS_ERR_UNSUPPORTED;
+  if (!params_ok(means, log_scales, quats, opacity_logits, sh, N)) return GS_ERR_INVALID_ARGUMENT;
+  if (N > 0 && (!d_means || !d_log_scales || !d_quats || !d_opacity_logits || !d_sh)) return GS_ERR_INVALID_ARGUMENT;
+  MultiViewBwdArgs mv;
+  mv.n_views = n_views;
+  for (int v = 0; v < n_views; ++v) {
+    if (!camera_ok(&cams[v]) || !records_ok(&ins[v]) || (N > 0 && !grad2ds[v])) return GS_ERR_INVALID_ARGUMENT;
+    mv.cam[v] = make_devcam(cams[v]);
+    mv.rec[v] = to_records(&ins[v]);
+    mv.grad2d[v] = reinterpret_cast<const float4*>(grad2ds[v]);
+  }
+  Params p{means, log_scales, quats, opacity_logits, sh, N, sh_degree, nullptr, nullptr};
+  Grads g{d_means, d_log_scales, d_quats, d_opacity_logits, d_sh};
+  return cuda_status(launch_preprocess_bwd_multiview(p, mv, g, static_cast<cudaStream_t>(stream)));
+}
+
 GS_API int gs_preprocess_bwd_accumulate(const float* means, const float* log_scales, const float* quats,
                                         const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
                                         const int32_t* active_idx, const int32_t* n_active, const gs_camera* cam,

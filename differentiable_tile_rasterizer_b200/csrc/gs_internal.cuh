@@ -102,6 +102,15 @@ struct MultiViewArgs {
   int n_views;
 };
 cudaError_t launch_preprocess_multiview(const Params& p, const MultiViewArgs& mv, cudaStream_t s);
+struct MultiViewBwdArgs {
+  DevCam cam[kMaxViews];
+  Records rec[kMaxViews];
+  const float4* grad2d[kMaxViews];  // [N][3] per view
+  int n_views;
+};
+// The parameter gradients summed over the views (every row written).
+cudaError_t launch_preprocess_bwd_multiview(const Params& p, const MultiViewBwdArgs& mv, const Grads& g,
+                                            cudaStream_t s);
 
 // stats.cu: norm_sum[g] += |(dpx, dpy)|, view_count[g] += 1 for every
 // visible record of the view (Gaussian g = active_idx[i] or i).

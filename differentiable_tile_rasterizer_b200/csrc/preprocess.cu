@@ -490,6 +490,223 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
     put_grad<kMode>(&gr.d_means[m * N + g], g_mu[m] + g_t[0] * W[m] + g_t[1] * W[3 + m] + g_t[2] * W[6 + m]);
 }
 
+
+// Backward of several views of one model in one pass: the parameter
+// gradients of a loss summed over the views (record i of every view is
+// Gaussian i, no cull, as gs_preprocess_multiview writes them). Each
+// Gaussian's parameters are read once; its view-independent quantities
+// (scales, rotation, Sigma, opacity) are computed once; per view that sees
+// it, the chain to (Sigma, t, colour) runs as in preprocess_bwd_kernel and
+// its gradients with respect to Sigma, the opacity, the mean and the SH
+// coefficients are summed in registers; the chain from Sigma to the scales
+// and the rotation, which is linear in dL/dSigma, then runs once on the sum.
+// Every gradient row is written once (zeros for a Gaussian no view sees).
+// The Gaussian's 3K SH coefficients and their 3K gradient sums live in
+// shared memory ([coefficient][thread]: each thread its own column,
+// conflict-free), the rest in registers.
+constexpr int kMvBwdBlock = 128;
+template <int K>
+__global__ void __launch_bounds__(kMvBwdBlock, 3) preprocess_bwd_multiview_kernel(Params p, MultiViewBwdArgs a,
+                                                                             Grads gr) {
+  __shared__ float s_gsh[3 * K][kMvBwdBlock];
+  __shared__ float s_sh[3 * K][kMvBwdBlock];
+  float* sum_gsh = &s_gsh[0][threadIdx.x];  // coefficient k at sum_gsh[k * kMvBwdBlock]
+  float* shc = &s_sh[0][threadIdx.x];
+  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t N = p.N;
+  if (g >= N) return;
+  bool seen = false;
+  for (int v = 0; v < a.n_views; ++v) seen |= a.rec[v].tiles[g] > 0;
+  if (!seen) {
+    zero_grads(gr, N, K, g);
+    return;
+  }
+  const float mu[3] = {p.means[g], p.means[N + g], p.means[2 * N + g]};
+  const float ls[3] = {p.log_scales[g], p.log_scales[N + g], p.log_scales[2 * N + g]};
+  const float q[4] = {p.quats[g], p.quats[N + g], p.quats[2 * N + g], p.quats[3 * N + g]};
+  const float logit = p.logits[g];
+  // view-independent forward quantities
+  const float s[3] = {exp_spec(ls[0]), exp_spec(ls[1]), exp_spec(ls[2])};
+  const float nq = sqrtf(fmaf(q[3], q[3], fmaf(q[2], q[2], fmaf(q[1], q[1], q[0] * q[0]))));
+  const float inq = 1.0f / nq;
+  const float w = q[0] * inq, x = q[1] * inq, y = q[2] * inq, z = q[3] * inq;
+  float S6[6];  // Sigma = M M^T, upper triangle
+  {
+    const float Rq[9] = {1.f - 2.f * (y * y + z * z), 2.f * (x * y - w * z), 2.f * (x * z + w * y),
+                         2.f * (x * y + w * z), 1.f - 2.f * (x * x + z * z), 2.f * (y * z - w * x),
+                         2.f * (x * z - w * y), 2.f * (y * z + w * x), 1.f - 2.f * (x * x + y * y)};
+    float M[9];
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j) M[3 * i + j] = Rq[3 * i + j] * s[j];
+    int u = 0;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+#pragma unroll
+      for (int j = i; j < 3; ++j)
+        S6[u++] = fmaf(M[3 * i + 2], M[3 * j + 2], fmaf(M[3 * i + 1], M[3 * j + 1], M[3 * i] * M[3 * j]));
+  }
+  // sums over the views
+  // sums over the views; dL/dSigma as its upper triangle (Sigma is symmetric)
+  float sum_gS[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, sum_gmu[3] = {0.f, 0.f, 0.f}, sum_gop = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 3 * K; ++k) {
+    sum_gsh[k * kMvBwdBlock] = 0.0f;
+    shc[k * kMvBwdBlock] = p.sh[(int64_t)k * N + g];
+  }
+#pragma unroll 1
+  for (int v = 0; v < a.n_views; ++v) {
+    if (a.rec[v].tiles[g] <= 0) continue;
+    const DevCam& cam = a.cam[v];
+    const float4* g2d = a.grad2d[v];
+    // colour first (its temporaries die before the geometry's are born)
+    float gmu_dir[3];
+    {
+      const float4 g2 = g2d[3 * g + 2];
+      const float4 colour = a.rec[v].rgb[g];
+      const float dv[3] = {mu[0] - cam.campos[0], mu[1] - cam.campos[1], mu[2] - cam.campos[2]};
+      const float nd = sqrtf(fmaf(dv[2], dv[2], fmaf(dv[1], dv[1], dv[0] * dv[0])));
+      const float ind = 1.0f / nd;
+      const float dir[3] = {dv[0] * ind, dv[1] * ind, dv[2] * ind};
+      float Y[K];
+      sh_basis<K>(dir[0], dir[1], dir[2], Y);
+      const float gv[3] = {colour.x > 0.0f ? g2.x : 0.0f, colour.y > 0.0f ? g2.y : 0.0f,
+                           colour.z > 0.0f ? g2.z : 0.0f};
+      float gdir[3] = {0.f, 0.f, 0.f};
+      float DY[K][3];
+      sh_basis_grad<K>(dir[0], dir[1], dir[2], DY);
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        float gY = 0.0f;
+#pragma unroll
+        for (int ch = 0; ch < 3; ++ch) {
+          sum_gsh[(3 * k + ch) * kMvBwdBlock] += gv[ch] * Y[k];
+          gY = fmaf(gv[ch], shc[(3 * k + ch) * kMvBwdBlock], gY);
+        }
+#pragma unroll
+        for (int m = 0; m < 3; ++m) gdir[m] = fmaf(gY, DY[k][m], gdir[m]);
+      }
+      const float ddot = gdir[0] * dir[0] + gdir[1] * dir[1] + gdir[2] * dir[2];
+#pragma unroll
+      for (int m = 0; m < 3; ++m) gmu_dir[m] = (gdir[m] - ddot * dir[m]) * ind;
+    }
+    // geometry
+    const float4 g0 = g2d[3 * g], g1 = g2d[3 * g + 1];
+    sum_gop += g0.z;
+    const float* W = cam.W;
+    float t[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+      t[r] = fmaf(W[3 * r + 2], mu[2], fmaf(W[3 * r + 1], mu[1], W[3 * r] * mu[0])) + cam.t[r];
+    const float fx = cam.fx, fy = cam.fy, tz = t[2], itz = 1.0f / tz, itz2 = itz * itz;
+    const float J00 = fx * itz, J11 = fy * itz, J02 = -fx * t[0] * itz2, J12 = -fy * t[1] * itz2;
+    float T[6];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      T[j] = fmaf(J02, W[6 + j], J00 * W[j]);
+      T[3 + j] = fmaf(J12, W[6 + j], J11 * W[3 + j]);
+    }
+    // TS = T Sigma, Sigma from its upper triangle S6 = (00, 01, 02, 11, 12, 22)
+    const float Sf[9] = {S6[0], S6[1], S6[2], S6[1], S6[3], S6[4], S6[2], S6[4], S6[5]};
+    float TS[6];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j)
+        TS[3 * i + j] = fmaf(T[3 * i + 2], Sf[6 + j], fmaf(T[3 * i + 1], Sf[3 + j], T[3 * i] * Sf[j]));
+    const float ca = fmaf(TS[2], T[2], fmaf(TS[1], T[1], TS[0] * T[0])) + kDilation;
+    const float cb = fmaf(TS[2], T[5], fmaf(TS[1], T[4], TS[0] * T[3]));
+    const float cc = fmaf(TS[5], T[5], fmaf(TS[4], T[4], TS[3] * T[3])) + kDilation;
+    const float det = fmaf(ca, cc, -cb * cb);
+    const float id = 1.0f / det, id2 = id * id;
+    const float gpx = g0.x, gpy = g0.y, gA = g1.x, gB = g1.y, gC = g1.z;
+    float g_t[3];
+    g_t[0] = gpx * fx * itz;
+    g_t[1] = gpy * fy * itz;
+    g_t[2] = -(gpx * fx * t[0] + gpy * fy * t[1]) * itz2;
+    // conic -> Sigma'
+    const float ga = (-cc * cc * gA + cb * cc * gB - cb * cb * gC) * id2;
+    const float gb = (2.f * cb * cc * gA - (ca * cc + cb * cb) * gB + 2.f * ca * cb * gC) * id2;
+    const float gc = (-cb * cb * gA + ca * cb * gB - ca * ca * gC) * id2;
+    const float Gm[4] = {ga, 0.5f * gb, 0.5f * gb, gc};
+    float GT[6];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j) GT[3 * i + j] = Gm[2 * i] * T[j] + Gm[2 * i + 1] * T[3 + j];
+    // dL/dSigma = T^T Gm T (upper triangle)
+    {
+      int u = 0;
+#pragma unroll
+      for (int i = 0; i < 3; ++i)
+#pragma unroll
+        for (int j = i; j < 3; ++j) sum_gS[u++] += T[i] * GT[j] + T[3 + i] * GT[3 + j];
+    }
+    float gJ00 = 0.f, gJ02 = 0.f, gJ11 = 0.f, gJ12 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const float gT0 = 2.f * (Gm[0] * TS[j] + Gm[1] * TS[3 + j]);
+      const float gT1 = 2.f * (Gm[2] * TS[j] + Gm[3] * TS[3 + j]);
+      gJ00 = fmaf(gT0, W[j], gJ00);
+      gJ02 = fmaf(gT0, W[6 + j], gJ02);
+      gJ11 = fmaf(gT1, W[3 + j], gJ11);
+      gJ12 = fmaf(gT1, W[6 + j], gJ12);
+    }
+    g_t[0] += -fx * itz2 * gJ02;
+    g_t[1] += -fy * itz2 * gJ12;
+    g_t[2] += -(fx * gJ00 + fy * gJ11) * itz2 + 2.f * (fx * t[0] * gJ02 + fy * t[1] * gJ12) * itz2 * itz;
+#pragma unroll
+    for (int m = 0; m < 3; ++m) sum_gmu[m] += gmu_dir[m] + g_t[0] * W[m] + g_t[1] * W[3 + m] + g_t[2] * W[6 + m];
+  }
+  // the view-independent chain, once, on the sums
+  const float op = 1.0f / (1.0f + exp_spec(-logit));
+  gr.d_logits[g] = sum_gop * op * (1.0f - op);
+#pragma unroll
+  for (int k = 0; k < 3 * K; ++k) gr.d_sh[(int64_t)k * N + g] = sum_gsh[k * kMvBwdBlock];
+#pragma unroll
+  for (int m = 0; m < 3; ++m) gr.d_means[m * N + g] = sum_gmu[m];
+  const float Rq[9] = {1.f - 2.f * (y * y + z * z), 2.f * (x * y - w * z), 2.f * (x * z + w * y),
+                       2.f * (x * y + w * z), 1.f - 2.f * (x * x + z * z), 2.f * (y * z - w * x),
+                       2.f * (x * z - w * y), 2.f * (y * z + w * x), 1.f - 2.f * (x * x + y * y)};
+  float M[9];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = 0; j < 3; ++j) M[3 * i + j] = Rq[3 * i + j] * s[j];
+  const float gS[9] = {sum_gS[0], sum_gS[1], sum_gS[2], sum_gS[1], sum_gS[3], sum_gS[4],
+                       sum_gS[2], sum_gS[4], sum_gS[5]};
+  float gM[9];
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      gM[3 * i + j] = 2.f * (gS[3 * i] * M[j] + gS[3 * i + 1] * M[3 + j] + gS[3 * i + 2] * M[6 + j]);
+  float gR[9];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    float gs = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      gs = fmaf(gM[3 * i + j], Rq[3 * i + j], gs);
+      gR[3 * i + j] = gM[3 * i + j] * s[j];
+    }
+    gr.d_log_scales[j * N + g] = gs * s[j];
+  }
+  const float gw = 2.f * (-z * gR[1] + y * gR[2] + z * gR[3] - x * gR[5] - y * gR[6] + x * gR[7]);
+  const float gx = 2.f * (y * gR[1] + z * gR[2] + y * gR[3] - 2.f * x * gR[4] - w * gR[5] + z * gR[6] +
+                          w * gR[7] - 2.f * x * gR[8]);
+  const float gy = 2.f * (-2.f * y * gR[0] + x * gR[1] + w * gR[2] + x * gR[3] + z * gR[5] - w * gR[6] +
+                          z * gR[7] - 2.f * y * gR[8]);
+  const float gz = 2.f * (-2.f * z * gR[0] - w * gR[1] + x * gR[2] + w * gR[3] - 2.f * z * gR[4] + y * gR[5] +
+                          x * gR[6] + y * gR[7]);
+  const float qdot = gw * w + gx * x + gy * y + gz * z;
+  gr.d_quats[g] = (gw - qdot * w) * inq;
+  gr.d_quats[N + g] = (gx - qdot * x) * inq;
+  gr.d_quats[2 * N + g] = (gy - qdot * y) * inq;
+  gr.d_quats[3 * N + g] = (gz - qdot * z) * inq;
+}
+
 }  // namespace
 
 cudaError_t launch_preprocess(const Params& p, const DevCam& cam, const Records& out, cudaStream_t s) {
@@ -551,6 +768,20 @@ cudaError_t launch_preprocess_bwd(const Params& p, const uint8_t* mask, const De
     launch_chain<kPreZeroed>(p, mask, cam, in, grad2d, g, s);
   } else {
     launch_chain<kWriteAll>(p, mask, cam, in, grad2d, g, s);
+  }
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_preprocess_bwd_multiview(const Params& p, const MultiViewBwdArgs& mv, const Grads& g,
+                                            cudaStream_t s) {
+  if (p.N == 0) return cudaSuccess;
+  const unsigned grid = grid_for(p.N, kMvBwdBlock);
+  switch (p.sh_degree) {
+    case 0: preprocess_bwd_multiview_kernel<1><<<grid, kMvBwdBlock, 0, s>>>(p, mv, g); break;
+    case 1: preprocess_bwd_multiview_kernel<4><<<grid, kMvBwdBlock, 0, s>>>(p, mv, g); break;
+    case 2: preprocess_bwd_multiview_kernel<9><<<grid, kMvBwdBlock, 0, s>>>(p, mv, g); break;
+    default: preprocess_bwd_multiview_kernel<16><<<grid, kMvBwdBlock, 0, s>>>(p, mv, g); break;
   }
   count_launches(1);
   return cudaGetLastError();

@@ -28,7 +28,7 @@ EXPORTED = ["gs_version", "gs_status_string", "gs_cull", "gs_preprocess", "gs_pr
             "gs_quant_decode", "gs_adam_sh_quant", "gs_route_ctas", "gs_route_count", "gs_route_pack",
             "gs_merge_received", "gs_unmerge_grad2d", "gs_return_grad2d",
             "gs_rasterize_fwd", "gs_rasterize_fwd_importance", "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd",
-            "gs_preprocess_bwd_accumulate",
+            "gs_preprocess_bwd_accumulate", "gs_preprocess_bwd_multiview",
             "gs_debug_set_stalled_sort_tile", "gs_debug_kernel_launches", "gs_debug_is_checked_build",
             "gs_debug_checked_status", "gs_cull_noalloc"]
 GS_CULL_NOALLOC_MAX_N = 16777216
@@ -115,6 +115,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         L.gs_rasterize_bwd_2d.argtypes = [PPROJ, I64, P, P, P, P, PCAM, P, P, P, P, P, P]
         L.gs_preprocess_bwd_accumulate.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, P, PCAM, PPROJ, P,
                                                    P, P, P, P, P, P]
+        L.gs_preprocess_bwd_multiview.argtypes = [P, P, P, P, P, ctypes.c_int, I64, P, ctypes.c_int, P, P,
+                                                  P, P, P, P, P, P]
         L.gs_cull_noalloc.argtypes = [P, P, I64, PCAM, ctypes.c_float, ctypes.c_float, P, P, P, P]
         L.gs_cull_noalloc.restype = ctypes.c_int
         L.gs_debug_kernel_launches.restype = ctypes.c_int64
@@ -129,7 +131,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
                      "gs_quant_encode", "gs_quant_decode", "gs_adam_sh_quant", "gs_route_count", "gs_route_pack",
                      "gs_merge_received", "gs_unmerge_grad2d", "gs_return_grad2d", "gs_bin_sort_async", "gs_rasterize_fwd",
                      "gs_rasterize_fwd_importance",
-                     "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd", "gs_preprocess_bwd_accumulate"]:
+                     "gs_rasterize_bwd", "gs_rasterize_bwd_2d", "gs_preprocess_bwd", "gs_preprocess_bwd_accumulate",
+                     "gs_preprocess_bwd_multiview"]:
             getattr(L, name).restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -370,6 +373,22 @@ def gs_preprocess_bwd_accumulate(means, log_scales, quats, opacity_logits, sh, s
     _check("gs_preprocess_bwd_accumulate", load().gs_preprocess_bwd_accumulate(
         _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
         _p(active_idx), _p(n_active), ctypes.byref(cam), ctypes.byref(rec), _p(grad2d),
+        _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
+
+
+def gs_preprocess_bwd_multiview(means, log_scales, quats, opacity_logits, sh, sh_degree, N, cams, recs, grad2ds,
+                                d_means, d_log_scales, d_quats, d_opacity_logits, d_sh, stream=None):
+    """cams: list of GsCamera, recs: list of GsProjected, grad2ds: list of
+    [N][12] float32 device tensors (one per view)."""
+    if not len(cams) == len(recs) == len(grad2ds):
+        raise ValueError("one record set and one 2-D gradient per camera")
+    V = len(cams)
+    cam_arr = (GsCamera * max(V, 1))(*cams)
+    rec_arr = (GsProjected * max(V, 1))(*recs)
+    g_arr = (ctypes.c_void_p * max(V, 1))(*[_p(t) for t in grad2ds])
+    _check("gs_preprocess_bwd_multiview", load().gs_preprocess_bwd_multiview(
+        _p(means), _p(log_scales), _p(quats), _p(opacity_logits), _p(sh), int(sh_degree), int(N),
+        ctypes.cast(cam_arr, P), V, ctypes.cast(rec_arr, P), ctypes.cast(g_arr, P),
         _p(d_means), _p(d_log_scales), _p(d_quats), _p(d_opacity_logits), _p(d_sh), _stream(stream)))
 
 

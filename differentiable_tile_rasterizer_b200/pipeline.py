@@ -398,12 +398,28 @@ class Rasterizer:
                 "offsets": self.offsets.cpu().numpy(), "n_instances": I}
 
 
+def flat_gradient_buffers(N: int, sh_degree: int, device):
+    """One flat float32 buffer for a whole parameter gradient and a dict of
+    views of it in the library's SoA shapes (means [3][N], log_scales
+    [3][N], quats [4][N], opacity_logits [N], sh [3K][N])."""
+    K, n = (sh_degree + 1) ** 2, max(int(N), 1)
+    flat = torch.empty((11 + 3 * K) * n, dtype=torch.float32, device=device)
+    views, o = {}, 0
+    for name, rows in (("means", 3), ("log_scales", 3), ("quats", 4), ("opacity_logits", 1), ("sh", 3 * K)):
+        v = flat[o: o + rows * n]
+        views[name] = v if name == "opacity_logits" else v.view(rows, n)
+        o += rows * n
+    return flat, views
+
+
 class MultiViewRenderer:
-    """Forward rendering of several views of one model: one pass over the
+    """Rendering of several views of one model: one pass over the
     parameters projects every Gaussian into all views
     (gs_preprocess_multiview), then each view runs its bin/sort and raster
     forward on its own buffers (a Rasterizer per view). No cull: every
-    Gaussian is projected into every view.
+    Gaussian is projected into every view. backward() gives the parameter
+    gradients of a loss summed over the views, again with one pass over the
+    parameters (gs_preprocess_bwd_multiview).
 
     The views' bin/sorts and raster forwards run on n_streams streams (view
     v on stream v mod n_streams), forked from and joined to the caller's
@@ -424,6 +440,10 @@ class MultiViewRenderer:
         d = torch.device(device or "cuda")
         self.streams = [torch.cuda.Stream(device=d) for _ in range(min(max(int(n_streams), 1), len(self.cams)))]
         self.stage_events = None
+        self.params = None
+        # parameter gradients of the loss summed over the views (backward):
+        # views into one flat buffer, so that one collective can reduce them
+        self.grads_flat, self.grads = flat_gradient_buffers(self.N, self.sh_degree, d)
 
     def _timed(self, stage):
         ev = self.stage_events
@@ -431,6 +451,7 @@ class MultiViewRenderer:
 
     def forward(self, params: GaussianParams, bg=(0.0, 0.0, 0.0)) -> list:
         bg = tuple(float(b) for b in bg)
+        self.params = params
         with self._timed("preprocess_multiview"):
             gs.gs_preprocess_multiview(params.means, params.log_scales, params.quats, params.opacity_logits,
                                        params.sh, params.sh_degree, self.N, self.cams,
@@ -450,6 +471,39 @@ class MultiViewRenderer:
         for st in streams:
             cur.wait_stream(st)
         return [R.image for R in self.views]
+
+    def backward(self, dL_dimages, into: Optional[dict] = None) -> dict:
+        """Parameter gradients of a loss summed over the views of the last
+        forward, given each view's dL/dimage ([3][H][W] float32 on the
+        device): per view the 2-D gradients (gs_rasterize_bwd_2d, on the
+        views' streams, with the forward's hit bytes), then one pass over
+        the parameters that chains and sums them
+        (gs_preprocess_bwd_multiview). Written into `into` (a dict of
+        parameter-shaped float32 tensors) if given, else into self.grads;
+        returns that dict (every row overwritten)."""
+        if len(dL_dimages) != len(self.views):
+            raise ValueError("one image gradient per view")
+        p = self.params
+        if p is None:
+            raise RuntimeError("backward() before forward()")
+        cur = torch.cuda.current_stream()
+        streams = self.streams if self.stage_events is None else self.streams[:1]
+        for st in streams:
+            st.wait_stream(cur)
+        for v, (R, g) in enumerate(zip(self.views, dL_dimages)):
+            with torch.cuda.stream(streams[v % len(streams)]):
+                with self._timed("raster_bwd"):
+                    gs.gs_rasterize_bwd_2d(R._proj, R.N, R.vals, R.ranges, R.cam, R.bg, R.final_T, R.last, g,
+                                           R.grad2d, tile_order=R._order(), hit_bits=R._hits_in())
+        for st in streams:
+            cur.wait_stream(st)
+        a = self.grads if into is None else into
+        with self._timed("preprocess_bwd_multiview"):
+            gs.gs_preprocess_bwd_multiview(p.means, p.log_scales, p.quats, p.opacity_logits, p.sh, p.sh_degree,
+                                           self.N, self.cams, [R._proj for R in self.views],
+                                           [R.grad2d for R in self.views], a["means"], a["log_scales"],
+                                           a["quats"], a["opacity_logits"], a["sh"])
+        return a
 
     def set_deferred(self, on: bool):
         for R in self.views:

@@ -492,6 +492,33 @@ GS_API int gs_preprocess_bwd_accumulate(const float* means, const float* log_sca
                                         float* d_log_scales, float* d_quats, float* d_opacity_logits, float* d_sh,
                                         void* stream);
 
+/* Backward of gs_preprocess_multiview: the parameter gradients of a loss
+ * summed over several views of one model, from each view's per-record 2-D
+ * gradients (gs_rasterize_bwd_2d), in one pass over the parameters. The
+ * gradient of a sum over views is the sum of the views' gradients (the
+ * problem statement's backward pass, applied per view); the pages print no
+ * kernel for it. Record i of every view is Gaussian i, as
+ * gs_preprocess_multiview writes them (no cull).
+ *   params, sh_degree, N   as for gs_preprocess_multiview
+ *   cams     [host] [n_views] the views' cameras
+ *   n_views  1 .. GS_MAX_VIEWS
+ *   ins      [host] [n_views] the views' records (capacity N each)
+ *   grad2ds  [host] [n_views] pointers to each view's [device] [N][12] 2-D
+ *            gradients
+ *   d_*      [device] parameter-shaped gradients out: every row is written
+ *            (zeros for a Gaussian that no view sees)
+ * Per Gaussian the chain from the 3-D covariance to the log-scales and the
+ * quaternion, and from the opacity to its logit, runs once on the summed
+ * dL/dSigma and dL/dopacity (those chains are linear), so the result equals
+ * the sum of gs_preprocess_bwd over the views up to fp32 rounding, not bit
+ * for bit. HBM traffic: (11 + 3K) * 4 bytes read and written once, plus
+ * 52 bytes per (Gaussian, view) of records and 2-D gradients. Asynchronous. */
+GS_API int gs_preprocess_bwd_multiview(const float* means, const float* log_scales, const float* quats,
+                                       const float* opacity_logits, const float* sh, int sh_degree, int64_t N,
+                                       const gs_camera* cams, int n_views, const gs_projected* ins,
+                                       const float* const* grad2ds, float* d_means, float* d_log_scales,
+                                       float* d_quats, float* d_opacity_logits, float* d_sh, void* stream);
+
 /* Number of kernels this library has launched in the process so far (all
  * devices, all streams). Host-side counter, for accounting in benchmarks. */
 GS_API int64_t gs_debug_kernel_launches(void);

@@ -73,3 +73,19 @@ def test_step_roofline_sums_the_binding_bound_of_each_stage():
         assert abs(r["stages"][k]["frac"] - t / 1.0) < 1e-12
     assert abs(r["frac"] - want / 10.0) < 1e-12
     assert r["stages"]["raster_bwd"]["bound"] == "alu" and r["stages"]["preprocess"]["bound"] == "hbm"
+
+
+def test_step_roofline_of_the_multiview_step():
+    # the per-Gaussian stages of a multi-view step read the parameters once
+    from differentiable_tile_rasterizer_b200 import synthetic as S
+    sc = S.random_scene(1000, 160, 96, sh_degree=3, seed=1)
+    c = {"V": 900, "I": 5000, "E": 10 ** 9, "E_bwd": 2 * 10 ** 9, "B": 10 ** 8, "A": 1000, "culled": False}
+    counts = [c, dict(c, V=700)]
+    w = bench.stage_work(sc, counts, multiview=True)
+    par = 236
+    assert "preprocess" not in w and "preprocess_bwd" not in w
+    assert w["preprocess_multiview"]["bytes"] == 1000 * (par + 64 * 2)
+    assert w["preprocess_bwd_multiview"]["bytes"] == 2 * 1000 * par + (4 * 1000 + 64 * 900) + (4 * 1000 + 64 * 700)
+    single = bench.stage_work(sc, counts)
+    for k in ("bin_sort", "raster_fwd", "raster_bwd"):
+        assert w[k] == single[k]

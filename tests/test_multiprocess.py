@@ -123,11 +123,12 @@ def _reduce_main(rank, world, port, out):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     import bench
+    from differentiable_tile_rasterizer_b200.pipeline import flat_gradient_buffers
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        N, K = 5, 16
-        flat, views = bench.flat_gradients(N, K, "cpu")
+        N, sh_degree = 5, 3
+        flat, views = flat_gradient_buffers(N, sh_degree, "cpu")
         flat.copy_(torch.arange(flat.numel(), dtype=torch.float32) * (rank + 1))
         views["sh"][2, 3] += 100.0 * rank  # writes through the views land in the flat buffer
         bench.reduce_gradients(flat, world)

@@ -246,13 +246,41 @@ __global__ void __launch_bounds__(256) preprocess_kernel(Params p, DevCam cam, R
 }
 
 // Several views in one pass: each Gaussian's 11 + 3K parameters are read from
-// HBM once, into registers, and projected into every view.
+// HBM once and projected into every view. The 11 geometric parameters stay
+// in registers, the 3K SH coefficients in shared memory (a column per
+// thread, conflict-free), read through a volatile pointer where they are
+// used so that the compiler does not hoist them into registers across the
+// view loop: 64 registers, 4 CTAs per SM.
+constexpr int kMvBlock = 256;
 template <int K>
-__global__ void __launch_bounds__(256) preprocess_multiview_kernel(Params p, MultiViewArgs mv) {
+struct StagedSource {
+  float m[3], l[3], q[4], lg;
+  const volatile float* c;  // the thread's column: plane k at c[k * kMvBlock] (volatile: read where used)
+  __device__ __forceinline__ void load(const Params& p, int64_t g, float* column) {
+#pragma unroll
+    for (int r = 0; r < 3; ++r) m[r] = p.means[r * p.N + g];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) l[r] = p.log_scales[r * p.N + g];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) q[r] = p.quats[r * p.N + g];
+    lg = p.logits[g];
+#pragma unroll
+    for (int k = 0; k < 3 * K; ++k) column[k * kMvBlock] = p.sh[(int64_t)k * p.N + g];
+    c = column;
+  }
+  __device__ __forceinline__ float mean(int r) const { return m[r]; }
+  __device__ __forceinline__ float log_scale(int r) const { return l[r]; }
+  __device__ __forceinline__ float quat(int r) const { return q[r]; }
+  __device__ __forceinline__ float logit() const { return lg; }
+  __device__ __forceinline__ float sh(int plane) const { return c[plane * kMvBlock]; }
+};
+template <int K>
+__global__ void __launch_bounds__(kMvBlock, 4) preprocess_multiview_kernel(Params p, MultiViewArgs mv) {
+  __shared__ float s_sh[3 * K][kMvBlock];
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= p.N) return;
-  RegisterSource<K> src;
-  src.load(p, i);
+  StagedSource<K> src;
+  src.load(p, i, &s_sh[0][threadIdx.x]);
   for (int v = 0; v < mv.n_views; ++v) {
     Proj o;
     project<K>(src, mv.cam[v], o);
@@ -503,15 +531,18 @@ __global__ void __launch_bounds__(256) preprocess_bwd_kernel(Params p, const uin
 // Every gradient row is written once (zeros for a Gaussian no view sees).
 // The Gaussian's 3K SH coefficients and their 3K gradient sums live in
 // shared memory ([coefficient][thread]: each thread its own column,
-// conflict-free), the rest in registers.
-constexpr int kMvBwdBlock = 128;
+// conflict-free), the rest in registers: 96 registers and 24 KB per CTA of
+// 64 threads, 9 CTAs (18 warps) per SM.
+constexpr int kMvBwdBlock = 64;
 template <int K>
-__global__ void __launch_bounds__(kMvBwdBlock, 3) preprocess_bwd_multiview_kernel(Params p, MultiViewBwdArgs a,
+__global__ void __launch_bounds__(kMvBwdBlock, 9) preprocess_bwd_multiview_kernel(Params p, MultiViewBwdArgs a,
                                                                              Grads gr) {
   __shared__ float s_gsh[3 * K][kMvBwdBlock];
   __shared__ float s_sh[3 * K][kMvBwdBlock];
-  float* sum_gsh = &s_gsh[0][threadIdx.x];  // coefficient k at sum_gsh[k * kMvBwdBlock]
-  float* shc = &s_sh[0][threadIdx.x];
+  // coefficient k at [k * kMvBwdBlock]; volatile: each use reads shared memory
+  // instead of a register copy hoisted out of the view loop
+  volatile float* sum_gsh = &s_gsh[0][threadIdx.x];
+  volatile float* shc = &s_sh[0][threadIdx.x];
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t N = p.N;
   if (g >= N) return;
@@ -724,12 +755,12 @@ cudaError_t launch_preprocess(const Params& p, const DevCam& cam, const Records&
 
 cudaError_t launch_preprocess_multiview(const Params& p, const MultiViewArgs& mv, cudaStream_t s) {
   if (p.N == 0 || mv.n_views == 0) return cudaSuccess;
-  const unsigned grid = grid_for(p.N, 256);
+  const unsigned grid = grid_for(p.N, kMvBlock);
   switch (p.sh_degree) {
-    case 0: preprocess_multiview_kernel<1><<<grid, 256, 0, s>>>(p, mv); break;
-    case 1: preprocess_multiview_kernel<4><<<grid, 256, 0, s>>>(p, mv); break;
-    case 2: preprocess_multiview_kernel<9><<<grid, 256, 0, s>>>(p, mv); break;
-    default: preprocess_multiview_kernel<16><<<grid, 256, 0, s>>>(p, mv); break;
+    case 0: preprocess_multiview_kernel<1><<<grid, kMvBlock, 0, s>>>(p, mv); break;
+    case 1: preprocess_multiview_kernel<4><<<grid, kMvBlock, 0, s>>>(p, mv); break;
+    case 2: preprocess_multiview_kernel<9><<<grid, kMvBlock, 0, s>>>(p, mv); break;
+    default: preprocess_multiview_kernel<16><<<grid, kMvBlock, 0, s>>>(p, mv); break;
   }
   count_launches(1);
   return cudaGetLastError();

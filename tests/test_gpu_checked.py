@@ -19,7 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_core_parity_under_the_checked_build():
     env = dict(os.environ, GS_CHECKED="1")
     files = ["tests/test_gpu_parity.py", "tests/test_gpu_binning.py", "tests/test_gpu_hit_bits.py",
-             "tests/test_gpu_async.py"]
+             "tests/test_gpu_async.py", "tests/test_gpu_multiview.py"]
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-s", *files], cwd=ROOT, env=env,
                        capture_output=True, text=True, timeout=1200)
     tail = r.stdout[-4000:] + r.stderr[-2000:]

@@ -421,11 +421,12 @@ class MultiViewRenderer:
     gradients of a loss summed over the views, again with one pass over the
     parameters (gs_preprocess_bwd_multiview).
 
-    The views' bin/sorts and raster forwards run on n_streams streams (view
-    v on stream v mod n_streams), forked from and joined to the caller's
-    stream, so that one view's latency-bound sort kernels overlap another
-    view's compositing. With deferred mode on (set_deferred) no call waits
-    on the host; otherwise each bin/sort waits for its own stream only.
+    The views' bin/sorts, raster forwards and raster backwards run on
+    n_streams streams (view v on stream v mod n_streams), forked from and
+    joined to the caller's stream, so that the views' latency-bound sort
+    kernels run beside one another (and beside other views' raster kernels
+    where the SMs have room). With deferred mode on (set_deferred) no call
+    waits on the host; otherwise each bin/sort waits for its own stream only.
     While stage timing is on (stage_events not None) the views run one after
     another on one stream, so that each stage's events bracket its own work."""
 

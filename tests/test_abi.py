@@ -64,6 +64,23 @@ def test_tile_order_argument_checks_need_no_gpu():
     assert L.gs_tile_order(None, 1 << 31, None, None) == gs.GS_ERR_INVALID_ARGUMENT
 
 
+def test_multiview_backward_argument_checks_need_no_gpu():
+    L = gs.load()
+    cams = (gs.GsCamera * 17)()
+    recs = (gs.GsProjected * 17)()
+    g2d = (ctypes.c_void_p * 17)()
+    args = lambda deg, nv: (None, None, None, None, None, deg, 0, ctypes.cast(cams, ctypes.c_void_p), nv,
+                            ctypes.cast(recs, ctypes.c_void_p), ctypes.cast(g2d, ctypes.c_void_p),
+                            None, None, None, None, None, None)
+    assert L.gs_preprocess_bwd_multiview(*args(3, 0)) == gs.GS_ERR_INVALID_ARGUMENT   # no view
+    assert L.gs_preprocess_bwd_multiview(*args(3, 17)) == gs.GS_ERR_INVALID_ARGUMENT  # past GS_MAX_VIEWS
+    assert L.gs_preprocess_bwd_multiview(*args(-1, 2)) == gs.GS_ERR_INVALID_ARGUMENT
+    assert L.gs_preprocess_bwd_multiview(*args(4, 2)) == gs.GS_ERR_UNSUPPORTED       # SH degree > 3
+    with pytest.raises(ValueError):  # one record set and one 2-D gradient per camera, checked first
+        gs.gs_preprocess_bwd_multiview(None, None, None, None, None, 3, 0, [gs.GsCamera()], [], [],
+                                       None, None, None, None, None)
+
+
 @pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++17")])
 def test_header_is_plain_c_and_cxx(lang, std):
     # the boundary is a C ABI: the header compiles as strict C99 and as C++
